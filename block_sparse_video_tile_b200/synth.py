@@ -1,0 +1,102 @@
+"""Seeded synthetic inputs for 3-D block-sparse video attention.
+
+This module only draws numbers.  It holds none of the attention arithmetic
+(no tiling, pooling, scoring, selection or softmax), so both the CUDA path and
+the CPU oracle can take their inputs from it without sharing any of the
+method.
+
+Layout of every tensor it returns: ``[B, H, N, d]`` with the token index
+``n = (t * Hh + y) * W + x`` (raster order over the post-patch latent grid
+``(T, Hh, W)``), as ``uint16`` arrays holding bfloat16 bit patterns.
+
+Two input families, matching the workloads the FastVideo VSA user guide and the
+fastbsa page describe (video DiT attention over a latent grid):
+
+* ``normal``:  Q, K, V i.i.d. N(0, 1), drawn in that order from one
+  ``numpy.random.Generator(PCG64(seed))`` stream as float32, then rounded to
+  bfloat16 (round to nearest even).
+* ``field``:   Q and K share, per (batch, head, channel), a smooth
+  low-frequency field over (t, y, x) -- a sum of 8 sinusoids with amplitude
+  0.5, frequencies U(0, 1.5) cycles per grid extent on each axis and phase
+  U(0, 2*pi) -- plus independent 0.5 * N(0, 1) noise each; V is N(0, 1).
+  Neighbouring tiles therefore have related content, so tile selection is
+  structured the way it is on real video latents.  Draw order: field
+  parameters for all (b, h, c), then Q noise, then K noise, then V.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = ["f32_to_bf16_bits", "bf16_bits_to_f32", "make_qkv", "N_SINUSOIDS"]
+
+N_SINUSOIDS = 8
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to bfloat16 (nearest, ties to even); return the bits."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    rounding = np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))
+    return ((u + rounding) >> np.uint32(16)).astype(np.uint16)
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """Widen bfloat16 bit patterns to float32 (exact)."""
+    return (bits.astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def _field(rng: np.random.Generator, B: int, H: int, grid: tuple, d: int) -> np.ndarray:
+    """Sum-of-sinusoids field, float32 ``[B, H, N, d]``.
+
+    Each sinusoid is sin(2*pi*(ft*t/T + fy*y/Hh + fx*x/W) + phi).  It is built
+    as Im(e^{i phi} e^{i 2 pi ft t/T} * e^{i 2 pi (fy y/Hh + fx x/W)}), so the
+    grid-sized product is a batched complex matrix product with an inner
+    dimension of 8 (one term per sinusoid).
+    """
+    T, Hh, W = grid
+    S = N_SINUSOIDS
+    freq = rng.uniform(0.0, 1.5, size=(B, H, d, S, 3))
+    phase = rng.uniform(0.0, 2.0 * np.pi, size=(B, H, d, S))
+    amp = 0.5
+    t = np.arange(T) / T
+    y = np.arange(Hh) / Hh
+    x = np.arange(W) / W
+    out = np.empty((B, H, T * Hh * W, d), dtype=np.float32)
+    for b in range(B):
+        for h in range(H):
+            f = freq[b, h]                                            # [d, S, 3]
+            ph = phase[b, h]                                          # [d, S]
+            et = np.exp(2j * np.pi * f[:, :, 0, None] * t)            # [d, S, T]
+            et = et * (amp * np.exp(1j * ph))[:, :, None]
+            ey = np.exp(2j * np.pi * f[:, :, 1, None] * y)            # [d, S, Hh]
+            ex = np.exp(2j * np.pi * f[:, :, 2, None] * x)            # [d, S, W]
+            eyx = (ey[:, :, :, None] * ex[:, :, None, :]).reshape(d, S, Hh * W)
+            # [d, T, S] @ [d, S, Hh*W] -> [d, T, Hh*W]
+            prod = np.matmul(et.transpose(0, 2, 1).astype(np.complex64),
+                             eyx.astype(np.complex64))
+            out[b, h] = prod.imag.reshape(d, T * Hh * W).T
+    return out
+
+
+def make_qkv(B: int, H: int, grid: tuple, d: int, seed: int = 0,
+             kind: str = "normal"):
+    """Return (q, k, v) as uint16 bfloat16-bit arrays of shape [B, H, N, d]."""
+    T, Hh, W = grid
+    N = T * Hh * W
+    rng = np.random.Generator(np.random.PCG64(seed))
+    shape = (B, H, N, d)
+    if kind == "normal":
+        q = rng.standard_normal(shape, dtype=np.float32)
+        q = f32_to_bf16_bits(q)
+        k = f32_to_bf16_bits(rng.standard_normal(shape, dtype=np.float32))
+        v = f32_to_bf16_bits(rng.standard_normal(shape, dtype=np.float32))
+        return q, k, v
+    if kind == "field":
+        fld = _field(rng, B, H, grid, d)
+        q = fld + np.float32(0.5) * rng.standard_normal(shape, dtype=np.float32)
+        q = f32_to_bf16_bits(q)
+        k = fld + np.float32(0.5) * rng.standard_normal(shape, dtype=np.float32)
+        del fld
+        k = f32_to_bf16_bits(k)
+        v = f32_to_bf16_bits(rng.standard_normal(shape, dtype=np.float32))
+        return q, k, v
+    raise ValueError(f"unknown input kind {kind!r}")

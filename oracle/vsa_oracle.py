@@ -1,0 +1,197 @@
+"""Plain float64 CPU oracle for VSA-style 3-D block-sparse attention.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import this module:
+only the tests, the package's smoke check and the benchmark's CPU-baseline leg
+call it.  It shares no code with the CUDA library (its own geometry, its own
+pooling, scoring, selection and softmax), and takes its inputs as bfloat16 bit
+patterns widened exactly to float64.
+
+What it computes, and where the pages fix each step:
+
+1. Tiling (FastVideo VSA user guide, intro and "Wan top-k behavior"): the
+   post-patch latent grid (T, Hh, W) is cut into spatio-temporal blocks of
+   (tt, th, tw) tokens; the number of blocks per axis is the ceiling of
+   extent / block, so edge blocks are partial -- the guide's routing log gives
+   (31, 22, 40) with (4, 8, 8) blocks -> num_blocks = 120 = 8 * 3 * 5.
+   Blocks are numbered in raster order over block coordinates (t-major, then
+   y, then x), the same order as tokens.
+2. Scoring (guide intro: "for every query block, VSA scores the key/value
+   blocks"): each block is summarised by the mean of its Q rows (resp. K rows)
+   over its valid tokens; the score of (query block i, key block j) is the dot
+   product of the two means.  Reading: mean over valid tokens only (a partial
+   block divides by its own token count), and no scale factor (a positive
+   scale changes neither the order nor the relative gaps).
+3. Selection (guide "Wan top-k behavior": top-k counts key/value blocks per
+   query block, 0 < topk <= num_blocks): keep the topk largest scores; equal
+   scores are broken by the lower block index; the kept list is stored in
+   ascending block order.
+4. Attention (guide intro and "Verify routing and fallback": non-causal
+   self-attention, no mask, scale head_size ** -0.5 by default): for every
+   token of query block i, exact softmax attention over the tokens of the kept
+   blocks; LSE is the natural log of the softmax denominator.
+5. Dense reference (fastbsa page, "How it works": outputs are validated
+   against dense attention): plain softmax attention over all N tokens, with no
+   tiles at all.  With topk == num_blocks (all blocks kept) step 4 equals it.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+NEAR_TIE_REL = 1e-4      # relative k-th / (k+1)-th score gap that counts as a near-tie
+EPS_ROW_REL = 1e-6       # guards the relative gap when both scores are ~0
+
+
+# ---------------------------------------------------------------- conversions
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Widen bfloat16 bit patterns (uint16) exactly to float64."""
+    u32 = bits.astype(np.uint32) << np.uint32(16)
+    return u32.view(np.float32).astype(np.float64)
+
+
+# ------------------------------------------------------------------- geometry
+def tiles_per_axis(grid, tile):
+    """Blocks per axis: ceil(extent / block extent)."""
+    return tuple(-(-g // t) for g, t in zip(grid, tile))
+
+
+def num_tiles(grid, tile) -> int:
+    nt, nh, nw = tiles_per_axis(grid, tile)
+    return nt * nh * nw
+
+
+def tile_tokens(grid, tile):
+    """Raster token indices of every block, in block raster order.
+
+    Returns a list of 1-D int64 arrays; list entry j holds the tokens
+    n = (t * Hh + y) * W + x of block j, in raster order inside the block.
+    """
+    T, Hh, W = grid
+    tt, th, tw = tile
+    nt, nh, nw = tiles_per_axis(grid, tile)
+    out = []
+    for bt in range(nt):
+        ts = np.arange(bt * tt, min(T, (bt + 1) * tt))
+        for bh in range(nh):
+            ys = np.arange(bh * th, min(Hh, (bh + 1) * th))
+            for bw in range(nw):
+                xs = np.arange(bw * tw, min(W, (bw + 1) * tw))
+                n = (ts[:, None, None] * Hh + ys[None, :, None]) * W + xs[None, None, :]
+                out.append(n.reshape(-1).astype(np.int64))
+    return out
+
+
+# -------------------------------------------------------------------- scoring
+def pool(X: np.ndarray, grid, tile) -> np.ndarray:
+    """Per-block mean of the rows of X ([N, d] float64) over valid tokens."""
+    return np.stack([X[tok].mean(axis=0) for tok in tile_tokens(grid, tile)])
+
+
+def tile_scores(qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
+    """s[i, j] = qbar_i . kbar_j (float64)."""
+    return qbar @ kbar.T
+
+
+def topk_row(s_row: np.ndarray, topk: int) -> np.ndarray:
+    """The topk largest entries of one score row, ties -> lower index, ascending."""
+    order = np.lexsort((np.arange(s_row.shape[0]), -s_row))   # by (-s, j)
+    return np.sort(order[:topk])
+
+
+def tie_gap(s_row: np.ndarray, topk: int):
+    """(relative gap, absolute band delta) between the k-th and (k+1)-th scores.
+
+    Returns (inf, 0) when topk == number of blocks (nothing is left out).
+    """
+    nT = s_row.shape[0]
+    if topk >= nT:
+        return math.inf, 0.0
+    srt = np.sort(s_row)[::-1]
+    a, b = srt[topk - 1], srt[topk]
+    denom = max(abs(a), abs(b), EPS_ROW_REL * float(np.max(np.abs(s_row))))
+    if denom == 0.0:
+        return 0.0, 0.0
+    return abs(a - b) / denom, NEAR_TIE_REL * denom
+
+
+def select_head(Q: np.ndarray, K: np.ndarray, grid, tile, topk: int):
+    """One head: (idx [nT, topk] int32 ascending, scores [nT, nT], near_tie [nT] bool)."""
+    nT = num_tiles(grid, tile)
+    if not 0 < topk <= nT:
+        raise ValueError(f"topk must be in [1, {nT}], got {topk}")
+    s = tile_scores(pool(Q, grid, tile), pool(K, grid, tile))
+    idx = np.stack([topk_row(s[i], topk) for i in range(nT)]).astype(np.int32)
+    near = np.array([tie_gap(s[i], topk)[0] < NEAR_TIE_REL for i in range(nT)])
+    return idx, s, near
+
+
+def select(q_bits, k_bits, grid, tile, topk: int):
+    """All (b, h): idx [B, H, nT, topk], scores [B, H, nT, nT], near_tie [B, H, nT]."""
+    B, H = q_bits.shape[:2]
+    nT = num_tiles(grid, tile)
+    idx = np.empty((B, H, nT, topk), np.int32)
+    sc = np.empty((B, H, nT, nT), np.float64)
+    near = np.empty((B, H, nT), bool)
+    for b in range(B):
+        for h in range(H):
+            idx[b, h], sc[b, h], near[b, h] = select_head(
+                bf16_to_f64(q_bits[b, h]), bf16_to_f64(k_bits[b, h]), grid, tile, topk)
+    return idx, sc, near
+
+
+def selection_is_valid(gpu_row: np.ndarray, s_row: np.ndarray, topk: int) -> bool:
+    """Is a selection other than the oracle's still correct under a near-tie?
+
+    It is when it has topk distinct ascending entries and every block in the
+    symmetric difference with the oracle's list scores inside the band
+    [s_(k+1) - delta, s_(k) + delta] around the cut.
+    """
+    nT = s_row.shape[0]
+    g = np.asarray(gpu_row)
+    if g.shape != (topk,) or np.any(g < 0) or np.any(g >= nT) or np.any(np.diff(g) <= 0):
+        return False
+    ref = topk_row(s_row, topk)
+    diff = np.setxor1d(ref, g)
+    if diff.size == 0:
+        return True
+    rel, delta = tie_gap(s_row, topk)
+    if rel >= NEAR_TIE_REL:
+        return False
+    srt = np.sort(s_row)[::-1]
+    lo, hi = srt[topk] - delta, srt[topk - 1] + delta
+    return bool(np.all((s_row[diff] >= lo) & (s_row[diff] <= hi)))
+
+
+# ------------------------------------------------------------------ attention
+def attend_head(Q, K, V, grid, tile, idx, scale: float, query_tiles=None):
+    """Block-sparse exact attention for one head.
+
+    Q, K, V: [N, d] float64.  idx: [nT, topk] kept blocks per query block.
+    Returns O [N, d] and LSE [N]; rows of query blocks not in ``query_tiles``
+    (default: all) are NaN.
+    """
+    toks = tile_tokens(grid, tile)
+    N, d = Q.shape
+    O = np.full((N, V.shape[1]), np.nan)
+    L = np.full(N, np.nan)
+    tiles = range(len(toks)) if query_tiles is None else query_tiles
+    for i in tiles:
+        rows = toks[i]
+        keys = np.concatenate([toks[j] for j in idx[i]])
+        z = scale * (Q[rows] @ K[keys].T)
+        m = z.max(axis=1, keepdims=True)
+        e = np.exp(z - m)
+        l = e.sum(axis=1, keepdims=True)
+        O[rows] = (e @ V[keys]) / l
+        L[rows] = (m + np.log(l))[:, 0]
+    return O, L
+
+
+def dense_bruteforce(Q, K, V, scale: float):
+    """Dense softmax attention over all N tokens (no tiles): O [N, d], LSE [N]."""
+    z = scale * (Q @ K.T)
+    m = z.max(axis=1, keepdims=True)
+    e = np.exp(z - m)
+    l = e.sum(axis=1, keepdims=True)
+    return (e @ V) / l, (m + np.log(l))[:, 0]

@@ -1,0 +1,72 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that a pin fails.
+
+Each case swaps one oracle function for a subtly wrong version -- the kind of
+slip a restatement of the method could make -- and runs the pin that should
+catch it.  A pin that still passed would not be pinning anything.
+"""
+import numpy as np
+import pytest
+
+from oracle import vsa_oracle as vo
+import tests.test_oracle_pins as pins
+
+
+def _zero_padded_pool(X, grid, tile):
+    vol = tile[0] * tile[1] * tile[2]
+    return np.stack([X[t].sum(axis=0) / vol for t in vo.tile_tokens(grid, tile)])
+
+
+def _transposed_scores(qbar, kbar):
+    return kbar @ qbar.T
+
+
+def _ties_to_higher(s_row, topk):
+    order = np.lexsort((-np.arange(s_row.shape[0]), -s_row))
+    return np.sort(order[:topk])
+
+
+_orig_attend = vo.attend_head
+
+
+def _drop_last_kept(Q, K, V, grid, tile, idx, scale, query_tiles=None):
+    return _orig_attend(Q, K, V, grid, tile, idx[:, :-1], scale, query_tiles)
+
+
+def _dense_no_scale(Q, K, V, scale):
+    z = Q @ K.T
+    m = z.max(axis=1, keepdims=True)
+    e = np.exp(z - m)
+    l = e.sum(axis=1, keepdims=True)
+    return (e @ V) / l, (m + np.log(l))[:, 0]
+
+
+def _attend_log2_lse(Q, K, V, grid, tile, idx, scale, query_tiles=None):
+    O, L = _orig_attend(Q, K, V, grid, tile, idx, scale, query_tiles)
+    return O, L / np.log(2.0)
+
+
+_orig_tokens = vo.tile_tokens
+
+
+def _floor_tiles(grid, tile):
+    return [t for t in _orig_tokens(grid, tile) if t.size == tile[0] * tile[1] * tile[2]]
+
+
+CASES = [
+    ("pool", _zero_padded_pool, lambda: pins.test_pool_constant_per_block_partial_edges()),
+    ("tile_scores", _transposed_scores, lambda: pins.test_scores_hand_example()),
+    ("topk_row", _ties_to_higher, lambda: pins.test_ties_go_to_lower_index()),
+    ("attend_head", _drop_last_kept,
+     lambda: pins.test_all_blocks_equals_dense((5, 6, 7), (4, 4, 4))),
+    ("dense_bruteforce", _dense_no_scale, lambda: pins.test_dense_vs_library_sdpa()),
+    ("attend_head", _attend_log2_lse, lambda: pins.test_lse_normalises_weights()),
+    ("tile_tokens", _floor_tiles, lambda: pins.test_block_token_counts(
+        pins.WAN5B, {256: 70, 192: 45, 144: 5})),
+]
+
+
+@pytest.mark.parametrize("name,bad,pin", CASES, ids=[f"{c[0]}:{c[1].__name__}" for c in CASES])
+def test_pin_catches_planted_mistake(monkeypatch, name, bad, pin):
+    monkeypatch.setattr(vo, name, bad)
+    with pytest.raises((AssertionError, ValueError, IndexError)):
+        pin()
