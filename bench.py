@@ -1,0 +1,386 @@
+#!/usr/bin/env python
+"""Benchmark: VSA-style block-sparse attention forward (select + attend).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload wan5b]
+                    [--impl ours|reference] [--no-cpu-baseline]
+
+A step is one pass of the whole hot path over one batch: tile selection
+(mean-pool Q and K per tile, score every tile pair, keep the top-k) and the
+block-sparse attention forward, on the Wan2.2-5B latent shape by default
+(B=1, 24 heads x 128, grid (31, 22, 40), 4x8x8 tiles -> 120, topk 64).
+Inputs (Q, K, V: 3 x 167.6 MB bf16) are resident in HBM and larger than L2,
+so no L2 flush is needed between steps.
+
+value = effective TFLOP/s of the step, counting the exact attention FLOPs
+4 * d * sum_{b,h,i} c_i * sum_{j kept} c_j over valid tokens (c = token count
+of a tile), summed over all ranks, over the max-over-ranks device time.
+With N > 1 (torchrun), every rank runs its own replica of the workload (the
+path shards by (batch, head) with no exchange): weak scaling.
+
+--impl reference times the float64 CPU oracle on a bounded sample of the same
+workload (the only other place this script runs the oracle, besides the
+cpu_baseline field of the default run).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+import torch.distributed as dist
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_video_tile_b200 import api  # noqa: E402
+from block_sparse_video_tile_b200.workloads import ALL  # noqa: E402
+
+METRIC = "block-sparse attn fwd ms/call & effective TFLOP/s (select+attend) at Wan shape"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ helpers
+def tile_counts(w) -> np.ndarray:
+    """Valid token count of every tile (raster tile order)."""
+    (T, Hh, W), (tt, th, tw) = w.grid, w.tile
+    ct = np.minimum(tt, T - np.arange(0, T, tt))
+    cy = np.minimum(th, Hh - np.arange(0, Hh, th))
+    cx = np.minimum(tw, W - np.arange(0, W, tw))
+    return (ct[:, None, None] * cy[None, :, None] * cx[None, None, :]).reshape(-1).astype(np.int64)
+
+
+def exact_flops(idx: np.ndarray, w) -> float:
+    c = tile_counts(w)
+    kept = c[idx].sum(axis=-1)                      # [B, H, nT] kept key tokens per query tile
+    return float(4 * w.d * (kept * c[None, None, :]).sum())
+
+
+def nominal_flops(w) -> float:
+    vol = w.tile[0] * w.tile[1] * w.tile[2]
+    return float(4 * w.B * w.H * w.N * w.topk * vol * w.d)
+
+
+def select_bytes(w) -> float:
+    nT = len(tile_counts(w))
+    return float(2 * w.B * w.H * w.N * w.d * 2 + w.B * w.H * nT * w.topk * 4)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("attn_kernel.cuh", "vsa_ptx.cuh", "vsa_geometry.cuh", "select_kernels.cuh"):
+        with open(os.path.join(ROOT, "block_sparse_video_tile_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    e = rec.get(kernel, {}).get(workload)
+    if not e or e.get("source_sha") != kernel_source_sha():
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons during a region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            sel = str(device)
+        self.sel = sel
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.sel, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            out, _ = self.proc.communicate(timeout=10)
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[3:]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for n, v in zip(names, r[3][1:]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "samples": len(rows), "reasons": sorted(reasons)}
+
+
+def make_inputs(w, device, seed):
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    shape = (w.B, w.H, w.N, w.d)
+    return [torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+            for _ in range(3)]
+
+
+# ---------------------------------------------------------------- oracle arm
+def oracle_sample(q_bits, k_bits, v_bits, w, n_tiles):
+    """Time the float64 oracle on one head: full selection, then attention for
+    the first n_tiles query tiles.  Returns (seconds, exact FLOPs of the sample)."""
+    from oracle import vsa_oracle as vo
+    t0 = time.perf_counter()
+    Q, K, V = (vo.bf16_to_f64(x) for x in (q_bits, k_bits, v_bits))
+    idx, _, _ = vo.select_head(Q, K, w.grid, w.tile, w.topk)
+    vo.attend_head(Q, K, V, w.grid, w.tile, idx, w.d ** -0.5, query_tiles=range(n_tiles))
+    dt = time.perf_counter() - t0
+    c = tile_counts(w)
+    fl = float(4 * w.d * sum(c[i] * c[idx[i]].sum() for i in range(n_tiles)))
+    return dt, fl
+
+
+def head_bits(x: torch.Tensor, b=0, h=0) -> np.ndarray:
+    return x[b, h].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return None
+    torch.manual_seed(0)
+    shape = (w.N, w.d)
+    g = torch.Generator().manual_seed(0)
+    qkv = [torch.randn(shape, generator=g).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+           for _ in range(3)]
+    n_tiles = max(1, len(tile_counts(w)) // 8)
+    for _ in range(args.warmup):
+        oracle_sample(*qkv, w, 1)
+    secs, flops = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, fl = oracle_sample(*qkv, w, n_tiles)
+        secs += dt
+        flops += fl
+    value = flops / secs / 1e12
+    sample = (f"one head of {w.name}: full tile selection + attention for {n_tiles} of "
+              f"{len(tile_counts(w))} query tiles per step")
+    return {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": describe(w), "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def describe(w) -> str:
+    return (f"{w.name}: B={w.B} H={w.H} d={w.d} grid={tuple(w.grid)} tile={tuple(w.tile)} "
+            f"topk={w.topk} inputs={w.kind}")
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, w, rank, world, device):
+    q, k, v = make_inputs(w, device, seed=1000 + rank)
+    grid, tile = w.grid, w.tile
+    nT = len(tile_counts(w))
+    idx = torch.empty((w.B, w.H, nT, w.topk), dtype=torch.int32, device=device)
+    ws = torch.empty(api.select_workspace_bytes(w.B, w.H, grid, w.d, tile), dtype=torch.uint8,
+                     device=device)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        api.select(q, k, grid, tile, w.topk, out=idx, workspace=ws)
+        if ev is not None:
+            ev[1].record(stream)
+        api.attn_fwd(q, k, v, idx, grid, tile, out=o, lse=lse)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if api.device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+    flops = exact_flops(idx.cpu().numpy(), w)            # idx is the same every step
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(device.index) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = start.elapsed_time(end)
+    if api.device_error() != 0:
+        raise RuntimeError("device error during the timed region")
+    sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    att_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+
+    # end to end through the public API from pinned host buffers
+    hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    e2e_steps = max(3, min(args.steps, 10))
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        api.select(q, k, grid, tile, w.topk, out=idx, workspace=ws)
+        api.attn_fwd(q, k, v, idx, grid, tile, out=o, lse=lse)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max, e2e_max = t.tolist()
+    if rank != 0:
+        return None
+
+    peaks, src = load_peaks()
+    timed_s = ms_max / 1e3
+    tensor_peak = peaks["bf16_tflops"] if timed_s < 2.0 else peaks["bf16_tflops_sustained"]
+    peak_kind = "bf16_tflops (burst)" if timed_s < 2.0 else "bf16_tflops_sustained"
+    att_tflops = flops / (att_ms * 1e-3) / 1e12
+    sel_gbs = select_bytes(w) / (sel_ms * 1e-3) / 1e9
+    value = world * flops / (ms_max / args.steps * 1e-3) / 1e12
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": describe(w), "parallelism": f"replicas x{world} (heads shard, no exchange)",
+                   "l2": "inputs 3 x %.1f MB > 126 MB L2; no flush" % (w.B * w.H * w.N * w.d * 2 / 1e6),
+                   "inputs": "torch Philox N(0,1) on device, rounded to bf16"},
+        "select_ms": sel_ms, "attend_ms": att_ms,
+        "attend_tflops_exact": att_tflops,
+        "attend_tflops_nominal": nominal_flops(w) / (att_ms * 1e-3) / 1e12,
+        "exact_flops_per_step": flops, "nominal_flops_per_step": nominal_flops(w),
+        "roofline": {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": att_tflops,
+                     "peak": tensor_peak, "unit": "TFLOP/s", "frac": att_tflops / tensor_peak,
+                     "peak_source": f"{src} {peak_kind}",
+                     "traffic": recorded_traffic("attn_fwd_kernel", w.name)},
+        "select_roofline": {"kernels": "pool_kernel + score_topk_kernel", "bound": "hbm", "achieved": sel_gbs,
+                            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": sel_gbs / peaks["hbm_gbs"],
+                            "peak_source": f"{src} hbm_gbs",
+                            "traffic": recorded_traffic("pool_kernel", w.name)},
+        "e2e": {"value": world * flops / (e2e_max * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_max,
+                "h2d_bytes_per_step": int(3 * q.numel() * 2),
+                "d2h_bytes_per_step": int(o.numel() * 2 + lse.numel() * 4)},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        nt = nT                                   # one full head: ~10-30 s of CPU work
+        dt, fl = oracle_sample(head_bits(q), head_bits(k), head_bits(v), w, nt)
+        out["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
+                               "kind": "oracle",
+                               "sample": f"one head: full tile selection + attention for {nt} of {nT} "
+                                         f"query tiles ({dt:.1f} s)"}
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="wan5b", choices=sorted(ALL))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = ALL[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, w, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=device, timeout=datetime.timedelta(seconds=120))
+    try:
+        res = run_ours(args, w, rank, world, device)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,509 @@
+// attn_kernel.cuh -- block-sparse flash-attention forward for sm_100a.
+//
+// FastVideo VSA user guide (intro): each query block attends only to the
+// tokens of its selected top-k key/value blocks; "Verify routing and
+// fallback": non-causal self-attention, scale head_size ** -0.5 by default.
+// fastbsa page ("How it works"): Q/K/V stay in raster layout and the block
+// index map is evaluated in the kernel (here: 5-D TMA boxes over
+// [B*H, T, Hh, W, d], so a tile or half-tile is one box, zero-filled past the
+// grid edge).
+//
+// One CTA = one work unit with two "slots" of up to 128 query rows each.
+//   SHARED (tiles of 256 tokens, tt >= 2): the slots are the two t-halves of
+//     one query tile and share every K/V sub-block (a t-half of a kept tile).
+//   !SHARED (tiles of 64 or 128 tokens): the slots are two consecutive query
+//     tiles; a K/V sub-block packs 128 / vol kept tiles of one slot.
+// Warp roles (320 threads): warps 0-3 softmax slot 0, warps 4-7 softmax slot 1
+// (thread = query row = TMEM lane), warp 8 TMA producer, warp 9 MMA issuer.
+// TMEM (512 columns): S_h at [128h, 128h+128), P_h (bf16 pairs) aliases the
+// first 64 columns of S_h, O_h at [256 + 128h, ...).  The MMA warp issues, per
+// K/V sub-block: PV_0(prev), S_0(cur), PV_1(prev), S_1(cur); tcgen05.mma ops
+// from one thread execute in issue order, so S_h(cur) overwrites P_h(prev)
+// only after PV_h(prev) has read it, and softmax h works while the tensor
+// pipe runs the other slot.  Online softmax in float32 with lazy rescaling (O
+// and l are only rescaled when the running max grows by more than 2^8).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "vsa_geometry.cuh"
+#include "vsa_ptx.cuh"
+
+namespace vsa {
+
+constexpr int kAttnThreads = 320;
+constexpr int kSlotRows = 128;          // MMA M
+constexpr int kSubRows = 128;           // K/V rows per sub-block (S: N, PV: K)
+constexpr float kRescaleLog2 = 8.0f;
+constexpr uint32_t kErrBadIndex = 2u;
+
+struct AttnArgs {
+  Geom g;
+  int topk;
+  float scale_log2;          // softmax_scale * log2(e)
+  const int32_t* idx;        // [B*H, nT, topk]
+  __nv_bfloat16* o;          // [B*H, N, d]
+  float* lse;                // [B*H, N]
+  unsigned int* err;         // device error word
+  int box_t;                 // t-extent of one TMA box (tt/2 when SHARED, else tt)
+};
+
+template <int D>
+struct AttnSmem {
+  static constexpr int kSlabBytes = 128 * 128;       // 128 rows x 64 bf16 (one 128B-swizzle slab)
+  static constexpr int kSlabs = D / 64;
+  static constexpr int kBufBytes = kSlabs * kSlabBytes;
+  static constexpr int kQ = 0;                        // 2 slot buffers
+  static constexpr int kK = 2 * kBufBytes;            // 2 buffers
+  static constexpr int kV = 4 * kBufBytes;            // 2 buffers
+  static constexpr int kBar = 6 * kBufBytes;
+  static constexpr int kNumBars = 17;
+  static constexpr int kMisc = kBar + kNumBars * 8;
+  static constexpr int kTotal = kMisc + 16;
+  static constexpr int kAlloc = kTotal + 1024;        // slack for 1024-byte alignment
+};
+
+enum : int {
+  BAR_Q_FULL = 0, BAR_K_FULL = 2, BAR_K_EMPTY = 4, BAR_V_FULL = 6, BAR_V_EMPTY = 8,
+  BAR_S_FULL = 10, BAR_P_FULL = 12, BAR_O_FULL = 14, BAR_DRAIN = 16
+};
+
+struct Slot {
+  bool active;
+  int bh, tile;          // head index (b*H + h) and query tile
+  int t0, y0, x0;        // origin of the slot's query box
+};
+
+__device__ __forceinline__ int load_tile_index(const AttnArgs& a, const int32_t* row, int e,
+                                               bool report) {
+  int j = __ldg(row + e);
+  if (j < 0 || j >= a.g.nT) {
+    if (report) atomicCAS(a.err, 0u, kErrBadIndex);
+    j = 0;
+  }
+  return j;
+}
+
+// K/V sub-block sequence of one query tile.
+//   SHARED: for each kept tile (ascending), its t-halves that hold any token.
+//   !SHARED: groups of P = 128 / vol kept tiles; a short last group repeats its
+//            last tile in the missing pieces (masked out).
+template <bool SHARED>
+struct KvSeq {
+  const int32_t* row;
+  int pos, half;
+
+  __device__ void init(const AttnArgs& a, int bh, int tile) {
+    row = a.idx + (static_cast<size_t>(bh) * a.g.nT + tile) * a.topk;
+    pos = 0;
+    half = 0;
+  }
+  __device__ static bool second_half(const AttnArgs& a, int j) {
+    const int bt = j / (a.g.nTy * a.g.nTx);
+    return bt * a.g.tt + a.box_t < a.g.T;
+  }
+  __device__ int count(const AttnArgs& a) const {
+    if (!SHARED) {
+      const int P = kSubRows / a.g.vol;
+      return (a.topk + P - 1) / P;
+    }
+    int n = 0;
+    for (int e = 0; e < a.topk; ++e) n += 1 + (second_half(a, load_tile_index(a, row, e, false)) ? 1 : 0);
+    return n;
+  }
+  // Piece p of the current sub-block: tile j, t offset inside the tile, and
+  // whether it is a real piece (false: padding repeat of the last tile).
+  __device__ void piece(const AttnArgs& a, int p, bool report, int& j, int& toff, bool& real) const {
+    if (SHARED) {
+      j = load_tile_index(a, row, pos, report);
+      toff = half * a.box_t;
+      real = true;
+    } else {
+      const int e = pos + p;
+      real = e < a.topk;
+      j = load_tile_index(a, row, real ? e : a.topk - 1, report && real);
+      toff = 0;
+    }
+  }
+  __device__ void advance(const AttnArgs& a) {
+    if (SHARED) {
+      if (half == 0 && second_half(a, load_tile_index(a, row, pos, false))) {
+        half = 1;
+      } else {
+        half = 0;
+        ++pos;
+      }
+    } else {
+      pos += kSubRows / a.g.vol;
+    }
+  }
+};
+
+template <int D, bool SHARED>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+  using L = AttnSmem<D>;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* sp = smem_raw + (base - raw);
+  const uint32_t sQ = base + L::kQ, sK = base + L::kK, sV = base + L::kV, sBar = base + L::kBar;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sp + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sp + L::kMisc + 4);
+  auto bar = [&](int id) -> uint32_t { return sBar + 8u * static_cast<uint32_t>(id); };
+
+  const Geom& g = a.g;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int P = SHARED ? 1 : kSubRows / g.vol;             // pieces per sub-block
+  const int box_rows = SHARED ? kSubRows : g.vol;          // rows per TMA box
+  const uint32_t box_bytes = static_cast<uint32_t>(box_rows) * 128u;
+
+  // ---- work unit -> slots
+  Slot slot[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    int bh, tile, toff;
+    bool act;
+    if (SHARED) {
+      bh = blockIdx.x / g.nT;
+      tile = blockIdx.x % g.nT;
+      toff = h * a.box_t;
+      act = true;
+    } else {
+      const long long gidx = 2ll * blockIdx.x + h;
+      act = gidx < static_cast<long long>(g.B) * g.H * g.nT;
+      bh = act ? static_cast<int>(gidx / g.nT) : 0;
+      tile = act ? static_cast<int>(gidx % g.nT) : 0;
+      toff = 0;
+    }
+    const TileCoord c = tile_coord(g, tile);
+    slot[h].bh = bh;
+    slot[h].tile = tile;
+    slot[h].t0 = c.bt * g.tt + toff;
+    slot[h].y0 = c.by * g.th;
+    slot[h].x0 = c.bx * g.tw;
+    slot[h].active = act && slot[h].t0 < g.T;
+  }
+  const int last_active = slot[1].active ? 1 : 0;
+
+  // ---- setup: barriers, zero padding rows of Q, TMEM allocation
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < L::kNumBars; ++b) {
+      const bool p_bar = (b == BAR_P_FULL || b == BAR_P_FULL + 1);
+      mbar_init(bar(b), p_bar ? 128u : 1u);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (!SHARED && g.vol < kSlotRows) {
+    // rows [vol, 128) of the Q buffers are never loaded; make them zeros
+    for (int s = 0; s < 2; ++s)
+      for (int sl = 0; sl < L::kSlabs; ++sl) {
+        uint4* p = reinterpret_cast<uint4*>(sp + L::kQ + s * L::kBufBytes + sl * L::kSlabBytes +
+                                            g.vol * 128);
+        const int n16 = (kSlotRows - g.vol) * 128 / 16;
+        for (int e = threadIdx.x; e < n16; e += kAttnThreads) p[e] = make_uint4(0, 0, 0, 0);
+      }
+    fence_proxy_async_smem();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  KvSeq<SHARED> seq;
+  seq.init(a, slot[0].bh, slot[0].tile);
+
+  if (warp == 8) {
+    // ====================================================== TMA producer
+    if (lane == 0) {
+      bool ok = true;
+      for (int h = 0; h < 2; ++h) {
+        if (!slot[h].active) continue;
+        mbar_arrive_expect_tx(bar(BAR_Q_FULL + h), L::kSlabs * box_bytes);
+        for (int sl = 0; sl < L::kSlabs; ++sl)
+          tma_load_5d(sQ + h * L::kBufBytes + sl * L::kSlabBytes, &tmQ, bar(BAR_Q_FULL + h), sl * 64,
+                      slot[h].x0, slot[h].y0, slot[h].t0, slot[h].bh);
+      }
+      KvSeq<SHARED> sq[2];
+      sq[0].init(a, slot[0].bh, slot[0].tile);
+      sq[1].init(a, slot[1].bh, slot[1].tile);
+      const int n = sq[0].count(a);
+      int last_use[2][2] = {{-1, -1}, {-1, -1}};   // [K/V][stage]: last phase issued
+      for (int it = 0; it < n && ok; ++it) {
+        for (int kv = 0; kv < 2 && ok; ++kv) {         // K first, then V
+          const CUtensorMap* tm = kv == 0 ? &tmK : &tmV;
+          const uint32_t buf0 = kv == 0 ? sK : sV;
+          const int full = kv == 0 ? BAR_K_FULL : BAR_V_FULL;
+          const int empty = kv == 0 ? BAR_K_EMPTY : BAR_V_EMPTY;
+          for (int h = 0; h < (SHARED ? 1 : 2); ++h) {
+            if (!slot[h].active) continue;
+            const int st = SHARED ? (it & 1) : h;
+            const int use = SHARED ? (it >> 1) : it;
+            if (use > 0 && !mbar_wait(bar(empty + st), (use - 1) & 1, abort_flag, a.err)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(bar(full + st), static_cast<uint32_t>(P * L::kSlabs) * box_bytes);
+            last_use[kv][st] = use;
+            for (int p = 0; p < P; ++p) {
+              int j, toff;
+              bool real;
+              sq[h].piece(a, p, kv == 0, j, toff, real);
+              const TileCoord c = tile_coord(g, j);
+              for (int sl = 0; sl < L::kSlabs; ++sl)
+                tma_load_5d(buf0 + st * L::kBufBytes + sl * L::kSlabBytes + p * box_bytes, tm,
+                            bar(full + st), sl * 64, c.bx * g.tw, c.by * g.th, c.bt * g.tt + toff,
+                            slot[h].bh);
+            }
+          }
+        }
+        sq[0].advance(a);
+        sq[1].advance(a);
+      }
+      // Let every issued copy land before the CTA can exit (returns at once
+      // when the consumers already saw these phases complete).
+      for (int kv = 0; kv < 2; ++kv)
+        for (int st = 0; st < 2; ++st)
+          if (last_use[kv][st] >= 0)
+            mbar_wait(bar((kv == 0 ? BAR_K_FULL : BAR_V_FULL) + st), last_use[kv][st] & 1, nullptr, a.err);
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ====================================================== MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(kSlotRows, kSubRows, false);
+      constexpr uint32_t idPV = idesc_bf16_f32(kSlotRows, D, true);
+      const int n = seq.count(a);
+      bool ok = true;
+      for (int h = 0; h < 2 && ok; ++h)
+        if (slot[h].active) ok = mbar_wait(bar(BAR_Q_FULL + h), 0, abort_flag, a.err);
+
+      auto issue_pv = [&](int h, int vst, bool acc) {
+        const uint32_t tS = tmem + 128u * h, tO = tmem + 256u + 128u * h;
+#pragma unroll
+        for (int kk = 0; kk < kSubRows / 16; ++kk) {
+          const uint64_t bd = smem_desc_sw128(sV + vst * L::kBufBytes + kk * 2048, L::kSlabBytes, 1024);
+          mma_ts(tO, tS + 8u * kk, bd, idPV, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      auto issue_s = [&](int h, int kst) {
+        const uint32_t tS = tmem + 128u * h;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int sl = kk / 4, koff = (kk % 4) * 32;
+          const uint64_t ad = smem_desc_sw128(sQ + h * L::kBufBytes + sl * L::kSlabBytes + koff, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(sK + kst * L::kBufBytes + sl * L::kSlabBytes + koff, 16, 1024);
+          mma_ss(tS, ad, bd, idS, kk > 0 ? 1u : 0u);
+        }
+      };
+
+      for (int it = 0; it < n && ok; ++it) {
+        for (int h = 0; h < 2 && ok; ++h) {
+          if (!slot[h].active) continue;
+          const int kst = SHARED ? (it & 1) : h;
+          const int kpar = SHARED ? ((it >> 1) & 1) : (it & 1);
+          if (!mbar_wait(bar(BAR_K_FULL + kst), kpar, abort_flag, a.err)) { ok = false; break; }
+          if (it > 0) {
+            const int vst = SHARED ? ((it - 1) & 1) : h;
+            const int vpar = SHARED ? (((it - 1) >> 1) & 1) : ((it - 1) & 1);
+            if (!mbar_wait(bar(BAR_P_FULL + h), (it - 1) & 1, abort_flag, a.err) ||
+                !mbar_wait(bar(BAR_V_FULL + vst), vpar, abort_flag, a.err)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(h, vst, it - 1 > 0);
+            if (!SHARED || h == last_active) mma_commit(bar(BAR_V_EMPTY + vst));
+          }
+          tc_fence_after();
+          issue_s(h, kst);
+          mma_commit(bar(BAR_S_FULL + h));
+          if (!SHARED || h == last_active) mma_commit(bar(BAR_K_EMPTY + kst));
+        }
+      }
+      for (int h = 0; h < 2 && ok; ++h) {
+        if (!slot[h].active) continue;
+        const int it = n - 1;
+        const int vst = SHARED ? (it & 1) : h;
+        const int vpar = SHARED ? ((it >> 1) & 1) : (it & 1);
+        if (!mbar_wait(bar(BAR_P_FULL + h), it & 1, abort_flag, a.err) ||
+            !mbar_wait(bar(BAR_V_FULL + vst), vpar, abort_flag, a.err)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(h, vst, it > 0);
+        mma_commit(bar(BAR_O_FULL + h));
+      }
+      // Drain: every MMA issued above has finished before TMEM is freed.
+      mma_commit(bar(BAR_DRAIN));
+      mbar_wait(bar(BAR_DRAIN), 0, nullptr, a.err);
+    }
+    __syncwarp();
+  } else {
+    // ====================================================== softmax slot h
+    const int h = warp / 4;
+    const int q = warp % 4;
+    const int r = threadIdx.x % 128;                  // query row of the slot = TMEM lane
+    if (slot[h].active) {
+      const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+      const uint32_t tS = tmem + lane_base + 128u * h;
+      const uint32_t tO = tmem + lane_base + 256u + 128u * h;
+      const int lg_yx = g.lg_th + g.lg_tw;
+
+      // which token this row is (if any)
+      bool row_valid;
+      int tok_t, tok_y, tok_x;
+      {
+        const int rr = r;
+        const int lt = rr >> lg_yx, ly = (rr >> g.lg_tw) & (g.th - 1), lx = rr & (g.tw - 1);
+        tok_t = slot[h].t0 + lt;
+        tok_y = slot[h].y0 + ly;
+        tok_x = slot[h].x0 + lx;
+        row_valid = rr < box_rows && tok_t < g.T && tok_y < g.Hh && tok_x < g.W &&
+                    lt < (SHARED ? a.box_t : g.tt);
+      }
+
+      KvSeq<SHARED> sq;
+      sq.init(a, slot[h].bh, slot[h].tile);
+      const int n = sq.count(a);
+      float m = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int it = 0; it < n; ++it) {
+        // validity of the sub-block's 128 key columns (only needed at grid edges)
+        uint32_t mw[4] = {~0u, ~0u, ~0u, ~0u};
+        bool full = true;
+        {
+          int vt[2], vy[2], vx[2];
+          bool real[2];
+          for (int p = 0; p < P; ++p) {
+            int j, toff;
+            sq.piece(a, p, false, j, toff, real[p]);
+            const TileCoord c = tile_coord(g, j);
+            int et, ey, ex;
+            tile_extent(g, c, et, ey, ex);
+            vt[p] = SHARED ? min(a.box_t, et - toff) : et;
+            vy[p] = ey;
+            vx[p] = ex;
+            full = full && real[p] && vt[p] == (SHARED ? a.box_t : g.tt) && ey == g.th && ex == g.tw;
+          }
+          if (!full) {
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const int col = 32 * w + lane;
+              const int p = SHARED ? 0 : (col / g.vol);
+              const int rr = SHARED ? col : (col % g.vol);
+              const int lt = rr >> lg_yx, ly = (rr >> g.lg_tw) & (g.th - 1), lx = rr & (g.tw - 1);
+              const bool v = p < P && real[p] && lt < vt[p] && ly < vy[p] && lx < vx[p];
+              mw[w] = __ballot_sync(0xffffffffu, v);
+            }
+          }
+        }
+        sq.advance(a);
+
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(BAR_S_FULL + h), it & 1, abort_flag, a.err))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t s[128];
+        tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+        tmem_wait_ld();
+
+        if (!full) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (!((mw[c >> 5] >> (c & 31)) & 1u)) s[c] = __float_as_uint(-INFINITY);
+        }
+        float mx = __uint_as_float(s[0]);
+#pragma unroll
+        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
+        const float mx_s = mx * a.scale_log2;
+
+        // lazy rescale: move the reference max only when it grew by > 2^8
+        float alpha = 1.f;
+        if (it == 0) {
+          m = mx_s;
+        } else if (mx_s > m + kRescaleLog2) {
+          alpha = exp2f(m - mx_s);
+          m = mx_s;
+          l *= alpha;
+        }
+        const bool rescale = __any_sync(0xffffffffu, alpha != 1.f);
+        const float neg_m = -m;
+        float lsum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float p0 = exp2f(fmaf(__uint_as_float(s[2 * c]), a.scale_log2, neg_m));
+          const float p1 = exp2f(fmaf(__uint_as_float(s[2 * c + 1]), a.scale_log2, neg_m));
+          lsum += p0 + p1;
+          s[c] = pack_bf16x2(p0, p1);
+        }
+        l += lsum;
+        tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+        if (rescale) {
+          // O_h is idle here: PV_h(it-1) completed before S_h(it) did, and
+          // PV_h(it) waits for this slot's P_FULL arrival below.
+#pragma unroll
+          for (int c4 = 0; c4 < D / 32; ++c4) {
+            uint32_t ov[32];
+            tmem_ld32(tO + 32u * c4, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st32(tO + 32u * c4, ov);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(BAR_P_FULL + h));
+      }
+
+      // ---- epilogue: O / l -> bf16, LSE
+      if (ok && __all_sync(0xffffffffu, mbar_wait(bar(BAR_O_FULL + h), 0, abort_flag, a.err))) {
+        tc_fence_after();
+        const float inv_l = 1.f / l;
+        const size_t N = static_cast<size_t>(g.T) * g.Hh * g.W;
+        const size_t n_tok = (static_cast<size_t>(tok_t) * g.Hh + tok_y) * g.W + tok_x;
+        __nv_bfloat16* orow = a.o + (static_cast<size_t>(slot[h].bh) * N + n_tok) * D;
+#pragma unroll
+        for (int c4 = 0; c4 < D / 32; ++c4) {
+          uint32_t ov[32];
+          tmem_ld32(tO + 32u * c4, ov);
+          tmem_wait_ld();
+          if (row_valid) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l, __uint_as_float(ov[2 * e + 1]) * inv_l);
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c4);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          }
+        }
+        if (row_valid)
+          a.lse[static_cast<size_t>(slot[h].bh) * N + n_tok] = (m + log2f(l)) * 0.69314718055994530942f;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace vsa

@@ -1,0 +1,216 @@
+// libvsa.cu -- the C ABI (declared in include/vsa.h): argument checks, tile
+// geometry, TMA descriptor encoding and kernel launches.  The only translation
+// unit of libvsa.so; the kernels live in the headers it includes.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "vsa.h"
+#include "attn_kernel.cuh"
+#include "select_kernels.cuh"
+#include "tma_encode.cuh"
+#include "vsa_geometry.cuh"
+
+namespace vsa {
+
+__device__ unsigned int g_device_error = 0u;
+
+constexpr int kMaxTiles = 2048;          // score rows of one CTA must fit in shared memory
+constexpr int kMaxDevices = 64;
+
+// -------------------------------------------------------------- validation
+static int make_geom(const vsa_shape* s, Geom* g) {
+  if (s == nullptr) return VSA_ERR_INVALID_ARG;
+  if (s->B <= 0 || s->H <= 0 || s->T <= 0 || s->Hh <= 0 || s->W <= 0 || s->d <= 0 || s->tt <= 0 ||
+      s->th <= 0 || s->tw <= 0)
+    return VSA_ERR_INVALID_ARG;
+  if (s->d != 64 && s->d != 128) return VSA_ERR_UNSUPPORTED;
+  const int lt = ilog2_exact(s->tt), ly = ilog2_exact(s->th), lx = ilog2_exact(s->tw);
+  if (lt < 0 || ly < 0 || lx < 0) return VSA_ERR_UNSUPPORTED;
+  if (s->tt > 256 || s->th > 256 || s->tw > 256) return VSA_ERR_UNSUPPORTED;
+  const int vol = s->tt * s->th * s->tw;
+  if (vol != 64 && vol != 128 && vol != 256) return VSA_ERR_UNSUPPORTED;
+  if (vol == 256 && s->tt < 2) return VSA_ERR_UNSUPPORTED;
+  g->B = s->B; g->H = s->H; g->T = s->T; g->Hh = s->Hh; g->W = s->W; g->d = s->d;
+  g->tt = s->tt; g->th = s->th; g->tw = s->tw;
+  g->lg_tt = lt; g->lg_th = ly; g->lg_tw = lx;
+  g->vol = vol;
+  g->nTt = ceil_div(s->T, s->tt);
+  g->nTy = ceil_div(s->Hh, s->th);
+  g->nTx = ceil_div(s->W, s->tw);
+  const long long nT = 1ll * g->nTt * g->nTy * g->nTx;
+  const long long N = 1ll * s->T * s->Hh * s->W;
+  const long long BH = 1ll * s->B * s->H;
+  // grid-dimension and index limits of the kernels
+  if (nT > kMaxTiles || BH > 65535 || BH * nT > 0x7fffffffll || N * s->d * BH > (1ll << 40))
+    return VSA_ERR_TOO_LARGE;
+  g->nT = static_cast<int>(nT);
+  return VSA_OK;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int check_arch() {
+  static int cached[kMaxDevices];          // 0 unknown, 1 ok, 2 bad
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VSA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return VSA_ERR_ARCH;
+  if (cached[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return VSA_ERR_CUDA;
+    cached[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  return cached[dev] == 1 ? VSA_OK : VSA_ERR_ARCH;
+}
+
+static unsigned int* device_error_ptr() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+  return static_cast<unsigned int*>(p);
+}
+
+static size_t score_smem_bytes(const Geom& g) {
+  return sizeof(float) * (kScoreRows * g.d + g.d * kKtStride) + sizeof(uint32_t) * (kScoreRows * g.nT + 8 * 256);
+}
+
+template <int D>
+static int launch_select(const Geom& g, const void* q, const void* k, int topk, int32_t* idx, float* ws,
+                         cudaStream_t st) {
+  const int BH = g.B * g.H;
+  pool_kernel<D><<<dim3(g.nT, BH, 2), kPoolThreads, 0, st>>>(g, static_cast<const __nv_bfloat16*>(q),
+                                                            static_cast<const __nv_bfloat16*>(k), ws);
+  if (cudaGetLastError() != cudaSuccess) return VSA_ERR_CUDA;
+  const size_t smem = score_smem_bytes(g);
+  if (cudaFuncSetAttribute(score_topk_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return VSA_ERR_CUDA;
+  score_topk_kernel<D><<<dim3(ceil_div(g.nT, kScoreRows), BH), kScoreThreads, smem, st>>>(g, ws, topk, idx);
+  return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
+template <int D, bool SHARED>
+static int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnArgs& a,
+                       cudaStream_t st) {
+  const int smem = AttnSmem<D>::kAlloc;
+  if (cudaFuncSetAttribute(attn_fwd_kernel<D, SHARED>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return VSA_ERR_CUDA;
+  const long long tiles = 1ll * a.g.B * a.g.H * a.g.nT;
+  const long long grid = SHARED ? tiles : (tiles + 1) / 2;
+  attn_fwd_kernel<D, SHARED><<<static_cast<unsigned>(grid), kAttnThreads, smem, st>>>(mq, mk, mv, a);
+  return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
+}  // namespace vsa
+
+using namespace vsa;
+
+extern "C" {
+
+int vsa_tile_count(const vsa_shape* shape, int32_t* num_tiles, int32_t* tiles_per_axis) {
+  if (num_tiles == nullptr) return VSA_ERR_INVALID_ARG;
+  Geom g;
+  const int rc = make_geom(shape, &g);
+  if (rc != VSA_OK) return rc;
+  *num_tiles = g.nT;
+  if (tiles_per_axis != nullptr) {
+    tiles_per_axis[0] = g.nTt;
+    tiles_per_axis[1] = g.nTy;
+    tiles_per_axis[2] = g.nTx;
+  }
+  return VSA_OK;
+}
+
+size_t vsa_select_workspace_bytes(const vsa_shape* shape) {
+  Geom g;
+  if (make_geom(shape, &g) != VSA_OK) return 0;
+  return sizeof(float) * 2ull * g.B * g.H * g.nT * g.d;
+}
+
+int vsa_select(const vsa_shape* shape, const void* q, const void* k, int32_t topk, int32_t* idx_out,
+               void* workspace, size_t workspace_bytes, void* stream) {
+  Geom g;
+  int rc = make_geom(shape, &g);
+  if (rc != VSA_OK) return rc;
+  if (q == nullptr || k == nullptr || idx_out == nullptr) return VSA_ERR_INVALID_ARG;
+  if (topk <= 0 || topk > g.nT) return VSA_ERR_TOPK_RANGE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(idx_out) & 3u))
+    return VSA_ERR_ALIGNMENT;
+  if (workspace == nullptr || workspace_bytes < vsa_select_workspace_bytes(shape)) return VSA_ERR_WORKSPACE;
+  if ((rc = check_arch()) != VSA_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* ws = static_cast<float*>(workspace);
+  return g.d == 128 ? launch_select<128>(g, q, k, topk, idx_out, ws, st)
+                    : launch_select<64>(g, q, k, topk, idx_out, ws, st);
+}
+
+int vsa_attn_fwd(const vsa_shape* shape, const void* q, const void* k, const void* v, const int32_t* idx,
+                 int32_t topk, float softmax_scale, void* o, float* lse, void* stream) {
+  Geom g;
+  int rc = make_geom(shape, &g);
+  if (rc != VSA_OK) return rc;
+  if (q == nullptr || k == nullptr || v == nullptr || idx == nullptr || o == nullptr || lse == nullptr)
+    return VSA_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return VSA_ERR_INVALID_ARG;
+  if (topk <= 0 || topk > g.nT) return VSA_ERR_TOPK_RANGE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return VSA_ERR_ALIGNMENT;
+  if ((rc = check_arch()) != VSA_OK) return rc;
+
+  const bool shared = (g.vol == 256);
+  AttnArgs a;
+  a.g = g;
+  a.topk = topk;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.idx = idx;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.err = device_error_ptr();
+  a.box_t = shared ? g.tt / 2 : g.tt;
+  if (a.err == nullptr) return VSA_ERR_CUDA;
+  CUtensorMap mq, mk, mv;
+  if ((rc = encode_qkv_map(&mq, q, g, a.box_t)) != VSA_OK || (rc = encode_qkv_map(&mk, k, g, a.box_t)) != VSA_OK ||
+      (rc = encode_qkv_map(&mv, v, g, a.box_t)) != VSA_OK)
+    return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (g.d == 128)
+    return shared ? launch_attn<128, true>(mq, mk, mv, a, st) : launch_attn<128, false>(mq, mk, mv, a, st);
+  return shared ? launch_attn<64, true>(mq, mk, mv, a, st) : launch_attn<64, false>(mq, mk, mv, a, st);
+}
+
+int vsa_device_error(uint32_t* code, int32_t reset) {
+  if (code == nullptr) return VSA_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return VSA_ERR_CUDA;
+  unsigned int h = 0;
+  if (cudaMemcpyFromSymbol(&h, g_device_error, sizeof(h)) != cudaSuccess) return VSA_ERR_CUDA;
+  *code = h;
+  if (reset) {
+    const unsigned int z = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &z, sizeof(z)) != cudaSuccess) return VSA_ERR_CUDA;
+  }
+  return VSA_OK;
+}
+
+const char* vsa_status_string(int32_t status) {
+  switch (status) {
+    case VSA_OK: return "VSA_OK";
+    case VSA_ERR_INVALID_ARG: return "VSA_ERR_INVALID_ARG";
+    case VSA_ERR_TOPK_RANGE: return "VSA_ERR_TOPK_RANGE";
+    case VSA_ERR_UNSUPPORTED: return "VSA_ERR_UNSUPPORTED";
+    case VSA_ERR_ALIGNMENT: return "VSA_ERR_ALIGNMENT";
+    case VSA_ERR_WORKSPACE: return "VSA_ERR_WORKSPACE";
+    case VSA_ERR_ARCH: return "VSA_ERR_ARCH";
+    case VSA_ERR_CUDA: return "VSA_ERR_CUDA";
+    case VSA_ERR_TOO_LARGE: return "VSA_ERR_TOO_LARGE";
+    default: return "VSA_ERR_UNKNOWN";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,228 @@
+// select_kernels.cuh -- tile selection: mean-pooling, tile scores, top-k.
+//
+// FastVideo VSA user guide (intro): for every query block, VSA scores the
+// key/value blocks and keeps the top-k ("Wan top-k behavior": top-k counts
+// key/value blocks per query block).  Scores are dot products of the tiles'
+// mean-pooled Q and K.  fastbsa page ("How it works"): selection stays in
+// shared memory instead of round-tripping a score matrix through HBM.
+//
+// Two kernels:
+//   pool_kernel   HBM-bound: reads every Q and K byte once, writes the per-tile
+//                 means (float32 [2, B*H, nT, d]) to the caller's workspace.
+//   score_topk_kernel: per (head, block of query tiles) computes the score
+//                 rows into shared memory (float32 FMA in a fixed order) and
+//                 runs an exact radix select per row; writes ascending idx.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "vsa_geometry.cuh"
+
+namespace vsa {
+
+constexpr int kPoolThreads = 256;
+
+// One CTA per (tile j, head bh, tensor z in {Q, K}).  Threads split a row of d
+// bf16 values into 16-byte vectors (TPR threads per row) and stride over the
+// tile's valid rows; partial sums are combined in a fixed order, so the result
+// is deterministic.
+template <int D>
+__global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geom g, const __nv_bfloat16* __restrict__ q,
+                                                            const __nv_bfloat16* __restrict__ k,
+                                                            float* __restrict__ pooled) {
+  constexpr int TPR = D / 8;                 // threads per row (8 bf16 each)
+  constexpr int RP = kPoolThreads / TPR;     // rows in flight per pass
+  __shared__ float part[RP][D + 4];
+
+  const int j = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int z = blockIdx.z;
+  const __nv_bfloat16* src = (z == 0 ? q : k);
+  const size_t N = static_cast<size_t>(g.T) * g.Hh * g.W;
+  src += static_cast<size_t>(bh) * N * D;
+
+  const TileCoord c = tile_coord(g, j);
+  int vt, vy, vx;
+  tile_extent(g, c, vt, vy, vx);
+  const int cnt = vt * vy * vx;
+  const int t0 = c.bt * g.tt, y0 = c.by * g.th, x0 = c.bx * g.tw;
+
+  const int cg = threadIdx.x % TPR;
+  const int rl = threadIdx.x / TPR;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+
+  const int vyx = vy * vx;
+#pragma unroll 4
+  for (int r = rl; r < cnt; r += RP) {
+    const int lt = r / vyx;
+    const int rem = r - lt * vyx;
+    const int ly = rem / vx;
+    const int lx = rem - ly * vx;
+    const size_t n = (static_cast<size_t>(t0 + lt) * g.Hh + (y0 + ly)) * g.W + (x0 + lx);
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(src + n * D) + cg);
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h2[e]);
+      acc[2 * e] += f.x;
+      acc[2 * e + 1] += f.y;
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) part[rl][cg * 8 + e] = acc[e];
+  __syncthreads();
+  for (int col = threadIdx.x; col < D; col += kPoolThreads) {
+    float s = 0.f;
+#pragma unroll 8
+    for (int i = 0; i < RP; ++i) s += part[i][col];
+    pooled[((static_cast<size_t>(z) * g.B * g.H + bh) * g.nT + j) * D + col] = s / static_cast<float>(cnt);
+  }
+}
+
+constexpr int kScoreThreads = 256;  // 8 warps
+constexpr int kScoreRows = 16;      // query tiles per CTA (2 per warp for top-k)
+constexpr int kScoreChunk = 64;     // key tiles per shared-memory chunk
+constexpr int kKtStride = kScoreChunk + 1;  // padded row of the transposed chunk
+
+// Larger float -> larger unsigned key (total order; -0 < +0, scores are
+// canonicalised so -0 does not occur).
+__device__ __forceinline__ uint32_t order_key(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Dynamic shared memory: qb[R][D] | kT[D][CH+1] | keys[R][nT] (uint32) | hist[8][256]
+template <int D>
+__global__ void __launch_bounds__(kScoreThreads) score_topk_kernel(Geom g, const float* __restrict__ pooled,
+                                                                   int topk, int32_t* __restrict__ idx) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float* qb = reinterpret_cast<float*>(smem_raw);
+  float* kT = qb + kScoreRows * D;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(kT + D * kKtStride);
+  uint32_t* hist_all = keys + kScoreRows * g.nT;
+
+  const int nT = g.nT;
+  const int bh = blockIdx.y;
+  const int row0 = blockIdx.x * kScoreRows;
+  const int nrows = min(kScoreRows, nT - row0);
+  const size_t BH = static_cast<size_t>(g.B) * g.H;
+  const float* qp = pooled + (static_cast<size_t>(bh) * nT) * D;
+  const float* kp = pooled + ((BH + bh) * nT) * D;
+
+  for (int e = threadIdx.x; e < kScoreRows * D; e += kScoreThreads) {
+    const int r = e / D;
+    qb[e] = (r < nrows) ? qp[static_cast<size_t>(row0 + r) * D + (e % D)] : 0.f;
+  }
+
+  // score phase: thread -> (column jj, 4 consecutive rows)
+  const int jj = threadIdx.x % kScoreChunk;
+  const int rg = threadIdx.x / kScoreChunk;       // 0..3
+  for (int c0 = 0; c0 < nT; c0 += kScoreChunk) {
+    __syncthreads();
+    const int ncol = min(kScoreChunk, nT - c0);
+    for (int e = threadIdx.x; e < kScoreChunk * (D / 4); e += kScoreThreads) {
+      const int cc = e / (D / 4), k4 = e % (D / 4);
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (cc < ncol) v = *reinterpret_cast<const float4*>(kp + static_cast<size_t>(c0 + cc) * D + 4 * k4);
+      kT[(4 * k4 + 0) * kKtStride + cc] = v.x;
+      kT[(4 * k4 + 1) * kKtStride + cc] = v.y;
+      kT[(4 * k4 + 2) * kKtStride + cc] = v.z;
+      kT[(4 * k4 + 3) * kKtStride + cc] = v.w;
+    }
+    __syncthreads();
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    const float* q0 = qb + (rg * 4) * D;
+#pragma unroll 8
+    for (int kk = 0; kk < D; ++kk) {
+      const float kv = kT[kk * kKtStride + jj];
+      a0 = fmaf(q0[kk], kv, a0);
+      a1 = fmaf(q0[D + kk], kv, a1);
+      a2 = fmaf(q0[2 * D + kk], kv, a2);
+      a3 = fmaf(q0[3 * D + kk], kv, a3);
+    }
+    if (jj < ncol) {
+      uint32_t* kr = keys + (rg * 4) * nT + c0 + jj;
+      kr[0] = order_key(a0 + 0.f);
+      kr[nT] = order_key(a1 + 0.f);
+      kr[2 * nT] = order_key(a2 + 0.f);
+      kr[3 * nT] = order_key(a3 + 0.f);
+    }
+  }
+  __syncthreads();
+
+  // top-k phase: warp w handles rows 2w, 2w+1 with an exact 4-pass radix select.
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  uint32_t* hist = hist_all + warp * 256;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int rr = 0; rr < 2; ++rr) {
+    const int r = warp * 2 + rr;
+    if (r >= nrows) break;
+    const uint32_t* kr = keys + r * nT;
+    uint32_t prefix = 0, pmask = 0;
+    int want = topk;  // rank (1-based) of the threshold among remaining candidates
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int b = lane; b < 256; b += 32) hist[b] = 0;
+      __syncwarp();
+      for (int jx = lane; jx < nT; jx += 32) {
+        const uint32_t u = kr[jx];
+        if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+      }
+      __syncwarp();
+      // lane l owns bins 255-8l .. 248-8l (descending digit order)
+      uint32_t cnt8[8];
+      uint32_t tot = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        cnt8[e] = hist[255 - 8 * lane - e];
+        tot += cnt8[e];
+      }
+      uint32_t incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      uint32_t above = incl - tot;  // candidates with a larger digit than my bins
+      int found_digit = -1;
+      uint32_t found_above = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if (found_digit < 0 && above < static_cast<uint32_t>(want) &&
+            above + cnt8[e] >= static_cast<uint32_t>(want)) {
+          found_digit = 255 - 8 * lane - e;
+          found_above = above;
+        }
+        above += cnt8[e];
+      }
+      const uint32_t who = __ballot_sync(0xffffffffu, found_digit >= 0);
+      const int src = __ffs(who) - 1;
+      found_digit = __shfl_sync(0xffffffffu, found_digit, src);
+      found_above = __shfl_sync(0xffffffffu, found_above, src);
+      want -= static_cast<int>(found_above);
+      prefix |= static_cast<uint32_t>(found_digit) << shift;
+      pmask |= 255u << shift;
+      __syncwarp();
+    }
+    // prefix is the topk-th largest key; take every larger key and the first
+    // `want` keys equal to it (lowest tile index first), in ascending order.
+    int32_t* out = idx + (static_cast<size_t>(bh) * nT + row0 + r) * topk;
+    int base = 0, eq_seen = 0;
+    for (int j0 = 0; j0 < nT; j0 += 32) {
+      const int jx = j0 + lane;
+      const uint32_t u = (jx < nT) ? kr[jx] : 0u;
+      const bool gt = (jx < nT) && (u > prefix);
+      const bool eq = (jx < nT) && (u == prefix);
+      const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+      const bool take = gt || (eq && (eq_seen + __popc(eqm & lt_mask)) < want);
+      const uint32_t tm = __ballot_sync(0xffffffffu, take);
+      if (take) out[base + __popc(tm & lt_mask)] = jx;
+      base += __popc(tm);
+      eq_seen += __popc(eqm);
+    }
+  }
+}
+
+}  // namespace vsa

@@ -44,59 +44,63 @@ def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
     return (bits.astype(np.uint32) << np.uint32(16)).view(np.float32)
 
 
-def _field(rng: np.random.Generator, B: int, H: int, grid: tuple, d: int) -> np.ndarray:
-    """Sum-of-sinusoids field, float32 ``[B, H, N, d]``.
+def _field_params(rng: np.random.Generator, B: int, H: int, d: int):
+    """Frequencies [B, H, d, 8, 3] (cycles per grid extent) and phases [B, H, d, 8]."""
+    freq = rng.uniform(0.0, 1.5, size=(B, H, d, N_SINUSOIDS, 3))
+    phase = rng.uniform(0.0, 2.0 * np.pi, size=(B, H, d, N_SINUSOIDS))
+    return freq, phase
 
-    Each sinusoid is sin(2*pi*(ft*t/T + fy*y/Hh + fx*x/W) + phi).  It is built
-    as Im(e^{i phi} e^{i 2 pi ft t/T} * e^{i 2 pi (fy y/Hh + fx x/W)}), so the
-    grid-sized product is a batched complex matrix product with an inner
+
+def _field_head(freq: np.ndarray, phase: np.ndarray, grid: tuple) -> np.ndarray:
+    """Sum-of-sinusoids field of one head, float32 [N, d].
+
+    Each sinusoid is 0.5 * sin(2*pi*(ft*t/T + fy*y/Hh + fx*x/W) + phi).  It is
+    built as Im(0.5 e^{i phi} e^{i 2 pi ft t/T} * e^{i 2 pi (fy y/Hh + fx x/W)}),
+    so the grid-sized sum is a batched complex matrix product with an inner
     dimension of 8 (one term per sinusoid).
     """
     T, Hh, W = grid
-    S = N_SINUSOIDS
-    freq = rng.uniform(0.0, 1.5, size=(B, H, d, S, 3))
-    phase = rng.uniform(0.0, 2.0 * np.pi, size=(B, H, d, S))
-    amp = 0.5
+    d, S = phase.shape
     t = np.arange(T) / T
     y = np.arange(Hh) / Hh
     x = np.arange(W) / W
-    out = np.empty((B, H, T * Hh * W, d), dtype=np.float32)
-    for b in range(B):
-        for h in range(H):
-            f = freq[b, h]                                            # [d, S, 3]
-            ph = phase[b, h]                                          # [d, S]
-            et = np.exp(2j * np.pi * f[:, :, 0, None] * t)            # [d, S, T]
-            et = et * (amp * np.exp(1j * ph))[:, :, None]
-            ey = np.exp(2j * np.pi * f[:, :, 1, None] * y)            # [d, S, Hh]
-            ex = np.exp(2j * np.pi * f[:, :, 2, None] * x)            # [d, S, W]
-            eyx = (ey[:, :, :, None] * ex[:, :, None, :]).reshape(d, S, Hh * W)
-            # [d, T, S] @ [d, S, Hh*W] -> [d, T, Hh*W]
-            prod = np.matmul(et.transpose(0, 2, 1).astype(np.complex64),
-                             eyx.astype(np.complex64))
-            out[b, h] = prod.imag.reshape(d, T * Hh * W).T
-    return out
+    et = np.exp(2j * np.pi * freq[:, :, 0, None] * t)                 # [d, S, T]
+    et = et * (0.5 * np.exp(1j * phase))[:, :, None]
+    ey = np.exp(2j * np.pi * freq[:, :, 1, None] * y)                 # [d, S, Hh]
+    ex = np.exp(2j * np.pi * freq[:, :, 2, None] * x)                 # [d, S, W]
+    eyx = (ey[:, :, :, None] * ex[:, :, None, :]).reshape(d, S, Hh * W)
+    prod = np.matmul(et.transpose(0, 2, 1).astype(np.complex64), eyx.astype(np.complex64))
+    return np.ascontiguousarray(prod.imag.reshape(d, T * Hh * W).T)
 
 
 def make_qkv(B: int, H: int, grid: tuple, d: int, seed: int = 0,
              kind: str = "normal"):
-    """Return (q, k, v) as uint16 bfloat16-bit arrays of shape [B, H, N, d]."""
+    """Return (q, k, v) as uint16 bfloat16-bit arrays of shape [B, H, N, d].
+
+    Values are drawn head by head in (b, h) order within each tensor; a
+    Generator fills consecutive draws from one stream, so this equals drawing
+    each whole tensor at once.
+    """
     T, Hh, W = grid
     N = T * Hh * W
     rng = np.random.Generator(np.random.PCG64(seed))
-    shape = (B, H, N, d)
+    out = [np.empty((B, H, N, d), dtype=np.uint16) for _ in range(3)]
     if kind == "normal":
-        q = rng.standard_normal(shape, dtype=np.float32)
-        q = f32_to_bf16_bits(q)
-        k = f32_to_bf16_bits(rng.standard_normal(shape, dtype=np.float32))
-        v = f32_to_bf16_bits(rng.standard_normal(shape, dtype=np.float32))
-        return q, k, v
+        for x in out:
+            for b in range(B):
+                for h in range(H):
+                    x[b, h] = f32_to_bf16_bits(rng.standard_normal((N, d), dtype=np.float32))
+        return tuple(out)
     if kind == "field":
-        fld = _field(rng, B, H, grid, d)
-        q = fld + np.float32(0.5) * rng.standard_normal(shape, dtype=np.float32)
-        q = f32_to_bf16_bits(q)
-        k = fld + np.float32(0.5) * rng.standard_normal(shape, dtype=np.float32)
-        del fld
-        k = f32_to_bf16_bits(k)
-        v = f32_to_bf16_bits(rng.standard_normal(shape, dtype=np.float32))
-        return q, k, v
+        freq, phase = _field_params(rng, B, H, d)
+        for x in out[:2]:                  # the field is recomputed for K (same values)
+            for b in range(B):
+                for h in range(H):
+                    fld = _field_head(freq[b, h], phase[b, h], grid)
+                    noise = rng.standard_normal((N, d), dtype=np.float32)
+                    x[b, h] = f32_to_bf16_bits(fld + np.float32(0.5) * noise)
+        for b in range(B):
+            for h in range(H):
+                out[2][b, h] = f32_to_bf16_bits(rng.standard_normal((N, d), dtype=np.float32))
+        return tuple(out)
     raise ValueError(f"unknown input kind {kind!r}")

@@ -1,0 +1,129 @@
+/*
+ * vsa.h -- C ABI of libvsa: VSA-style 3-D block-sparse attention on B200 (sm_100a).
+ *
+ * The method (FastVideo VSA user guide, intro): the post-patch latent grid
+ * (T, Hh, W) of a video DiT is cut into spatio-temporal tiles; each query tile
+ * scores every key/value tile and attends only to the tokens of its top-k
+ * tiles.  Two calls make the forward pass:
+ *
+ *   vsa_select    mean-pool Q and K per tile, score every tile pair,
+ *                 keep the top-k key tiles per query tile   -> idx
+ *   vsa_attn_fwd  exact softmax attention of each query tile over the
+ *                 tokens of its kept tiles                  -> O, LSE
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Tensors are dense, row-major, on the current CUDA device:
+ *   Q, K, V, O : bfloat16 [B, H, N, d], N = T*Hh*W, token n = (t*Hh + y)*W + x
+ *                (raster order over the grid; no permutation to tile order is
+ *                 needed -- the kernels evaluate the tile index map themselves,
+ *                 as the fastbsa page's "How it works" describes)
+ *   idx        : int32 [B, H, nT, topk], kept key tiles of each query tile,
+ *                strictly ascending, each in [0, nT)
+ *   LSE        : float32 [B, H, N], natural log of the softmax denominator
+ * Tiles: nT = ceil(T/tt) * ceil(Hh/th) * ceil(W/tw) (the user guide's routing
+ * log: grid (31,22,40), tile (4,8,8) -> 120 tiles); edge tiles are partial and
+ * their missing tokens are left out of pooling and of the softmax.  Tile
+ * j = (bt * ceil(Hh/th) + by) * ceil(W/tw) + bx (raster over tile coordinates).
+ *
+ * Supported: d in {64, 128}; tt, th, tw powers of two with tt*th*tw in
+ * {64, 128, 256} (the guide's 4x4x4 = 64 and 4x8x8 = 256 blocks), and tt >= 2
+ * when tt*th*tw = 256; H_q = H_kv; non-causal self-attention, no mask.
+ * Inputs must be finite (NaN/Inf give unspecified results, never a fault).
+ *
+ * Ownership: the caller allocates every buffer (including the select
+ * workspace); the library allocates no device memory.  Calls are asynchronous
+ * on `stream` (a cudaStream_t; NULL = legacy default stream).  Every call
+ * checks its arguments before launching anything and returns a vsa_status;
+ * nothing is launched on error.  Faults inside a kernel are reported through
+ * vsa_device_error() (bounded waits in the kernels turn a stall into an error
+ * code instead of a hang).
+ */
+#ifndef VSA_H_
+#define VSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct vsa_shape {
+  int32_t B, H;          /* batch, heads (query heads == key/value heads)     */
+  int32_t T, Hh, W;      /* post-patch latent grid                            */
+  int32_t d;             /* head dimension: 64 or 128                         */
+  int32_t tt, th, tw;    /* tile extents along T, Hh, W                        */
+} vsa_shape;
+
+typedef enum vsa_status {
+  VSA_OK = 0,
+  VSA_ERR_INVALID_ARG = 1,  /* NULL pointer, non-positive extent, bad scale    */
+  VSA_ERR_TOPK_RANGE = 2,   /* topk <= 0 or topk > nT (guide: topk must be
+                               positive; topk > num_blocks is invalid)         */
+  VSA_ERR_UNSUPPORTED = 3,  /* d or tile shape outside the supported set       */
+  VSA_ERR_ALIGNMENT = 4,    /* a tensor pointer not 16-byte aligned            */
+  VSA_ERR_WORKSPACE = 5,    /* workspace NULL or smaller than required         */
+  VSA_ERR_ARCH = 6,         /* current device is not sm_100                    */
+  VSA_ERR_CUDA = 7,         /* a CUDA runtime/driver call failed               */
+  VSA_ERR_TOO_LARGE = 8     /* a size exceeds what the kernels index           */
+} vsa_status;
+
+/* Tile count of a shape (FastVideo VSA guide, "Wan top-k behavior": num_blocks).
+ * num_tiles: out, nT.  tiles_per_axis: out [3] (ceil per axis) or NULL.
+ * Host only; touches no device. */
+int vsa_tile_count(const vsa_shape* shape, int32_t* num_tiles, int32_t* tiles_per_axis);
+
+/* Bytes of device workspace vsa_select needs for `shape` (pooled Q and K tile
+ * means, float32 [2, B, H, nT, d]).  Returns 0 for an invalid shape. */
+size_t vsa_select_workspace_bytes(const vsa_shape* shape);
+
+/* Tile selection (FastVideo VSA guide intro and "Wan top-k behavior"; fastbsa
+ * page "How it works": selection kept on chip, no score matrix in HBM).
+ *   q, k      : device bfloat16 [B, H, N, d], 16-byte aligned
+ *   topk      : kept key tiles per query tile, 1 <= topk <= nT
+ *               (topk == nT keeps every tile: the dense case)
+ *   idx_out   : device int32 [B, H, nT, topk]; row i gets the topk tiles j with
+ *               the largest s_ij = mean_i(Q) . mean_j(K) (float32 means over the
+ *               tile's valid tokens, float32 dot), ties to the lower j, written
+ *               in ascending j order
+ *   workspace : device buffer of at least vsa_select_workspace_bytes(shape)
+ *               bytes, 16-byte aligned; contents on entry are ignored
+ * Two kernel launches on `stream`. */
+int vsa_select(const vsa_shape* shape, const void* q, const void* k, int32_t topk,
+               int32_t* idx_out, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Block-sparse attention forward (FastVideo VSA guide intro: attention only
+ * against the selected top-k blocks; "Verify routing and fallback": scale
+ * head_size ** -0.5 by default, non-causal, no mask).
+ *   q, k, v       : device bfloat16 [B, H, N, d], 16-byte aligned
+ *   idx           : device int32 [B, H, nT, topk], ascending distinct tiles
+ *                   (as vsa_select writes them); an entry outside [0, nT)
+ *                   raises a device error and is treated as an empty tile
+ *   softmax_scale : > 0 and finite; pass d ** -0.5 for the standard scale
+ *   o             : device bfloat16 [B, H, N, d] out, 16-byte aligned
+ *   lse           : device float32 [B, H, N] out, natural log
+ * For every token n of query tile i: O[n] = softmax_m(scale * Q[n].K[m]) V[m]
+ * over the valid tokens m of the tiles idx[i, :]; LSE[n] = log of the
+ * denominator.  One kernel launch on `stream`. */
+int vsa_attn_fwd(const vsa_shape* shape, const void* q, const void* k, const void* v,
+                 const int32_t* idx, int32_t topk, float softmax_scale,
+                 void* o, float* lse, void* stream);
+
+/* Reads (and with reset != 0 clears) the kernels' device error word on the
+ * current device: 0 = no error; otherwise a VSA_DEVERR_* code.  Synchronizes
+ * the device.  Returns a vsa_status for the read itself. */
+int vsa_device_error(uint32_t* code, int32_t reset);
+
+#define VSA_DEVERR_NONE 0u
+#define VSA_DEVERR_WAIT_TIMEOUT 1u   /* an mbarrier wait ran past its bound     */
+#define VSA_DEVERR_BAD_INDEX 2u      /* idx entry outside [0, nT)              */
+
+/* Human-readable name of a vsa_status value.  Never NULL. */
+const char* vsa_status_string(int32_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VSA_H_ */

@@ -1,0 +1,107 @@
+"""The C-ABI library without a GPU: it loads, exports every declared symbol,
+and its host-side geometry and argument checks behave as documented.  No
+kernel is launched here (every call returns before touching a device)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from block_sparse_video_tile_b200 import _native, api
+from block_sparse_video_tile_b200.workloads import ALL
+from oracle import vsa_oracle as vo
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "vsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return set(re.findall(r"^\s*(?:int|size_t|const char\*)\s+(vsa_\w+)\s*\(", src, flags=re.M))
+
+
+def test_library_exports_every_declared_symbol():
+    declared = _declared()
+    assert declared == set(_native.EXPORTS)
+    L = ctypes.CDLL(_native.LIB_PATH)
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+def test_status_strings():
+    for code, name in _native.STATUS.items():
+        assert _native.lib().vsa_status_string(code).decode() == name
+    assert _native.lib().vsa_status_string(999).decode() == "VSA_ERR_UNKNOWN"
+
+
+def test_routing_log_tile_count():
+    # FastVideo VSA user guide, "Wan top-k behavior": (31,22,40) with 4x8x8 -> 120
+    n, per = api.tile_count((31, 22, 40), (4, 8, 8))
+    assert (n, per) == (120, (8, 3, 5))
+
+
+@pytest.mark.parametrize("name", sorted(ALL))
+def test_tile_count_matches_oracle(name):
+    w = ALL[name]
+    n, per = api.tile_count(w.grid, w.tile, w.d, w.B, w.H)
+    assert n == vo.num_tiles(w.grid, w.tile)
+    assert per == vo.tiles_per_axis(w.grid, w.tile)
+    assert api.select_workspace_bytes(w.B, w.H, w.grid, w.d, w.tile) == 4 * 2 * w.B * w.H * n * w.d
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=96), 3), (dict(d=0), 1), (dict(tile=(3, 8, 8)), 3), (dict(tile=(1, 16, 16)), 3),
+    (dict(tile=(4, 8, 16)), 3), (dict(grid=(0, 22, 40)), 1), (dict(tile=(8, 8, 8)), 3),
+])
+def test_unsupported_shapes(kw, status):
+    args = dict(B=1, H=1, grid=(31, 22, 40), d=128, tile=(4, 8, 8))
+    args.update(kw)
+    shp = api.make_shape(**args)
+    n = ctypes.c_int32()
+    assert _native.lib().vsa_tile_count(ctypes.byref(shp), ctypes.byref(n), None) == status
+    assert _native.lib().vsa_select_workspace_bytes(ctypes.byref(shp)) == 0
+
+
+def _sel(shp, q=256, k=512, topk=4, idx=1024, ws=2048, ws_bytes=1 << 30):
+    return _native.lib().vsa_select(ctypes.byref(shp), q, k, topk, idx, ws, ws_bytes, None)
+
+
+def _att(shp, q=256, k=512, v=768, idx=1024, topk=4, scale=0.1, o=2048, lse=4096):
+    return _native.lib().vsa_attn_fwd(ctypes.byref(shp), q, k, v, idx, topk, scale, o, lse, None)
+
+
+def test_argument_checks_before_launch():
+    """Every one of these fails validation, so no device is ever touched."""
+    shp = api.make_shape(1, 2, (31, 22, 40), 128, (4, 8, 8))
+    assert _sel(shp, topk=0) == 2
+    assert _sel(shp, topk=121) == 2
+    assert _sel(shp, topk=-3) == 2
+    assert _sel(shp, q=0) == 1
+    assert _sel(shp, q=8) == 4                       # not 16-byte aligned
+    assert _sel(shp, idx=2) == 4
+    assert _sel(shp, ws=0) == 5
+    assert _sel(shp, ws_bytes=16) == 5
+    assert _att(shp, topk=0) == 2
+    assert _att(shp, topk=121) == 2
+    assert _att(shp, scale=0.0) == 1
+    assert _att(shp, scale=float("nan")) == 1
+    assert _att(shp, scale=float("inf")) == 1
+    assert _att(shp, v=0) == 1
+    assert _att(shp, o=24) == 4
+    assert _att(shp, lse=6) == 4
+    shp_bad = api.make_shape(1, 2, (31, 22, 40), 80, (4, 8, 8))
+    assert _att(shp_bad) == 3
+    assert _sel(shp_bad) == 3
+
+
+def test_too_large_rejected():
+    shp = api.make_shape(1, 1, (64, 64, 64), 128, (4, 4, 4))   # 4096 tiles
+    n = ctypes.c_int32()
+    assert _native.lib().vsa_tile_count(ctypes.byref(shp), ctypes.byref(n), None) == 8
+
+
+def test_python_wrapper_raises():
+    with pytest.raises(_native.VsaError) as e:
+        api.tile_count((31, 22, 40), (3, 8, 8))
+    assert e.value.status == 3

@@ -1,0 +1,184 @@
+"""CUDA path vs the float64 oracle, through the C ABI.
+
+Small cases are compared element by element on every token; they span
+several tiles and ragged (partial) edge tiles on every axis, both tile
+volumes (64 and 256 tokens, plus 128), both head sizes and batch > 1.  The
+five full-size workloads run in the configuration the benchmark times and are
+checked on every selected index and on sampled query tiles (edge tiles
+included) of the attention output.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_video_tile_b200 import api
+from block_sparse_video_tile_b200.workloads import ALL, LONGCAT, SWEEP, TINY, WAN14B, WAN5B, Workload
+from oracle import vsa_oracle as vo
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    TINY,
+    TINY.with_(name="tiny_s1"),
+    Workload("ragged256", 1, 2, (9, 20, 20), 128, (4, 8, 8), 5),
+    Workload("ragged256_d64", 2, 1, (9, 20, 20), 64, (4, 8, 8), 7),
+    Workload("ragged256_field", 1, 2, (10, 17, 24), 128, (4, 8, 8), 4, "field"),
+    Workload("ragged64", 1, 2, (6, 10, 14), 128, (4, 4, 4), 5),
+    Workload("ragged64_d64", 1, 3, (5, 9, 11), 64, (4, 4, 4), 6),
+    Workload("vol128", 2, 1, (6, 12, 20), 128, (2, 8, 8), 4),
+    Workload("topk1", 1, 2, (9, 20, 20), 128, (4, 8, 8), 1),
+]
+
+
+def _seed(w):
+    return 1 if w.name == "tiny_s1" else 0
+
+
+@pytest.mark.parametrize("w", SMALL, ids=[w.name for w in SMALL])
+def test_small_full_compare(w):
+    (q, k, v), (qd, kd, vd) = gu.inputs(w, seed=_seed(w))
+    scale = w.d ** -0.5
+    idx = api.select(qd, kd, w.grid, w.tile, w.topk)
+    torch.cuda.synchronize()
+    gu.assert_no_device_error()
+    scores = gu.oracle_scores(q, k, w)
+    rows, ties = gu.check_selection(idx.cpu().numpy(), scores, w.topk)
+    # attention on the GPU's own selection (so a tie row is still checked)
+    o, lse = api.attn_fwd(qd, kd, vd, idx, w.grid, w.tile, scale=scale)
+    gu.assert_no_device_error()
+    gu.check_attention(o, lse, q, k, v, w, idx.cpu().numpy(), scale)
+
+
+@pytest.mark.parametrize("w", [SMALL[2], SMALL[5], SMALL[7]], ids=lambda w: w.name)
+def test_oracle_indices_attention(w):
+    """Attention alone, fed the oracle's selection and an arbitrary one."""
+    (q, k, v), (qd, kd, vd) = gu.inputs(w, seed=3)
+    nT = vo.num_tiles(w.grid, w.tile)
+    rng = np.random.default_rng(5)
+    idx = np.sort(np.stack([[rng.choice(nT, w.topk, replace=False) for _ in range(nT)]
+                            for _ in range(w.B * w.H)]), axis=-1).reshape(w.B, w.H, nT, w.topk)
+    idx = idx.astype(np.int32)
+    o, lse = api.attn_fwd(qd, kd, vd, torch.from_numpy(idx).cuda(), w.grid, w.tile, scale=0.3)
+    gu.assert_no_device_error()
+    gu.check_attention(o, lse, q, k, v, w, idx, 0.3)
+
+
+@pytest.mark.parametrize("w", [SMALL[2], SMALL[5], SMALL[3]], ids=lambda w: w.name)
+def test_all_tiles_equal_dense(w):
+    """topk == num_blocks keeps every tile: the result is dense attention
+    (FastVideo VSA user guide, "Wan top-k behavior")."""
+    (q, k, v), (qd, kd, vd) = gu.inputs(w, seed=4)
+    nT = vo.num_tiles(w.grid, w.tile)
+    idx = api.select(qd, kd, w.grid, w.tile, nT)
+    assert (idx.cpu().numpy() == np.arange(nT)).all()
+    scale = w.d ** -0.5
+    o, lse = api.attn_fwd(qd, kd, vd, idx, w.grid, w.tile, scale=scale)
+    gu.assert_no_device_error()
+    og, lg = o.float().cpu().numpy(), lse.cpu().numpy()
+    for b in range(w.B):
+        for h in range(w.H):
+            Od, Ld = vo.dense_bruteforce(*(vo.bf16_to_f64(x[b, h]) for x in (q, k, v)), scale)
+            e = np.abs(og[b, h] - Od)
+            assert e.max() <= gu.O_MAX_ABS and e.mean() <= gu.O_MEAN_ABS
+            assert np.abs(lg[b, h] - Ld).max() <= gu.LSE_ABS
+
+
+def test_deterministic():
+    w = SMALL[2]
+    _, (qd, kd, vd) = gu.inputs(w, seed=9)
+    outs = []
+    for _ in range(2):
+        idx = api.select(qd, kd, w.grid, w.tile, w.topk)
+        o, lse = api.attn_fwd(qd, kd, vd, idx, w.grid, w.tile)
+        outs.append((idx.clone(), o.clone(), lse.clone()))
+    assert torch.equal(outs[0][0], outs[1][0])
+    assert torch.equal(outs[0][1].view(torch.int16), outs[1][1].view(torch.int16))
+    assert torch.equal(outs[0][2], outs[1][2])
+
+
+def test_out_of_range_index_reports_error():
+    """An index outside [0, nT) is reported through the device error word;
+    the kernel reads tile 0 in its place (every load stays in bounds)."""
+    w = SMALL[2]
+    _, (qd, kd, vd) = gu.inputs(w, seed=2)
+    idx = api.select(qd, kd, w.grid, w.tile, w.topk)
+    gu.assert_no_device_error()
+    idx[0, 0, 3, 1] = 10_000
+    o, lse = api.attn_fwd(qd, kd, vd, idx, w.grid, w.tile)
+    assert api.device_error(reset=True) == 2
+    assert torch.isfinite(lse).all()
+
+
+def test_bad_topk_raises():
+    w = SMALL[2]
+    _, (qd, kd, vd) = gu.inputs(w)
+    with pytest.raises(Exception):
+        api.select(qd, kd, w.grid, w.tile, 0)
+    with pytest.raises(Exception):
+        api.select(qd, kd, w.grid, w.tile, 28)
+
+
+# ----------------------------------------------------------- full-size workloads
+FULL = [WAN5B, WAN14B, LONGCAT]
+
+
+def _sample_tiles(w, rng, n_heads=2, n_tiles=4):
+    nT = vo.num_tiles(w.grid, w.tile)
+    heads = sorted(rng.choice(w.B * w.H, n_heads, replace=False).tolist())
+    out = []
+    for bh in heads:
+        b, h = divmod(bh, w.H)
+        for i in sorted({0, nT - 1, *rng.choice(nT, n_tiles - 2, replace=False).tolist()}):
+            out.append((b, h, i))
+    return out
+
+
+def _full_case(w, seed=0, topks=None):
+    (q, k, v), (qd, kd, vd) = gu.inputs(w, seed=seed)
+    scores = gu.oracle_scores(q, k, w)
+    rng = np.random.default_rng(11)
+    report = {}
+    for topk in (topks or [w.topk]):
+        idx = api.select(qd, kd, w.grid, w.tile, topk)
+        gi = idx.cpu().numpy()
+        rows, ties = gu.check_selection(gi, scores, topk)
+        o, lse = api.attn_fwd(qd, kd, vd, idx, w.grid, w.tile)
+        gu.assert_no_device_error()
+        errs = gu.check_attention(o, lse, q, k, v, w, gi, w.d ** -0.5, tiles=_sample_tiles(w, rng))
+        report[topk] = (rows, ties, errs)
+    return report
+
+
+@pytest.mark.parametrize("w", FULL, ids=lambda w: w.name)
+def test_full_size(w):
+    rep = _full_case(w)
+    print(w.name, rep)
+
+
+@pytest.mark.parametrize("kind", ["normal", "field"])
+def test_full_size_sweep(kind):
+    base = [s for s in SWEEP if s.kind == kind][0]
+    rep = _full_case(base, topks=[s.topk for s in SWEEP if s.kind == kind])
+    print("sweep", kind, rep)
+
+
+def test_full_size_sweep_all_tiles_is_dense():
+    """Wan-5B shape, topk 120 = every tile: sampled rows equal dense attention."""
+    w = WAN5B.with_(topk=120)
+    (q, k, v), (qd, kd, vd) = gu.inputs(w, seed=1)
+    idx = api.select(qd, kd, w.grid, w.tile, 120)
+    o, lse = api.attn_fwd(qd, kd, vd, idx, w.grid, w.tile)
+    gu.assert_no_device_error()
+    rng = np.random.default_rng(0)
+    og, lg = o.float().cpu().numpy(), lse.cpu().numpy()
+    scale = w.d ** -0.5
+    for bh in (0, 17):
+        rows = np.concatenate([[0, w.N - 1], rng.choice(w.N, 30, replace=False)])
+        Q, K, V = (vo.bf16_to_f64(x[0, bh]) for x in (q, k, v))
+        Od, Ld = vo.dense_bruteforce(Q[rows], K, V, scale)
+        e = np.abs(og[0, bh][rows] - Od)
+        assert e.max() <= gu.O_MAX_ABS and e.mean() <= gu.O_MEAN_ABS
+        assert np.abs(lg[0, bh][rows] - Ld).max() <= gu.LSE_ABS
