@@ -19,8 +19,9 @@ STATUS = {
 }
 DEVERR = {0: "none", 1: "wait timeout", 2: "tile index out of range"}
 
-EXPORTS = ("vsa_tile_count", "vsa_select_workspace_bytes", "vsa_select", "vsa_attn_fwd",
-           "vsa_device_error", "vsa_status_string")
+EXPORTS = ("vsa_tile_count", "vsa_select_workspace_bytes", "vsa_select", "vsa_select_noalloc",
+           "vsa_attn_fwd", "vsa_device_error", "vsa_status_string")
+SELECT_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 class VsaShape(ctypes.Structure):
@@ -52,6 +53,8 @@ def lib() -> ctypes.CDLL:
         L.vsa_select_workspace_bytes.restype = SZ
         L.vsa_select.argtypes = [S, P, P, I32, P, P, SZ, P]
         L.vsa_select.restype = ctypes.c_int
+        L.vsa_select_noalloc.argtypes = [S, P, P, I32, P, P]
+        L.vsa_select_noalloc.restype = ctypes.c_int
         L.vsa_attn_fwd.argtypes = [S, P, P, P, P, I32, ctypes.c_float, P, P, P]
         L.vsa_attn_fwd.restype = ctypes.c_int
         L.vsa_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), I32]

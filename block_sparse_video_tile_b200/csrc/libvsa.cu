@@ -107,6 +107,28 @@ static int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 
+// Scratch of vsa_select_noalloc: file-scope device array, one per GPU that
+// loads the library.  Host code must not pass `g_select_scratch` itself to a
+// kernel (on the host it is only a stand-in symbol); its device address comes
+// from cudaGetSymbolAddress, looked up once per device.
+static __device__ __align__(256) float g_select_scratch[VSA_SELECT_NOALLOC_SCRATCH_BYTES / sizeof(float)];
+
+static int select_scratch_ptr(float** out) {
+  static float* cached[kMaxDevices];
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VSA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return VSA_ERR_ARCH;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess || p == nullptr) return VSA_ERR_CUDA;
+    cached[dev] = static_cast<float*>(p);
+  }
+  *out = cached[dev];
+  return VSA_OK;
+}
+
 }  // namespace vsa
 
 using namespace vsa;
@@ -146,6 +168,23 @@ int vsa_select(const vsa_shape* shape, const void* q, const void* k, int32_t top
   if ((rc = check_arch()) != VSA_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* ws = static_cast<float*>(workspace);
+  return g.d == 128 ? launch_select<128>(g, q, k, topk, idx_out, ws, st)
+                    : launch_select<64>(g, q, k, topk, idx_out, ws, st);
+}
+
+int vsa_select_noalloc(const vsa_shape* shape, const void* q, const void* k, int32_t topk, int32_t* idx_out,
+                       void* stream) {
+  Geom g;
+  int rc = make_geom(shape, &g);
+  if (rc != VSA_OK) return rc;
+  if (q == nullptr || k == nullptr || idx_out == nullptr) return VSA_ERR_INVALID_ARG;
+  if (topk <= 0 || topk > g.nT) return VSA_ERR_TOPK_RANGE;
+  if (!aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(idx_out) & 3u)) return VSA_ERR_ALIGNMENT;
+  if (vsa_select_workspace_bytes(shape) > VSA_SELECT_NOALLOC_SCRATCH_BYTES) return VSA_ERR_WORKSPACE;
+  if ((rc = check_arch()) != VSA_OK) return rc;
+  float* ws = nullptr;
+  if ((rc = select_scratch_ptr(&ws)) != VSA_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
   return g.d == 128 ? launch_select<128>(g, q, k, topk, idx_out, ws, st)
                     : launch_select<64>(g, q, k, topk, idx_out, ws, st);
 }

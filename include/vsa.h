@@ -32,7 +32,9 @@
  * Inputs must be finite (NaN/Inf give unspecified results, never a fault).
  *
  * Ownership: the caller allocates every buffer (including the select
- * workspace); the library allocates no device memory.  Calls are asynchronous
+ * workspace); no call allocates device memory.  (The one piece of device
+ * memory the library owns is the fixed scratch array of vsa_select_noalloc,
+ * reserved when the library is loaded.)  Calls are asynchronous
  * on `stream` (a cudaStream_t; NULL = legacy default stream).  Every call
  * checks its arguments before launching anything and returns a vsa_status;
  * nothing is launched on error.  Faults inside a kernel are reported through
@@ -93,13 +95,38 @@ size_t vsa_select_workspace_bytes(const vsa_shape* shape);
 int vsa_select(const vsa_shape* shape, const void* q, const void* k, int32_t topk,
                int32_t* idx_out, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Tile selection for callers that cannot allocate device memory (no
+ * counterpart in the paper; an addition of this library).
+ *
+ * Same arguments and results as vsa_select, minus the workspace: the pooled
+ * tile means live in a fixed scratch array inside the library
+ * (VSA_SELECT_NOALLOC_SCRATCH_BYTES, allocated once per GPU when the library
+ * loads and held until the process exits).  Meant for callers that must not
+ * call cudaMalloc -- a host framework that owns all device memory through its
+ * own pool, code running inside a region where allocation is forbidden, or a
+ * plugin with no allocator handle.  This call itself allocates nothing (no
+ * cudaMalloc, no cudaFree, no allocating library routine).
+ *   - The scratch needs 2*B*H*nT*d*4 bytes; larger shapes are rejected with
+ *     VSA_ERR_WORKSPACE before anything is launched.
+ *   - The first call on a device (with that device current) looks up the
+ *     scratch array's device address; make that first call before any CUDA
+ *     stream capture.
+ *   - Every call on a device shares the one scratch array: calls that can
+ *     overlap on the GPU (different streams, no ordering) race and give
+ *     wrong indices.  Nothing needs clearing between calls (each call
+ *     overwrites every scratch element it reads).
+ * Two kernel launches on `stream`. */
+#define VSA_SELECT_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+int vsa_select_noalloc(const vsa_shape* shape, const void* q, const void* k, int32_t topk,
+                       int32_t* idx_out, void* stream);
+
 /* Block-sparse attention forward (FastVideo VSA guide intro: attention only
  * against the selected top-k blocks; "Verify routing and fallback": scale
  * head_size ** -0.5 by default, non-causal, no mask).
  *   q, k, v       : device bfloat16 [B, H, N, d], 16-byte aligned
  *   idx           : device int32 [B, H, nT, topk], ascending distinct tiles
  *                   (as vsa_select writes them); an entry outside [0, nT)
- *                   raises a device error and is treated as an empty tile
+ *                   raises a device error and is read as tile 0 instead
  *   softmax_scale : > 0 and finite; pass d ** -0.5 for the standard scale
  *   o             : device bfloat16 [B, H, N, d] out, 16-byte aligned
  *   lse           : device float32 [B, H, N] out, natural log

@@ -105,3 +105,16 @@ def test_python_wrapper_raises():
     with pytest.raises(_native.VsaError) as e:
         api.tile_count((31, 22, 40), (3, 8, 8))
     assert e.value.status == 3
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch():
+    """vsa_select_noalloc has a fixed scratch of 32 MiB: larger pooled-mean
+    buffers are refused before any launch."""
+    big = api.make_shape(8, 40, (18, 48, 80), 128, (4, 8, 8))     # 2*320*300*128*4 B = 98 MB
+    small = api.make_shape(1, 24, (31, 22, 40), 128, (4, 8, 8))
+    L = _native.lib()
+    assert L.vsa_select_workspace_bytes(ctypes.byref(big)) > _native.SELECT_NOALLOC_SCRATCH_BYTES
+    assert L.vsa_select_workspace_bytes(ctypes.byref(small)) <= _native.SELECT_NOALLOC_SCRATCH_BYTES
+    assert L.vsa_select_noalloc(ctypes.byref(big), 256, 512, 4, 1024, None) == 5
+    assert L.vsa_select_noalloc(ctypes.byref(small), 256, 512, 0, 1024, None) == 2
+    assert L.vsa_select_noalloc(ctypes.byref(small), 8, 512, 4, 1024, None) == 4
