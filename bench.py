@@ -20,6 +20,9 @@ path shards by (batch, head) with no exchange): weak scaling.
 --impl reference times the float64 CPU oracle on a bounded sample of the same
 workload (the only other place this script runs the oracle, besides the
 cpu_baseline field of the default run).
+
+--heads H runs the same workload with H heads (a smaller case of the same
+kernels, used for ncu captures).
 """
 from __future__ import annotations
 
@@ -355,10 +358,14 @@ def main():
     ap.add_argument("--workload", default="wan5b", choices=sorted(ALL))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override the head count (a smaller case of the same kernel, for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = ALL[args.workload]
+    if args.heads is not None:
+        w = w.with_(name=f"{w.name}_h{args.heads}", H=args.heads)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
