@@ -13,8 +13,10 @@
 //     one query tile and share every K/V sub-block (a t-half of a kept tile).
 //   !SHARED (tiles of 64 or 128 tokens): the slots are two consecutive query
 //     tiles; a K/V sub-block packs 128 / vol kept tiles of one slot.
-// Warp roles (320 threads): warps 0-3 softmax slot 0, warps 4-7 softmax slot 1
-// (thread = query row = TMEM lane), warp 8 TMA producer, warp 9 MMA issuer.
+// Warp roles (384 threads): warps 0-3 softmax slot 0, warps 4-7 softmax slot 1
+// (thread = query row = TMEM lane), warp 8 TMA producer, warp 9 MMA issuer,
+// warps 10-11 idle.  The producer warpgroup gives registers to the softmax
+// warpgroups (setmaxnreg): 2*128*208 + 128*80 = 63488 <= 384*168, the launch budget.
 // TMEM (512 columns): S_h at [128h, 128h+128), P_h (bf16 pairs) aliases the
 // first 64 columns of S_h, O_h at [256 + 128h, ...).  The MMA warp issues, per
 // K/V sub-block: PV_0(prev), S_0(cur), PV_1(prev), S_1(cur); tcgen05.mma ops
@@ -33,7 +35,9 @@
 
 namespace vsa {
 
-constexpr int kAttnThreads = 320;
+constexpr int kAttnThreads = 384;        // 3 warpgroups
+constexpr int kSoftmaxRegs = 208;        // per thread, warpgroups 0-1 (after setmaxnreg)
+constexpr int kProducerRegs = 80;        // per thread, warpgroup 2 (TMA + MMA warps)
 constexpr int kSlotRows = 128;          // MMA M
 constexpr int kSubRows = 128;           // K/V rows per sub-block (S: N, PV: K)
 constexpr float kRescaleLog2 = 8.0f;
@@ -226,6 +230,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   KvSeq<SHARED> seq;
   seq.init(a, slot[0].bh, slot[0].tile);
 
+  if (warp >= 8) {
+    setmaxnreg_dec<kProducerRegs>();
+  }
   if (warp == 8) {
     // ====================================================== TMA producer
     if (lane == 0) {
@@ -288,8 +295,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       constexpr uint32_t idPV = idesc_bf16_f32(kSlotRows, D, true);
       const int n = seq.count(a);
       bool ok = true;
-      for (int h = 0; h < 2 && ok; ++h)
-        if (slot[h].active) ok = mbar_wait(bar(BAR_Q_FULL + h), 0, abort_flag, a.err);
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        if (ok && slot[h].active) ok = mbar_wait(bar(BAR_Q_FULL + h), 0, abort_flag, a.err);
 
       auto issue_pv = [&](int h, int vst, bool acc) {
         const uint32_t tS = tmem + 128u * h, tO = tmem + 256u + 128u * h;
@@ -311,16 +319,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       };
 
       for (int it = 0; it < n && ok; ++it) {
-        for (int h = 0; h < 2 && ok; ++h) {
-          if (!slot[h].active) continue;
+        #pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (!ok || !slot[h].active) continue;
           const int kst = SHARED ? (it & 1) : h;
           const int kpar = SHARED ? ((it >> 1) & 1) : (it & 1);
-          if (!mbar_wait(bar(BAR_K_FULL + kst), kpar, abort_flag, a.err)) { ok = false; break; }
+          if (!mbar_wait(bar(BAR_K_FULL + kst), kpar, abort_flag, a.err)) { ok = false; continue; }
           if (it > 0) {
             const int vst = SHARED ? ((it - 1) & 1) : h;
             const int vpar = SHARED ? (((it - 1) >> 1) & 1) : ((it - 1) & 1);
             if (!mbar_wait(bar(BAR_P_FULL + h), (it - 1) & 1, abort_flag, a.err) ||
-                !mbar_wait(bar(BAR_V_FULL + vst), vpar, abort_flag, a.err)) { ok = false; break; }
+                !mbar_wait(bar(BAR_V_FULL + vst), vpar, abort_flag, a.err)) { ok = false; continue; }
             tc_fence_after();
             issue_pv(h, vst, it - 1 > 0);
             if (!SHARED || h == last_active) mma_commit(bar(BAR_V_EMPTY + vst));
@@ -331,13 +340,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (!SHARED || h == last_active) mma_commit(bar(BAR_K_EMPTY + kst));
         }
       }
-      for (int h = 0; h < 2 && ok; ++h) {
-        if (!slot[h].active) continue;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (!ok || !slot[h].active) continue;
         const int it = n - 1;
         const int vst = SHARED ? (it & 1) : h;
         const int vpar = SHARED ? ((it >> 1) & 1) : (it & 1);
         if (!mbar_wait(bar(BAR_P_FULL + h), it & 1, abort_flag, a.err) ||
-            !mbar_wait(bar(BAR_V_FULL + vst), vpar, abort_flag, a.err)) { ok = false; break; }
+            !mbar_wait(bar(BAR_V_FULL + vst), vpar, abort_flag, a.err)) { ok = false; continue; }
         tc_fence_after();
         issue_pv(h, vst, it > 0);
         mma_commit(bar(BAR_O_FULL + h));
@@ -347,12 +357,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_wait(bar(BAR_DRAIN), 0, nullptr, a.err);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 8) {
     // ====================================================== softmax slot h
+    setmaxnreg_inc<kSoftmaxRegs>();
     const int h = warp / 4;
     const int q = warp % 4;
     const int r = threadIdx.x % 128;                  // query row of the slot = TMEM lane
-    if (slot[h].active) {
+    Slot me;                                          // slot[h] without run-time indexing
+    me.active = h ? slot[1].active : slot[0].active;
+    me.bh = h ? slot[1].bh : slot[0].bh;
+    me.tile = h ? slot[1].tile : slot[0].tile;
+    me.t0 = h ? slot[1].t0 : slot[0].t0;
+    me.y0 = h ? slot[1].y0 : slot[0].y0;
+    me.x0 = h ? slot[1].x0 : slot[0].x0;
+    if (me.active) {
       const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
       const uint32_t tS = tmem + lane_base + 128u * h;
       const uint32_t tO = tmem + lane_base + 256u + 128u * h;
@@ -364,15 +382,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       {
         const int rr = r;
         const int lt = rr >> lg_yx, ly = (rr >> g.lg_tw) & (g.th - 1), lx = rr & (g.tw - 1);
-        tok_t = slot[h].t0 + lt;
-        tok_y = slot[h].y0 + ly;
-        tok_x = slot[h].x0 + lx;
+        tok_t = me.t0 + lt;
+        tok_y = me.y0 + ly;
+        tok_x = me.x0 + lx;
         row_valid = rr < box_rows && tok_t < g.T && tok_y < g.Hh && tok_x < g.W &&
                     lt < (SHARED ? a.box_t : g.tt);
       }
 
       KvSeq<SHARED> sq;
-      sq.init(a, slot[h].bh, slot[h].tile);
+      sq.init(a, me.bh, me.tile);
       const int n = sq.count(a);
       float m = -INFINITY, l = 0.f;
       bool ok = true;
@@ -381,27 +399,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         uint32_t mw[4] = {~0u, ~0u, ~0u, ~0u};
         bool full = true;
         {
-          int vt[2], vy[2], vx[2];
-          bool real[2];
-          for (int p = 0; p < P; ++p) {
-            int j, toff;
-            sq.piece(a, p, false, j, toff, real[p]);
-            const TileCoord c = tile_coord(g, j);
-            int et, ey, ex;
-            tile_extent(g, c, et, ey, ex);
-            vt[p] = SHARED ? min(a.box_t, et - toff) : et;
-            vy[p] = ey;
-            vx[p] = ex;
-            full = full && real[p] && vt[p] == (SHARED ? a.box_t : g.tt) && ey == g.th && ex == g.tw;
+          // extents of the (at most two) pieces, kept in scalars so that no
+          // array is indexed at run time
+          int vt0 = 0, vy0 = 0, vx0 = 0, vt1 = 0, vy1 = 0, vx1 = 0;
+          bool real0 = false, real1 = false;
+#pragma unroll
+          for (int p = 0; p < 2; ++p) {
+            if (p < P) {
+              int j, toff;
+              bool real;
+              sq.piece(a, p, false, j, toff, real);
+              const TileCoord c = tile_coord(g, j);
+              int et, ey, ex;
+              tile_extent(g, c, et, ey, ex);
+              const int vt = SHARED ? min(a.box_t, et - toff) : et;
+              full = full && real && vt == (SHARED ? a.box_t : g.tt) && ey == g.th && ex == g.tw;
+              if (p == 0) { vt0 = vt; vy0 = ey; vx0 = ex; real0 = real; }
+              else        { vt1 = vt; vy1 = ey; vx1 = ex; real1 = real; }
+            }
           }
           if (!full) {
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
               const int col = 32 * w + lane;
-              const int p = SHARED ? 0 : (col / g.vol);
-              const int rr = SHARED ? col : (col % g.vol);
+              const bool second = !SHARED && col >= g.vol;
+              const int rr = second ? col - g.vol : col;
               const int lt = rr >> lg_yx, ly = (rr >> g.lg_tw) & (g.th - 1), lx = rr & (g.tw - 1);
-              const bool v = p < P && real[p] && lt < vt[p] && ly < vy[p] && lx < vx[p];
+              const bool v = second ? (real1 && lt < vt1 && ly < vy1 && lx < vx1)
+                                    : (real0 && lt < vt0 && ly < vy0 && lx < vx0);
               mw[w] = __ballot_sync(0xffffffffu, v);
             }
           }
@@ -425,9 +450,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int c = 0; c < 128; ++c)
             if (!((mw[c >> 5] >> (c & 31)) & 1u)) s[c] = __float_as_uint(-INFINITY);
         }
-        float mx = __uint_as_float(s[0]);
+        // row max as a tree of 8 independent chains (short dependency depth)
+        float mx8[8];
 #pragma unroll
-        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
+        for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(s[e]);
+#pragma unroll
+        for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(s[c]));
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float mx_s = mx * a.scale_log2;
 
         // lazy rescale: move the reference max only when it grew by > 2^8
@@ -435,21 +465,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (it == 0) {
           m = mx_s;
         } else if (mx_s > m + kRescaleLog2) {
-          alpha = exp2f(m - mx_s);
+          alpha = ex2_approx(m - mx_s);
           m = mx_s;
           l *= alpha;
         }
         const bool rescale = __any_sync(0xffffffffu, alpha != 1.f);
         const float neg_m = -m;
-        float lsum = 0.f;
+        float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const float p0 = exp2f(fmaf(__uint_as_float(s[2 * c]), a.scale_log2, neg_m));
-          const float p1 = exp2f(fmaf(__uint_as_float(s[2 * c + 1]), a.scale_log2, neg_m));
-          lsum += p0 + p1;
+          const float p0 = ex2_approx(fmaf(__uint_as_float(s[2 * c]), a.scale_log2, neg_m));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(s[2 * c + 1]), a.scale_log2, neg_m));
+          ls8[c & 7] += p0 + p1;
           s[c] = pack_bf16x2(p0, p1);
         }
-        l += lsum;
+        l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
         tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
         tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
         if (rescale) {
@@ -476,7 +506,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const float inv_l = 1.f / l;
         const size_t N = static_cast<size_t>(g.T) * g.Hh * g.W;
         const size_t n_tok = (static_cast<size_t>(tok_t) * g.Hh + tok_y) * g.W + tok_x;
-        __nv_bfloat16* orow = a.o + (static_cast<size_t>(slot[h].bh) * N + n_tok) * D;
+        __nv_bfloat16* orow = a.o + (static_cast<size_t>(me.bh) * N + n_tok) * D;
 #pragma unroll
         for (int c4 = 0; c4 < D / 32; ++c4) {
           uint32_t ov[32];
@@ -493,7 +523,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
         if (row_valid)
-          a.lse[static_cast<size_t>(slot[h].bh) * N + n_tok] = (m + log2f(l)) * 0.69314718055994530942f;
+          a.lse[static_cast<size_t>(me.bh) * N + n_tok] = (m + log2f(l)) * 0.69314718055994530942f;
       }
     }
   }

@@ -75,23 +75,49 @@ static unsigned int* device_error_ptr() {
   return static_cast<unsigned int*>(p);
 }
 
+template <int R>
 static size_t score_smem_bytes(const Geom& g) {
-  return sizeof(float) * (kScoreRows * g.d + g.d * kKtStride) + sizeof(uint32_t) * (kScoreRows * g.nT + 8 * 256);
+  return sizeof(float) * (R * g.d + g.d * kKtStride) + sizeof(uint32_t) * (R * g.nT + 8 * 256);
+}
+
+template <int D, int R>
+static int launch_score(const Geom& g, int topk, int32_t* idx, const float* ws, cudaStream_t st) {
+  const size_t smem = score_smem_bytes<R>(g);
+  if (cudaFuncSetAttribute(score_topk_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return VSA_ERR_CUDA;
+  // programmatic dependent launch: the grid may start while pooling drains;
+  // its griddepcontrol.wait holds it until the pooled means are complete
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ceil_div(g.nT, R), g.B * g.H);
+  cfg.blockDim = dim3(kScoreThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, score_topk_kernel<D, R>, g, ws, topk, idx) == cudaSuccess ? VSA_OK
+                                                                                          : VSA_ERR_CUDA;
 }
 
 template <int D>
 static int launch_select(const Geom& g, const void* q, const void* k, int topk, int32_t* idx, float* ws,
                          cudaStream_t st) {
-  const int BH = g.B * g.H;
-  pool_kernel<D><<<dim3(g.nT, BH, 2), kPoolThreads, 0, st>>>(g, static_cast<const __nv_bfloat16*>(q),
-                                                            static_cast<const __nv_bfloat16*>(k), ws);
-  if (cudaGetLastError() != cudaSuccess) return VSA_ERR_CUDA;
-  const size_t smem = score_smem_bytes(g);
-  if (cudaFuncSetAttribute(score_topk_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
+  CUtensorMap mq, mk;
+  int rc;
+  if ((rc = encode_qkv_map(&mq, q, g, g.tt)) != VSA_OK || (rc = encode_qkv_map(&mk, k, g, g.tt)) != VSA_OK)
+    return rc;
+  unsigned int* err = device_error_ptr();
+  if (err == nullptr) return VSA_ERR_CUDA;
+  const size_t psmem = pool_smem_bytes<D>(g);
+  if (cudaFuncSetAttribute(pool_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(psmem)) != cudaSuccess)
     return VSA_ERR_CUDA;
-  score_topk_kernel<D><<<dim3(ceil_div(g.nT, kScoreRows), BH), kScoreThreads, smem, st>>>(g, ws, topk, idx);
-  return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+  pool_kernel<D><<<dim3(g.nT, g.B * g.H, 2), kPoolThreads, psmem, st>>>(mq, mk, g, ws, err);
+  if (cudaGetLastError() != cudaSuccess) return VSA_ERR_CUDA;
+  return g.nT <= 256 ? launch_score<D, 4>(g, topk, idx, ws, st) : launch_score<D, 16>(g, topk, idx, ws, st);
 }
 
 template <int D, bool SHARED>

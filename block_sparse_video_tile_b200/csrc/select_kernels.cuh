@@ -17,73 +17,94 @@
 #include <cstdint>
 #include <cuda_bf16.h>
 
+#include <cuda.h>
+
 #include "vsa_geometry.cuh"
+#include "vsa_ptx.cuh"
 
 namespace vsa {
 
 constexpr int kPoolThreads = 256;
 
-// One CTA per (tile j, head bh, tensor z in {Q, K}).  Threads split a row of d
-// bf16 values into 16-byte vectors (TPR threads per row) and stride over the
-// tile's valid rows; partial sums are combined in a fixed order, so the result
-// is deterministic.
+// One CTA per (tile j, head bh, tensor z in {Q, K}).  The whole tile is one
+// 5-D TMA box per 64-channel slab (the same [B*H, T, Hh, W, d] view the
+// attend kernel uses), so a 256-token tile of d = 128 puts 64 KB in flight
+// per CTA without using registers; positions past the grid edge arrive as
+// zeros and add nothing to the sums.  Threads then sum 16-byte chunks down the
+// rows in a fixed order (deterministic) and divide by the tile's valid count.
+// Dynamic shared memory: box (slabs x vol x 128 B, 1024-aligned) | partial sums | mbarrier.
 template <int D>
-__global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geom g, const __nv_bfloat16* __restrict__ q,
-                                                            const __nv_bfloat16* __restrict__ k,
-                                                            float* __restrict__ pooled) {
-  constexpr int TPR = D / 8;                 // threads per row (8 bf16 each)
-  constexpr int RP = kPoolThreads / TPR;     // rows in flight per pass
-  __shared__ float part[RP][D + 4];
+__global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                                            const __grid_constant__ CUtensorMap tmK, Geom g,
+                                                            float* __restrict__ pooled, unsigned int* err) {
+  constexpr int kSlabs = D / 64;
+  constexpr int TPR = D / 8;                 // threads per row (one 16-byte chunk each)
+  constexpr int RP = kPoolThreads / TPR;     // row groups
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* sp = smem_raw + (base - raw);
+  const int vol = g.vol;
+  const int box_bytes = vol * 128;
+  float* part = reinterpret_cast<float*>(sp + kSlabs * box_bytes);     // [RP][D]
+  const uint32_t bar = base + kSlabs * box_bytes + RP * D * 4;
 
   const int j = blockIdx.x;
   const int bh = blockIdx.y;
   const int z = blockIdx.z;
-  const __nv_bfloat16* src = (z == 0 ? q : k);
-  const size_t N = static_cast<size_t>(g.T) * g.Hh * g.W;
-  src += static_cast<size_t>(bh) * N * D;
-
   const TileCoord c = tile_coord(g, j);
-  int vt, vy, vx;
-  tile_extent(g, c, vt, vy, vx);
-  const int cnt = vt * vy * vx;
-  const int t0 = c.bt * g.tt, y0 = c.by * g.th, x0 = c.bx * g.tw;
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(kSlabs * box_bytes));
+    for (int sl = 0; sl < kSlabs; ++sl)
+      tma_load_5d(base + sl * box_bytes, z == 0 ? static_cast<const void*>(&tmQ) : static_cast<const void*>(&tmK),
+                  bar, sl * 64, c.bx * g.tw, c.by * g.th, c.bt * g.tt, bh);
+  }
+  // let the score kernel's launch begin while this grid drains
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __syncthreads();
+  const bool ok = mbar_wait(bar, 0, nullptr, err);
 
-  const int cg = threadIdx.x % TPR;
-  const int rl = threadIdx.x / TPR;
+  const int cc = threadIdx.x % TPR;          // 16-byte chunk of the row: slab cc/8, chunk cc%8
+  const int rg = threadIdx.x / TPR;
+  const unsigned char* slab = sp + (cc / 8) * box_bytes;
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-
-  const int vyx = vy * vx;
+  if (ok) {
 #pragma unroll 4
-  for (int r = rl; r < cnt; r += RP) {
-    const int lt = r / vyx;
-    const int rem = r - lt * vyx;
-    const int ly = rem / vx;
-    const int lx = rem - ly * vx;
-    const size_t n = (static_cast<size_t>(t0 + lt) * g.Hh + (y0 + ly)) * g.W + (x0 + lx);
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(src + n * D) + cg);
-    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+    for (int r = rg; r < vol; r += RP) {
+      const uint4 u = *reinterpret_cast<const uint4*>(slab + r * 128 + (((cc % 8) ^ (r & 7)) << 4));
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = __bfloat1622float2(h2[e]);
-      acc[2 * e] += f.x;
-      acc[2 * e + 1] += f.y;
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h2[e]);
+        acc[2 * e] += f.x;
+        acc[2 * e + 1] += f.y;
+      }
     }
   }
 #pragma unroll
-  for (int e = 0; e < 8; ++e) part[rl][cg * 8 + e] = acc[e];
+  for (int e = 0; e < 8; ++e) part[rg * D + cc * 8 + e] = acc[e];
   __syncthreads();
+  int vt, vy, vx;
+  tile_extent(g, c, vt, vy, vx);
+  const float cnt = static_cast<float>(vt * vy * vx);
   for (int col = threadIdx.x; col < D; col += kPoolThreads) {
-    float s = 0.f;
+    float sum = 0.f;
 #pragma unroll 8
-    for (int i = 0; i < RP; ++i) s += part[i][col];
-    pooled[((static_cast<size_t>(z) * g.B * g.H + bh) * g.nT + j) * D + col] = s / static_cast<float>(cnt);
+    for (int i = 0; i < RP; ++i) sum += part[i * D + col];
+    pooled[((static_cast<size_t>(z) * g.B * g.H + bh) * g.nT + j) * D + col] = sum / cnt;
   }
 }
 
+template <int D>
+inline size_t pool_smem_bytes(const Geom& g) {
+  return static_cast<size_t>(D / 64) * g.vol * 128 + (kPoolThreads / (D / 8)) * D * 4 + 16 + 1024;
+}
+
 constexpr int kScoreThreads = 256;  // 8 warps
-constexpr int kScoreRows = 16;      // query tiles per CTA (2 per warp for top-k)
 constexpr int kScoreChunk = 64;     // key tiles per shared-memory chunk
 constexpr int kKtStride = kScoreChunk + 1;  // padded row of the transposed chunk
 
@@ -94,10 +115,16 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
+// R query tiles per CTA (4 or 16: fewer rows give more CTAs when nT is small,
+// more rows amortise the key-mean reads when nT is large).
 // Dynamic shared memory: qb[R][D] | kT[D][CH+1] | keys[R][nT] (uint32) | hist[8][256]
-template <int D>
+template <int D, int R>
 __global__ void __launch_bounds__(kScoreThreads) score_topk_kernel(Geom g, const float* __restrict__ pooled,
                                                                    int topk, int32_t* __restrict__ idx) {
+  constexpr int kScoreRows = R;
+  constexpr int RPT = R / 4;               // rows per thread in the score phase
+  // wait until the pooling grid has finished and its writes are visible
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   extern __shared__ __align__(16) unsigned char smem_raw[];
   float* qb = reinterpret_cast<float*>(smem_raw);
   float* kT = qb + kScoreRows * D;
@@ -117,7 +144,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_topk_kernel(Geom g, const
     qb[e] = (r < nrows) ? qp[static_cast<size_t>(row0 + r) * D + (e % D)] : 0.f;
   }
 
-  // score phase: thread -> (column jj, 4 consecutive rows)
+  // score phase: thread -> (column jj, RPT consecutive rows)
   const int jj = threadIdx.x % kScoreChunk;
   const int rg = threadIdx.x / kScoreChunk;       // 0..3
   for (int c0 = 0; c0 < nT; c0 += kScoreChunk) {
@@ -133,33 +160,29 @@ __global__ void __launch_bounds__(kScoreThreads) score_topk_kernel(Geom g, const
       kT[(4 * k4 + 3) * kKtStride + cc] = v.w;
     }
     __syncthreads();
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    const float* q0 = qb + (rg * 4) * D;
+    float acc[RPT];
+#pragma unroll
+    for (int e = 0; e < RPT; ++e) acc[e] = 0.f;
+    const float* q0 = qb + (rg * RPT) * D;
 #pragma unroll 8
     for (int kk = 0; kk < D; ++kk) {
       const float kv = kT[kk * kKtStride + jj];
-      a0 = fmaf(q0[kk], kv, a0);
-      a1 = fmaf(q0[D + kk], kv, a1);
-      a2 = fmaf(q0[2 * D + kk], kv, a2);
-      a3 = fmaf(q0[3 * D + kk], kv, a3);
+#pragma unroll
+      for (int e = 0; e < RPT; ++e) acc[e] = fmaf(q0[e * D + kk], kv, acc[e]);
     }
     if (jj < ncol) {
-      uint32_t* kr = keys + (rg * 4) * nT + c0 + jj;
-      kr[0] = order_key(a0 + 0.f);
-      kr[nT] = order_key(a1 + 0.f);
-      kr[2 * nT] = order_key(a2 + 0.f);
-      kr[3 * nT] = order_key(a3 + 0.f);
+      uint32_t* kr = keys + (rg * RPT) * nT + c0 + jj;
+#pragma unroll
+      for (int e = 0; e < RPT; ++e) kr[e * nT] = order_key(acc[e] + 0.f);
     }
   }
   __syncthreads();
 
-  // top-k phase: warp w handles rows 2w, 2w+1 with an exact 4-pass radix select.
+  // top-k phase: warp w handles rows w, w + 8, ... with an exact 4-pass radix select.
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   uint32_t* hist = hist_all + warp * 256;
   const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int rr = 0; rr < 2; ++rr) {
-    const int r = warp * 2 + rr;
-    if (r >= nrows) break;
+  for (int r = warp; r < nrows; r += kScoreThreads / 32) {
     const uint32_t* kr = keys + r * nT;
     uint32_t prefix = 0, pmask = 0;
     int want = topk;  // rank (1-based) of the threshold among remaining candidates
