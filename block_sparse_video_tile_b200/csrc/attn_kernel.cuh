@@ -41,6 +41,13 @@ constexpr int kProducerRegs = 80;        // per thread, warpgroup 2 (TMA + MMA w
 constexpr int kSlotRows = 128;          // MMA M
 constexpr int kSubRows = 128;           // K/V rows per sub-block (S: N, PV: K)
 constexpr float kRescaleLog2 = 8.0f;
+#ifndef VSA_EXP_POLY_PER8
+#define VSA_EXP_POLY_PER8 0
+#endif
+// Of every 8 column pairs of a score row, this many take 2^x on the FMA pipe
+// (exp2_poly_pair) and the rest on the multi-function unit (ex2.approx): the
+// two units then share the softmax's exponentials.
+constexpr int kExpPolyPer8 = VSA_EXP_POLY_PER8;
 constexpr uint32_t kErrBadIndex = 2u;
 
 struct AttnArgs {
@@ -65,7 +72,9 @@ struct AttnSmem {
   static constexpr int kBar = 6 * kBufBytes;
   static constexpr int kNumBars = 17;
   static constexpr int kMisc = kBar + kNumBars * 8;
-  static constexpr int kTotal = kMisc + 16;
+  static constexpr int kTiles = kMisc + 16;           // uint2 per tile: (bt, by | bx << 16)
+  static constexpr int kMaxTiles = 2048;
+  static constexpr int kTotal = kTiles + 8 * kMaxTiles;
   static constexpr int kAlloc = kTotal + 1024;        // slack for 1024-byte alignment
 };
 
@@ -94,19 +103,31 @@ __device__ __forceinline__ int load_tile_index(const AttnArgs& a, const int32_t*
 //   SHARED: for each kept tile (ascending), its t-halves that hold any token.
 //   !SHARED: groups of P = 128 / vol kept tiles; a short last group repeats its
 //            last tile in the missing pieces (masked out).
+// Tile coordinates from the per-CTA table built at kernel start (one shared
+// memory load instead of integer divisions in every iteration).
+__device__ __forceinline__ TileCoord table_coord(const uint2* tab, int j) {
+  const uint2 e = tab[j];
+  TileCoord c;
+  c.bt = static_cast<int>(e.x);
+  c.by = static_cast<int>(e.y & 0xffffu);
+  c.bx = static_cast<int>(e.y >> 16);
+  return c;
+}
+
 template <bool SHARED>
 struct KvSeq {
   const int32_t* row;
+  const uint2* tab;
   int pos, half;
 
-  __device__ void init(const AttnArgs& a, int bh, int tile) {
+  __device__ void init(const AttnArgs& a, const uint2* table, int bh, int tile) {
     row = a.idx + (static_cast<size_t>(bh) * a.g.nT + tile) * a.topk;
+    tab = table;
     pos = 0;
     half = 0;
   }
-  __device__ static bool second_half(const AttnArgs& a, int j) {
-    const int bt = j / (a.g.nTy * a.g.nTx);
-    return bt * a.g.tt + a.box_t < a.g.T;
+  __device__ bool second_half(const AttnArgs& a, int j) const {
+    return static_cast<int>(tab[j].x) * a.g.tt + a.box_t < a.g.T;
   }
   __device__ int count(const AttnArgs& a) const {
     if (!SHARED) {
@@ -157,6 +178,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t sQ = base + L::kQ, sK = base + L::kK, sV = base + L::kV, sBar = base + L::kBar;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sp + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sp + L::kMisc + 4);
+  uint2* tile_tab = reinterpret_cast<uint2*>(sp + L::kTiles);
   auto bar = [&](int id) -> uint32_t { return sBar + 8u * static_cast<uint32_t>(id); };
 
   const Geom& g = a.g;
@@ -193,7 +215,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   const int last_active = slot[1].active ? 1 : 0;
 
-  // ---- setup: barriers, zero padding rows of Q, TMEM allocation
+  // ---- setup: tile table, barriers, zero padding rows of Q, TMEM allocation
+  for (int j = threadIdx.x; j < g.nT; j += kAttnThreads) {
+    const TileCoord c = tile_coord(g, j);
+    tile_tab[j] = make_uint2(static_cast<uint32_t>(c.bt),
+                             static_cast<uint32_t>(c.by) | (static_cast<uint32_t>(c.bx) << 16));
+  }
   if (threadIdx.x == 0) {
     for (int b = 0; b < L::kNumBars; ++b) {
       const bool p_bar = (b == BAR_P_FULL || b == BAR_P_FULL + 1);
@@ -228,7 +255,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   KvSeq<SHARED> seq;
-  seq.init(a, slot[0].bh, slot[0].tile);
+  seq.init(a, tile_tab, slot[0].bh, slot[0].tile);
 
   if (warp >= 8) {
     setmaxnreg_dec<kProducerRegs>();
@@ -245,8 +272,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                       slot[h].x0, slot[h].y0, slot[h].t0, slot[h].bh);
       }
       KvSeq<SHARED> sq[2];
-      sq[0].init(a, slot[0].bh, slot[0].tile);
-      sq[1].init(a, slot[1].bh, slot[1].tile);
+      sq[0].init(a, tile_tab, slot[0].bh, slot[0].tile);
+      sq[1].init(a, tile_tab, slot[1].bh, slot[1].tile);
       const int n = sq[0].count(a);
       int last_use[2][2] = {{-1, -1}, {-1, -1}};   // [K/V][stage]: last phase issued
       for (int it = 0; it < n && ok; ++it) {
@@ -269,7 +296,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               int j, toff;
               bool real;
               sq[h].piece(a, p, kv == 0, j, toff, real);
-              const TileCoord c = tile_coord(g, j);
+              const TileCoord c = table_coord(tile_tab, j);
               for (int sl = 0; sl < L::kSlabs; ++sl)
                 tma_load_5d(buf0 + st * L::kBufBytes + sl * L::kSlabBytes + p * box_bytes, tm,
                             bar(full + st), sl * 64, c.bx * g.tw, c.by * g.th, c.bt * g.tt + toff,
@@ -390,7 +417,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
 
       KvSeq<SHARED> sq;
-      sq.init(a, me.bh, me.tile);
+      sq.init(a, tile_tab, me.bh, me.tile);
       const int n = sq.count(a);
       float m = -INFINITY, l = 0.f;
       bool ok = true;
@@ -409,7 +436,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               int j, toff;
               bool real;
               sq.piece(a, p, false, j, toff, real);
-              const TileCoord c = tile_coord(g, j);
+              const TileCoord c = table_coord(tile_tab, j);
               int et, ey, ex;
               tile_extent(g, c, et, ey, ex);
               const int vt = SHARED ? min(a.box_t, et - toff) : et;
@@ -450,14 +477,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int c = 0; c < 128; ++c)
             if (!((mw[c >> 5] >> (c & 31)) & 1u)) s[c] = __float_as_uint(-INFINITY);
         }
-        // row max as a tree of 8 independent chains (short dependency depth)
+        // row max as a tree of 8 independent chains of 3-input max (short depth)
         float mx8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(s[e]);
 #pragma unroll
-        for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(s[c]));
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        for (int c = 8; c < 128; c += 2)
+          mx8[(c >> 1) & 7] = fmax3(mx8[(c >> 1) & 7], __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
         const float mx_s = mx * a.scale_log2;
 
         // lazy rescale: move the reference max only when it grew by > 2^8
@@ -470,16 +497,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           l *= alpha;
         }
         const bool rescale = __any_sync(0xffffffffu, alpha != 1.f);
-        const float neg_m = -m;
-        float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        // P = 2^(scale*log2(e)*S - m) on pairs of columns; row sum in 4 packed chains
+        const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
+        const uint64_t nm2 = f2_pack(-m, -m);
+        uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(s[2 * c]), a.scale_log2, neg_m));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(s[2 * c + 1]), a.scale_log2, neg_m));
-          ls8[c & 7] += p0 + p1;
+          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), sc2, nm2);
+          float p0, p1;
+          if ((c & 7) < kExpPolyPer8) {
+            exp2_poly_pair(x2, p0, p1);
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          ls2[c & 3] = f2_add(ls2[c & 3], f2_pack(p0, p1));
           s[c] = pack_bf16x2(p0, p1);
         }
-        l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
+        {
+          float a0, a1;
+          f2_unpack(f2_add(f2_add(ls2[0], ls2[1]), f2_add(ls2[2], ls2[3])), a0, a1);
+          l += a0 + a1;
+        }
         tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
         tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
         if (rescale) {
@@ -517,13 +558,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
             for (int e = 0; e < 16; ++e)
               pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l, __uint_as_float(ov[2 * e + 1]) * inv_l);
+            // streaming stores: O is not read again by this kernel, so it
+            // should not sit dirty in L2 for whatever kernel runs next
             uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c4);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            for (int e = 0; e < 4; ++e) __stcs(dst + e, make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]));
           }
         }
         if (row_valid)
-          a.lse[static_cast<size_t>(me.bh) * N + n_tok] = (m + log2f(l)) * 0.69314718055994530942f;
+          __stcs(a.lse + static_cast<size_t>(me.bh) * N + n_tok, (m + log2f(l)) * 0.69314718055994530942f);
       }
     }
   }

@@ -80,11 +80,16 @@ static size_t score_smem_bytes(const Geom& g) {
   return sizeof(float) * (R * g.d + g.d * kKtStride) + sizeof(uint32_t) * (R * g.nT + 8 * 256);
 }
 
+// Up to 256 tiles: 8 query tiles per CTA with every key mean in shared memory.
+// More tiles: 16 query tiles per CTA, key means streamed in chunks.
 template <int D, int R>
 static int launch_score(const Geom& g, int topk, int32_t* idx, const float* ws, cudaStream_t st) {
-  const size_t smem = score_smem_bytes<R>(g);
-  if (cudaFuncSetAttribute(score_topk_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
+  const bool small = R == 8;
+  const size_t smem = small ? sizeof(float) * (8 * g.d + g.nT * g.d) + sizeof(uint32_t) * (8 * g.nT + 8 * 256)
+                            : score_smem_bytes<R>(g);
+  auto kernel = small ? score_topk_small_kernel<D> : score_topk_kernel<D, (R == 8 ? 16 : R)>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
     return VSA_ERR_CUDA;
   // programmatic dependent launch: the grid may start while pooling drains;
   // its griddepcontrol.wait holds it until the pooled means are complete
@@ -98,8 +103,7 @@ static int launch_score(const Geom& g, int topk, int32_t* idx, const float* ws, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, score_topk_kernel<D, R>, g, ws, topk, idx) == cudaSuccess ? VSA_OK
-                                                                                          : VSA_ERR_CUDA;
+  return cudaLaunchKernelEx(&cfg, kernel, g, ws, topk, idx) == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 
 template <int D>
@@ -117,7 +121,7 @@ static int launch_select(const Geom& g, const void* q, const void* k, int topk, 
     return VSA_ERR_CUDA;
   pool_kernel<D><<<dim3(g.nT, g.B * g.H, 2), kPoolThreads, psmem, st>>>(mq, mk, g, ws, err);
   if (cudaGetLastError() != cudaSuccess) return VSA_ERR_CUDA;
-  return g.nT <= 256 ? launch_score<D, 4>(g, topk, idx, ws, st) : launch_score<D, 16>(g, topk, idx, ws, st);
+  return g.nT <= 256 ? launch_score<D, 8>(g, topk, idx, ws, st) : launch_score<D, 16>(g, topk, idx, ws, st);
 }
 
 template <int D, bool SHARED>

@@ -115,6 +115,75 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
+// Exact top-k of one row of order keys by one warp: a 4-pass 8-bit radix
+// select finds the topk-th largest key; every larger key and the first equal
+// keys (lowest tile index first) are then written in ascending tile order.
+__device__ __forceinline__ void radix_topk_row(const uint32_t* kr, int nT, int topk, uint32_t* hist,
+                                               int32_t* out) {
+  const int lane = threadIdx.x % 32;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  uint32_t prefix = 0, pmask = 0;
+  int want = topk;  // rank (1-based) of the threshold among remaining candidates
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = lane; b < 256; b += 32) hist[b] = 0;
+    __syncwarp();
+    for (int jx = lane; jx < nT; jx += 32) {
+      const uint32_t u = kr[jx];
+      if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+    }
+    __syncwarp();
+    // lane l owns bins 255-8l .. 248-8l (descending digit order)
+    uint32_t cnt8[8];
+    uint32_t tot = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      cnt8[e] = hist[255 - 8 * lane - e];
+      tot += cnt8[e];
+    }
+    uint32_t incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    uint32_t above = incl - tot;  // candidates with a larger digit than my bins
+    int found_digit = -1;
+    uint32_t found_above = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      if (found_digit < 0 && above < static_cast<uint32_t>(want) &&
+          above + cnt8[e] >= static_cast<uint32_t>(want)) {
+        found_digit = 255 - 8 * lane - e;
+        found_above = above;
+      }
+      above += cnt8[e];
+    }
+    const uint32_t who = __ballot_sync(0xffffffffu, found_digit >= 0);
+    const int src = __ffs(who) - 1;
+    found_digit = __shfl_sync(0xffffffffu, found_digit, src);
+    found_above = __shfl_sync(0xffffffffu, found_above, src);
+    want -= static_cast<int>(found_above);
+    prefix |= static_cast<uint32_t>(found_digit) << shift;
+    pmask |= 255u << shift;
+    __syncwarp();
+  }
+  // prefix is the topk-th largest key; take every larger key and the first
+  // `want` keys equal to it (lowest tile index first), in ascending order.
+  int base = 0, eq_seen = 0;
+  for (int j0 = 0; j0 < nT; j0 += 32) {
+    const int jx = j0 + lane;
+    const uint32_t u = (jx < nT) ? kr[jx] : 0u;
+    const bool gt = (jx < nT) && (u > prefix);
+    const bool eq = (jx < nT) && (u == prefix);
+    const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+    const bool take = gt || (eq && (eq_seen + __popc(eqm & lt_mask)) < want);
+    const uint32_t tm = __ballot_sync(0xffffffffu, take);
+    if (take) out[base + __popc(tm & lt_mask)] = jx;
+    base += __popc(tm);
+    eq_seen += __popc(eqm);
+  }
+}
+
 // R query tiles per CTA (4 or 16: fewer rows give more CTAs when nT is small,
 // more rows amortise the key-mean reads when nT is large).
 // Dynamic shared memory: qb[R][D] | kT[D][CH+1] | keys[R][nT] (uint32) | hist[8][256]
@@ -178,74 +247,65 @@ __global__ void __launch_bounds__(kScoreThreads) score_topk_kernel(Geom g, const
   }
   __syncthreads();
 
-  // top-k phase: warp w handles rows w, w + 8, ... with an exact 4-pass radix select.
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  uint32_t* hist = hist_all + warp * 256;
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int r = warp; r < nrows; r += kScoreThreads / 32) {
-    const uint32_t* kr = keys + r * nT;
-    uint32_t prefix = 0, pmask = 0;
-    int want = topk;  // rank (1-based) of the threshold among remaining candidates
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int b = lane; b < 256; b += 32) hist[b] = 0;
-      __syncwarp();
-      for (int jx = lane; jx < nT; jx += 32) {
-        const uint32_t u = kr[jx];
-        if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
-      }
-      __syncwarp();
-      // lane l owns bins 255-8l .. 248-8l (descending digit order)
-      uint32_t cnt8[8];
-      uint32_t tot = 0;
+  // top-k phase: warp w handles rows w, w + 8, ...
+  const int warp = threadIdx.x / 32;
+  for (int r = warp; r < nrows; r += kScoreThreads / 32)
+    radix_topk_row(keys + r * nT, nT, topk, hist_all + warp * 256,
+                   idx + (static_cast<size_t>(bh) * nT + row0 + r) * topk);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kScoreThreads) score_topk_small_kernel(Geom g, const float* __restrict__ pooled,
+                                                                         int topk, int32_t* __restrict__ idx) {
+  constexpr int R = 8;
+  constexpr int C4 = D / 4;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int nT = g.nT;
+  float4* qb = reinterpret_cast<float4*>(smem_raw);
+  float4* kb = qb + R * C4;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(kb + nT * C4);
+  uint32_t* hist_all = keys + R * nT;
+
+  const int bh = blockIdx.y;
+  const int row0 = blockIdx.x * R;
+  const int nrows = min(R, nT - row0);
+  const size_t BH = static_cast<size_t>(g.B) * g.H;
+  const float4* qp = reinterpret_cast<const float4*>(pooled + (static_cast<size_t>(bh) * nT + row0) * D);
+  const float4* kp = reinterpret_cast<const float4*>(pooled + ((BH + bh) * nT) * D);
+  for (int e = threadIdx.x; e < R * C4; e += kScoreThreads)
+    qb[e] = (e / C4 < nrows) ? qp[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int e = threadIdx.x; e < nT * C4; e += kScoreThreads) kb[e] = kp[e];
+  __syncthreads();
+
+  const int lane = threadIdx.x % 32;
+  for (int j = threadIdx.x; j < nT; j += kScoreThreads) {
+    float acc[R];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        cnt8[e] = hist[255 - 8 * lane - e];
-        tot += cnt8[e];
-      }
-      uint32_t incl = tot;
+    for (int r = 0; r < R; ++r) acc[r] = 0.f;
+    const float4* krow = kb + j * C4;
+#pragma unroll 4
+    for (int i = 0; i < C4; ++i) {
+      const int c = (i + lane) % C4;
+      const float4 kv = krow[c];
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
+      for (int r = 0; r < R; ++r) {
+        const float4 qv = qb[r * C4 + c];
+        acc[r] = fmaf(qv.x, kv.x, acc[r]);
+        acc[r] = fmaf(qv.y, kv.y, acc[r]);
+        acc[r] = fmaf(qv.z, kv.z, acc[r]);
+        acc[r] = fmaf(qv.w, kv.w, acc[r]);
       }
-      uint32_t above = incl - tot;  // candidates with a larger digit than my bins
-      int found_digit = -1;
-      uint32_t found_above = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if (found_digit < 0 && above < static_cast<uint32_t>(want) &&
-            above + cnt8[e] >= static_cast<uint32_t>(want)) {
-          found_digit = 255 - 8 * lane - e;
-          found_above = above;
-        }
-        above += cnt8[e];
-      }
-      const uint32_t who = __ballot_sync(0xffffffffu, found_digit >= 0);
-      const int src = __ffs(who) - 1;
-      found_digit = __shfl_sync(0xffffffffu, found_digit, src);
-      found_above = __shfl_sync(0xffffffffu, found_above, src);
-      want -= static_cast<int>(found_above);
-      prefix |= static_cast<uint32_t>(found_digit) << shift;
-      pmask |= 255u << shift;
-      __syncwarp();
     }
-    // prefix is the topk-th largest key; take every larger key and the first
-    // `want` keys equal to it (lowest tile index first), in ascending order.
-    int32_t* out = idx + (static_cast<size_t>(bh) * nT + row0 + r) * topk;
-    int base = 0, eq_seen = 0;
-    for (int j0 = 0; j0 < nT; j0 += 32) {
-      const int jx = j0 + lane;
-      const uint32_t u = (jx < nT) ? kr[jx] : 0u;
-      const bool gt = (jx < nT) && (u > prefix);
-      const bool eq = (jx < nT) && (u == prefix);
-      const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
-      const bool take = gt || (eq && (eq_seen + __popc(eqm & lt_mask)) < want);
-      const uint32_t tm = __ballot_sync(0xffffffffu, take);
-      if (take) out[base + __popc(tm & lt_mask)] = jx;
-      base += __popc(tm);
-      eq_seen += __popc(eqm);
-    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) keys[r * nT + j] = order_key(acc[r] + 0.f);
   }
+  __syncthreads();
+
+  const int warp = threadIdx.x / 32;
+  if (warp < nrows)
+    radix_topk_row(keys + warp * nT, nT, topk, hist_all + warp * 256,
+                   idx + (static_cast<size_t>(bh) * nT + row0 + warp) * topk);
 }
 
 }  // namespace vsa

@@ -169,6 +169,20 @@ __global__ void diag_mma_ts_kernel(const uint32_t* P, const uint4* V, float* O, 
   }
 }
 
+__global__ void diag_exp2_kernel(const float* x, float* y_poly, float* y_mufu, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 >= n + 1) return;
+  const float a = x[i], b = (i + 1 < n) ? x[i + 1] : 0.f;
+  float p0, p1;
+  exp2_poly_pair(f2_pack(a, b), p0, p1);
+  y_poly[i] = p0;
+  y_mufu[i] = ex2_approx(a);
+  if (i + 1 < n) {
+    y_poly[i + 1] = p1;
+    y_mufu[i + 1] = ex2_approx(b);
+  }
+}
+
 static unsigned int* diag_err() {
   void* p = nullptr;
   if (cudaGetSymbolAddress(&p, g_diag_error) != cudaSuccess) return nullptr;
@@ -232,6 +246,13 @@ int vsa_diag_mma_ts(const void* P, const void* V, int32_t d, float* O, void* str
   } else {
     return VSA_ERR_UNSUPPORTED;
   }
+  return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
+// 2^x of n floats by the FMA-pipe polynomial (y_poly) and by ex2.approx (y_mufu).
+int vsa_diag_exp2(const float* x, float* y_poly, float* y_mufu, int32_t n, void* stream) {
+  const int pairs = (n + 1) / 2;
+  diag_exp2_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_poly, y_mufu, n);
   return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 

@@ -215,6 +215,64 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// ---------------------------------------------------- packed float32 pairs
+// sm_100 executes add/fma on two float32 lanes in one instruction.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair of float32 on the FMA pipe (no multi-function unit): x is
+// split as j + f with j = round(x) and f in [-1/2, 1/2] (Cody-Waite); 2^f is a
+// degree-3 polynomial fitted to minimise the relative error on [-1/2, 1/2]
+// (fit_exp2_poly.py, max relative error 7.5e-5, below the bfloat16 rounding
+// the probabilities get next); 2^j is added to the exponent field.  Inputs
+// below -125 (including -inf) give exactly 0; inputs are at most 2^8 here.
+__device__ __forceinline__ void exp2_poly_pair(uint64_t x2, float& p0, float& p1) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
+  const uint64_t magic2 = f2_pack(kMagic, kMagic);
+  const uint64_t nmagic2 = f2_pack(-kMagic, -kMagic);
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t2 = f2_add(xc, magic2);             // j + magic, j in the low mantissa bits
+  const uint64_t j2 = f2_add(t2, nmagic2);            // j as a float
+  float ja, jb;
+  f2_unpack(j2, ja, jb);
+  const uint64_t f2 = f2_add(xc, f2_pack(-ja, -jb));   // f = x - j
+  uint64_t q = f2_fma(f2_pack(5.517166853e-02f, 5.517166853e-02f), f2,
+                      f2_pack(2.426111251e-01f, 2.426111251e-01f));
+  q = f2_fma(q, f2, f2_pack(6.932609677e-01f, 6.932609677e-01f));
+  q = f2_fma(q, f2, f2_pack(9.999280572e-01f, 9.999280572e-01f));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t2, t0, t1);
+  // the low bits of t hold j (two's complement); j << 23 scales by 2^j
+  const float r0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  const float r1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+  p0 = x0 < -125.f ? 0.f : r0;
+  p1 = x1 < -125.f ? 0.f : r1;
+}
+
 // Per-warpgroup register budget changes (all warps of a warpgroup execute the
 // same one).  The totals must stay within the launch budget.
 template <int N>
