@@ -19,7 +19,7 @@ namespace vsa {
 
 __device__ unsigned int g_device_error = 0u;
 
-constexpr int kMaxTiles = 2048;          // score rows of one CTA must fit in shared memory
+constexpr int kMaxTiles = 1536;          // score rows of one CTA must fit in shared memory
 constexpr int kMaxDevices = 64;
 
 // -------------------------------------------------------------- validation
@@ -75,21 +75,13 @@ static unsigned int* device_error_ptr() {
   return static_cast<unsigned int*>(p);
 }
 
-template <int R>
-static size_t score_smem_bytes(const Geom& g) {
-  return sizeof(float) * (R * g.d + g.d * kKtStride) + sizeof(uint32_t) * (R * g.nT + 8 * 256);
-}
-
-// Up to 256 tiles: 8 query tiles per CTA with every key mean in shared memory.
-// More tiles: 16 query tiles per CTA, key means streamed in chunks.
+// Score + top-k grid: 8 query tiles per CTA up to 256 tiles per head, else
+// 16 (more reuse of each staged key-mean chunk).
 template <int D, int R>
 static int launch_score(const Geom& g, int topk, int32_t* idx, const float* ws, cudaStream_t st) {
-  const bool small = R == 8;
-  const size_t smem = small ? sizeof(float) * (8 * g.d + g.nT * g.d) + sizeof(uint32_t) * (8 * g.nT + 8 * 256)
-                            : score_smem_bytes<R>(g);
-  auto kernel = small ? score_topk_small_kernel<D> : score_topk_kernel<D, (R == 8 ? 16 : R)>;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-      cudaSuccess)
+  const size_t smem = score_smem_bytes<D, R>(g);
+  if (cudaFuncSetAttribute(score_topk_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
     return VSA_ERR_CUDA;
   // programmatic dependent launch: the grid may start while pooling drains;
   // its griddepcontrol.wait holds it until the pooled means are complete
@@ -103,7 +95,8 @@ static int launch_score(const Geom& g, int topk, int32_t* idx, const float* ws, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, g, ws, topk, idx) == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+  return cudaLaunchKernelEx(&cfg, score_topk_kernel<D, R>, g, ws, topk, idx) == cudaSuccess ? VSA_OK
+                                                                                               : VSA_ERR_CUDA;
 }
 
 template <int D>

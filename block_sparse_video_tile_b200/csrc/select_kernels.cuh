@@ -11,7 +11,7 @@
 //                 means (float32 [2, B*H, nT, d]) to the caller's workspace.
 //   score_topk_kernel: per (head, block of query tiles) computes the score
 //                 rows into shared memory (float32 FMA in a fixed order) and
-//                 runs an exact radix select per row; writes ascending idx.
+//                 selects each row's top-k exactly; writes ascending idx.
 #pragma once
 
 #include <cstdint>
@@ -105,8 +105,6 @@ inline size_t pool_smem_bytes(const Geom& g) {
 }
 
 constexpr int kScoreThreads = 256;  // 8 warps
-constexpr int kScoreChunk = 64;     // key tiles per shared-memory chunk
-constexpr int kKtStride = kScoreChunk + 1;  // padded row of the transposed chunk
 
 // Larger float -> larger unsigned key (total order; -0 < +0, scores are
 // canonicalised so -0 does not occur).
@@ -115,157 +113,84 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-// Exact top-k of one row of order keys by one warp: a 4-pass 8-bit radix
-// select finds the topk-th largest key; every larger key and the first equal
-// keys (lowest tile index first) are then written in ascending tile order.
-__device__ __forceinline__ void radix_topk_row(const uint32_t* kr, int nT, int topk, uint32_t* hist,
-                                               int32_t* out) {
+// Exact top-k of one row of order keys by one warp, keys held in registers
+// (lane l holds tiles l, l + 32, ...).  The topk-th largest key T is found
+// bit by bit from the top: T keeps a bit when at least topk keys are >= T
+// with that bit set (a warp-wide count per bit, no shared-memory atomics).
+// Every key above T is taken, then the keys equal to T in ascending tile
+// order until topk are taken (ties go to the lower tile index); indices are
+// written in ascending order.  Order keys of finite scores are never 0, so 0
+// marks the padding slots.
+template <int MAXE>
+__device__ __forceinline__ void bsearch_topk_row(const uint32_t* kr, int nT, int topk, int32_t* out) {
   const int lane = threadIdx.x % 32;
   const uint32_t lt_mask = (1u << lane) - 1u;
-  uint32_t prefix = 0, pmask = 0;
-  int want = topk;  // rank (1-based) of the threshold among remaining candidates
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int b = lane; b < 256; b += 32) hist[b] = 0;
-    __syncwarp();
-    for (int jx = lane; jx < nT; jx += 32) {
-      const uint32_t u = kr[jx];
-      if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
-    }
-    __syncwarp();
-    // lane l owns bins 255-8l .. 248-8l (descending digit order)
-    uint32_t cnt8[8];
-    uint32_t tot = 0;
+  uint32_t key[MAXE];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      cnt8[e] = hist[255 - 8 * lane - e];
-      tot += cnt8[e];
-    }
-    uint32_t incl = tot;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    uint32_t above = incl - tot;  // candidates with a larger digit than my bins
-    int found_digit = -1;
-    uint32_t found_above = 0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      if (found_digit < 0 && above < static_cast<uint32_t>(want) &&
-          above + cnt8[e] >= static_cast<uint32_t>(want)) {
-        found_digit = 255 - 8 * lane - e;
-        found_above = above;
-      }
-      above += cnt8[e];
-    }
-    const uint32_t who = __ballot_sync(0xffffffffu, found_digit >= 0);
-    const int src = __ffs(who) - 1;
-    found_digit = __shfl_sync(0xffffffffu, found_digit, src);
-    found_above = __shfl_sync(0xffffffffu, found_above, src);
-    want -= static_cast<int>(found_above);
-    prefix |= static_cast<uint32_t>(found_digit) << shift;
-    pmask |= 255u << shift;
-    __syncwarp();
+  for (int e = 0; e < MAXE; ++e) {
+    const int j = lane + 32 * e;
+    key[e] = (j < nT) ? kr[j] : 0u;
   }
-  // prefix is the topk-th largest key; take every larger key and the first
-  // `want` keys equal to it (lowest tile index first), in ascending order.
+  uint32_t T = 0;
+  for (int b = 31; b >= 0; --b) {
+    const uint32_t cand = T | (1u << b);
+    uint32_t c = 0;
+#pragma unroll
+    for (int e = 0; e < MAXE; ++e) c += (key[e] >= cand) ? 1u : 0u;
+    c = __reduce_add_sync(0xffffffffu, c);
+    if (c >= static_cast<uint32_t>(topk)) T = cand;
+  }
+  uint32_t gt = 0;
+#pragma unroll
+  for (int e = 0; e < MAXE; ++e) gt += (key[e] > T) ? 1u : 0u;
+  gt = __reduce_add_sync(0xffffffffu, gt);
+  const int want_eq = topk - static_cast<int>(gt);
   int base = 0, eq_seen = 0;
-  for (int j0 = 0; j0 < nT; j0 += 32) {
-    const int jx = j0 + lane;
-    const uint32_t u = (jx < nT) ? kr[jx] : 0u;
-    const bool gt = (jx < nT) && (u > prefix);
-    const bool eq = (jx < nT) && (u == prefix);
-    const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
-    const bool take = gt || (eq && (eq_seen + __popc(eqm & lt_mask)) < want);
+#pragma unroll
+  for (int e = 0; e < MAXE; ++e) {
+    if (32 * e >= nT) break;
+    const bool gtb = key[e] > T;
+    const bool eqb = key[e] == T;
+    const uint32_t eqm = __ballot_sync(0xffffffffu, eqb);
+    const bool take = gtb || (eqb && eq_seen + __popc(eqm & lt_mask) < want_eq);
     const uint32_t tm = __ballot_sync(0xffffffffu, take);
-    if (take) out[base + __popc(tm & lt_mask)] = jx;
+    if (take) out[base + __popc(tm & lt_mask)] = lane + 32 * e;
     base += __popc(tm);
     eq_seen += __popc(eqm);
   }
 }
 
-// R query tiles per CTA (4 or 16: fewer rows give more CTAs when nT is small,
-// more rows amortise the key-mean reads when nT is large).
-// Dynamic shared memory: qb[R][D] | kT[D][CH+1] | keys[R][nT] (uint32) | hist[8][256]
+// Tile scores and top-k.  One CTA takes R query tiles of one head (R = 8 when
+// the head has at most 256 tiles, else 16).  Their pooled Q means and the
+// pooled K means, in chunks of up to 64 key tiles (rows padded to d + 4
+// floats), are copied to shared memory with vector loads.  Thread t =
+// (quarter, j) forms, for key tile j of the chunk and all R query tiles, the
+// partial dot product over its quarter of the d channels: the padded rows make
+// the key reads of a quarter-warp hit 8 different bank groups, and the query
+// reads are warp-wide broadcasts.  The four partial sums are added in a fixed
+// order (deterministic); the score rows stay in shared memory as order keys,
+// and one warp per row selects its top-k.  Shared memory stays under 76 KB
+// for up to 256 tiles, so three CTAs fit on an SM.
+// Dynamic shared memory: qb[R][D] | kb[min(nT,64)][D+4] | part[4][R][64] | keys[R][nT]
+constexpr int kScoreChunk = 64;
+constexpr int kScoreSplit = kScoreThreads / kScoreChunk;   // d split in 4 parts
+
 template <int D, int R>
 __global__ void __launch_bounds__(kScoreThreads) score_topk_kernel(Geom g, const float* __restrict__ pooled,
                                                                    int topk, int32_t* __restrict__ idx) {
-  constexpr int kScoreRows = R;
-  constexpr int RPT = R / 4;               // rows per thread in the score phase
-  // wait until the pooling grid has finished and its writes are visible
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  float* qb = reinterpret_cast<float*>(smem_raw);
-  float* kT = qb + kScoreRows * D;
-  uint32_t* keys = reinterpret_cast<uint32_t*>(kT + D * kKtStride);
-  uint32_t* hist_all = keys + kScoreRows * g.nT;
-
-  const int nT = g.nT;
-  const int bh = blockIdx.y;
-  const int row0 = blockIdx.x * kScoreRows;
-  const int nrows = min(kScoreRows, nT - row0);
-  const size_t BH = static_cast<size_t>(g.B) * g.H;
-  const float* qp = pooled + (static_cast<size_t>(bh) * nT) * D;
-  const float* kp = pooled + ((BH + bh) * nT) * D;
-
-  for (int e = threadIdx.x; e < kScoreRows * D; e += kScoreThreads) {
-    const int r = e / D;
-    qb[e] = (r < nrows) ? qp[static_cast<size_t>(row0 + r) * D + (e % D)] : 0.f;
-  }
-
-  // score phase: thread -> (column jj, RPT consecutive rows)
-  const int jj = threadIdx.x % kScoreChunk;
-  const int rg = threadIdx.x / kScoreChunk;       // 0..3
-  for (int c0 = 0; c0 < nT; c0 += kScoreChunk) {
-    __syncthreads();
-    const int ncol = min(kScoreChunk, nT - c0);
-    for (int e = threadIdx.x; e < kScoreChunk * (D / 4); e += kScoreThreads) {
-      const int cc = e / (D / 4), k4 = e % (D / 4);
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (cc < ncol) v = *reinterpret_cast<const float4*>(kp + static_cast<size_t>(c0 + cc) * D + 4 * k4);
-      kT[(4 * k4 + 0) * kKtStride + cc] = v.x;
-      kT[(4 * k4 + 1) * kKtStride + cc] = v.y;
-      kT[(4 * k4 + 2) * kKtStride + cc] = v.z;
-      kT[(4 * k4 + 3) * kKtStride + cc] = v.w;
-    }
-    __syncthreads();
-    float acc[RPT];
-#pragma unroll
-    for (int e = 0; e < RPT; ++e) acc[e] = 0.f;
-    const float* q0 = qb + (rg * RPT) * D;
-#pragma unroll 8
-    for (int kk = 0; kk < D; ++kk) {
-      const float kv = kT[kk * kKtStride + jj];
-#pragma unroll
-      for (int e = 0; e < RPT; ++e) acc[e] = fmaf(q0[e * D + kk], kv, acc[e]);
-    }
-    if (jj < ncol) {
-      uint32_t* kr = keys + (rg * RPT) * nT + c0 + jj;
-#pragma unroll
-      for (int e = 0; e < RPT; ++e) kr[e * nT] = order_key(acc[e] + 0.f);
-    }
-  }
-  __syncthreads();
-
-  // top-k phase: warp w handles rows w, w + 8, ...
-  const int warp = threadIdx.x / 32;
-  for (int r = warp; r < nrows; r += kScoreThreads / 32)
-    radix_topk_row(keys + r * nT, nT, topk, hist_all + warp * 256,
-                   idx + (static_cast<size_t>(bh) * nT + row0 + r) * topk);
-}
-
-template <int D>
-__global__ void __launch_bounds__(kScoreThreads) score_topk_small_kernel(Geom g, const float* __restrict__ pooled,
-                                                                         int topk, int32_t* __restrict__ idx) {
-  constexpr int R = 8;
+  constexpr int KS = D + 4;                 // padded key-mean row (floats)
   constexpr int C4 = D / 4;
+  constexpr int PART4 = D / 4 / kScoreSplit;  // float4 chunks per part of a row
+  constexpr int MAXE = (R == 8) ? 8 : 48;   // keys per lane in the top-k (nT <= 256 / <= 1536)
+  // the pooled means are written by the previous grid: wait for it
   asm volatile("griddepcontrol.wait;" ::: "memory");
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int nT = g.nT;
-  float4* qb = reinterpret_cast<float4*>(smem_raw);
-  float4* kb = qb + R * C4;
-  uint32_t* keys = reinterpret_cast<uint32_t*>(kb + nT * C4);
-  uint32_t* hist_all = keys + R * nT;
+  const int chunk = min(nT, kScoreChunk);
+  float* qb = reinterpret_cast<float*>(smem_raw);
+  float* kb = qb + R * D;
+  float* part = kb + chunk * KS;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(part + kScoreSplit * R * kScoreChunk);
 
   const int bh = blockIdx.y;
   const int row0 = blockIdx.x * R;
@@ -273,39 +198,63 @@ __global__ void __launch_bounds__(kScoreThreads) score_topk_small_kernel(Geom g,
   const size_t BH = static_cast<size_t>(g.B) * g.H;
   const float4* qp = reinterpret_cast<const float4*>(pooled + (static_cast<size_t>(bh) * nT + row0) * D);
   const float4* kp = reinterpret_cast<const float4*>(pooled + ((BH + bh) * nT) * D);
-  for (int e = threadIdx.x; e < R * C4; e += kScoreThreads)
-    qb[e] = (e / C4 < nrows) ? qp[e] : make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int e = threadIdx.x; e < nT * C4; e += kScoreThreads) kb[e] = kp[e];
-  __syncthreads();
 
-  const int lane = threadIdx.x % 32;
-  for (int j = threadIdx.x; j < nT; j += kScoreThreads) {
-    float acc[R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) acc[r] = 0.f;
-    const float4* krow = kb + j * C4;
 #pragma unroll 4
-    for (int i = 0; i < C4; ++i) {
-      const int c = (i + lane) % C4;
-      const float4 kv = krow[c];
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const float4 qv = qb[r * C4 + c];
-        acc[r] = fmaf(qv.x, kv.x, acc[r]);
-        acc[r] = fmaf(qv.y, kv.y, acc[r]);
-        acc[r] = fmaf(qv.z, kv.z, acc[r]);
-        acc[r] = fmaf(qv.w, kv.w, acc[r]);
-      }
+  for (int e = threadIdx.x; e < R * C4; e += kScoreThreads)
+    reinterpret_cast<float4*>(qb)[e] = (e / C4 < nrows) ? __ldg(qp + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+
+  const int j = threadIdx.x % kScoreChunk;
+  const int quarter = threadIdx.x / kScoreChunk;
+  for (int c0 = 0; c0 < nT; c0 += kScoreChunk) {
+    const int ncol = min(kScoreChunk, nT - c0);
+    if (c0 > 0) __syncthreads();   // the previous chunk's partial sums are consumed
+#pragma unroll 8
+    for (int e = threadIdx.x; e < ncol * C4; e += kScoreThreads) {
+      const int r = e / C4, c = e % C4;
+      *reinterpret_cast<float4*>(kb + r * KS + 4 * c) = __ldg(kp + static_cast<size_t>(c0) * C4 + e);
     }
+    __syncthreads();
+    if (j < ncol) {
+      float acc[R];
 #pragma unroll
-    for (int r = 0; r < R; ++r) keys[r * nT + j] = order_key(acc[r] + 0.f);
+      for (int r = 0; r < R; ++r) acc[r] = 0.f;
+      const float4* krow = reinterpret_cast<const float4*>(kb + j * KS) + quarter * PART4;
+      const float4* qrow = reinterpret_cast<const float4*>(qb) + quarter * PART4;
+#pragma unroll 4
+      for (int i = 0; i < PART4; ++i) {
+        const float4 kv = krow[i];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const float4 qv = qrow[r * C4 + i];
+          acc[r] = fmaf(qv.x, kv.x, acc[r]);
+          acc[r] = fmaf(qv.y, kv.y, acc[r]);
+          acc[r] = fmaf(qv.z, kv.z, acc[r]);
+          acc[r] = fmaf(qv.w, kv.w, acc[r]);
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < R; ++r) part[(quarter * R + r) * kScoreChunk + j] = acc[r];
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < R * ncol; e += kScoreThreads) {
+      const int r = e / ncol, c = e % ncol;
+      const float sc = (part[r * kScoreChunk + c] + part[(R + r) * kScoreChunk + c]) +
+                       (part[(2 * R + r) * kScoreChunk + c] + part[(3 * R + r) * kScoreChunk + c]);
+      keys[r * nT + c0 + c] = order_key(sc + 0.f);
+    }
   }
   __syncthreads();
 
   const int warp = threadIdx.x / 32;
-  if (warp < nrows)
-    radix_topk_row(keys + warp * nT, nT, topk, hist_all + warp * 256,
-                   idx + (static_cast<size_t>(bh) * nT + row0 + warp) * topk);
+  for (int r = warp; r < nrows; r += kScoreThreads / 32)
+    bsearch_topk_row<MAXE>(keys + r * nT, nT, topk, idx + (static_cast<size_t>(bh) * nT + row0 + r) * topk);
+}
+
+template <int D, int R>
+inline size_t score_smem_bytes(const Geom& g) {
+  const size_t chunk = static_cast<size_t>(min(g.nT, kScoreChunk));
+  return sizeof(float) * (static_cast<size_t>(R) * D + chunk * (D + 4) + kScoreSplit * static_cast<size_t>(R) * kScoreChunk) +
+         sizeof(uint32_t) * (static_cast<size_t>(R) * g.nT);
 }
 
 }  // namespace vsa
