@@ -10,6 +10,9 @@
 //   vsa_diag_mma_ts   O[128xD] = P[128x128] * V[128xD] with P in TMEM (two
 //                     bf16 per column) and V in 128B-swizzled MN-major shared
 //                     memory (the O += P V step).
+//   vsa_diag_exp2     the FMA-pipe and multi-function-unit 2^x of the softmax.
+//   vsa_diag_wait_timeout  a bounded mbarrier wait that nothing completes:
+//                     it must end with a timeout in the error word.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -183,6 +186,20 @@ __global__ void diag_exp2_kernel(const float* x, float* y_poly, float* y_mufu, i
   }
 }
 
+// A wait that nothing ever completes: the bounded wait must give up after its
+// time limit, record the timeout in the error word and let the kernel return.
+__global__ void diag_wait_timeout_kernel(unsigned int* err, int* returned) {
+  __shared__ __align__(8) unsigned long long bar_storage;
+  const uint32_t bar = smem_u32(&bar_storage);
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const bool ok = mbar_wait(bar, 0, nullptr, err);   // nobody arrives
+  if (threadIdx.x == 0) *returned = ok ? 2 : 1;
+}
+
 static unsigned int* diag_err() {
   void* p = nullptr;
   if (cudaGetSymbolAddress(&p, g_diag_error) != cudaSuccess) return nullptr;
@@ -253,6 +270,13 @@ int vsa_diag_mma_ts(const void* P, const void* V, int32_t d, float* O, void* str
 int vsa_diag_exp2(const float* x, float* y_poly, float* y_mufu, int32_t n, void* stream) {
   const int pairs = (n + 1) / 2;
   diag_exp2_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_poly, y_mufu, n);
+  return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
+// Launches one CTA whose only wait can never complete; *returned becomes 1
+// once the bounded wait has given up.
+int vsa_diag_wait_timeout(int32_t* returned, void* stream) {
+  diag_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(diag_err(), returned);
   return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 

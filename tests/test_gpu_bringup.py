@@ -125,3 +125,18 @@ def test_exp2_polynomial_vs_bounds():
     assert np.max(np.abs(yp[ok] - ref[ok]) / ref[ok]) <= 8e-5
     assert np.all(yp[~ok] == 0.0)
     assert np.max(np.abs(ym[ok] - ref[ok]) / ref[ok]) <= 1e-6
+
+
+def test_bounded_wait_times_out_and_reports():
+    """Failure detection without a GPU fault: a wait on a barrier that nothing
+    arrives on gives up after its limit (1 s), the kernel returns, and the
+    timeout code (1) is in the error word; the context stays usable."""
+    L = _diag()
+    L.vsa_diag_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    assert L.vsa_diag_wait_timeout(flag.data_ptr(), None) == 0
+    assert _err(L) == 1
+    assert int(flag.item()) == 1
+    assert _err(L) == 0                       # read-and-clear
+    x = torch.ones(4, device="cuda")
+    assert float((x * 2).sum()) == 8.0        # the context still works
