@@ -48,6 +48,12 @@ constexpr float kRescaleLog2 = 8.0f;
 // (exp2_poly_pair) and the rest on the multi-function unit (ex2.approx): the
 // two units then share the softmax's exponentials.
 constexpr int kExpPolyPer8 = VSA_EXP_POLY_PER8;
+#ifndef VSA_P_PACK_ALU
+#define VSA_P_PACK_ALU 0
+#endif
+// Convert P to bf16 on the integer ALU (pack_bf16x2_alu) rather than with the
+// float conversion instruction.
+constexpr bool kPackAlu = VSA_P_PACK_ALU != 0;
 constexpr uint32_t kErrBadIndex = 2u;
 
 struct AttnArgs {
@@ -514,7 +520,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             p1 = ex2_approx(x1);
           }
           ls2[c & 3] = f2_add(ls2[c & 3], f2_pack(p0, p1));
-          s[c] = pack_bf16x2(p0, p1);
+          s[c] = kPackAlu ? pack_bf16x2_alu(p0, p1) : pack_bf16x2(p0, p1);
         }
         {
           float a0, a1;

@@ -292,6 +292,17 @@ __device__ __forceinline__ void setmaxnreg_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// Two non-negative finite float32 -> bf16x2 on the integer ALU: add half a
+// bf16 unit in the last place to the bits (a carry into the exponent rounds up
+// a binade) and keep the upper halves.  Equals round-to-nearest except at
+// exact ties, which round up.  Used for softmax probabilities, keeping the
+// conversion off the unit that evaluates the exponentials.
+__device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
+  const uint32_t a = __float_as_uint(lo) + 0x8000u;
+  const uint32_t b = __float_as_uint(hi) + 0x8000u;
+  return __byte_perm(a, b, 0x7632);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
