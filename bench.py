@@ -221,6 +221,21 @@ def run_reference(args, w, rank):
     }
 
 
+def max_over_ranks(values, world, device=None):
+    """Element-wise maximum of per-rank timings (every rank gets the result).
+    Multi-GPU numbers are the slowest rank's device time, never a wall clock."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def aggregate_tflops(flops_per_rank_step: float, ms_max: float, steps: int, world: int) -> float:
+    """Whole-job throughput: every rank runs its own replica (weak scaling), so
+    the job does world * flops per step in the slowest rank's time per step."""
+    return world * flops_per_rank_step / (ms_max / steps * 1e-3) / 1e12
+
+
 def describe(w) -> str:
     return (f"{w.name}: B={w.B} H={w.H} d={w.d} grid={tuple(w.grid)} tile={tuple(w.tile)} "
             f"topk={w.topk} inputs={w.kind}")
@@ -301,10 +316,7 @@ def run_ours(args, w, rank, world, device):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
 
-    t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max, e2e_max = t.tolist()
+    ms_max, e2e_max = max_over_ranks([ms, e2e_ms], world, device)
     if rank != 0:
         return None
 
@@ -314,7 +326,7 @@ def run_ours(args, w, rank, world, device):
     peak_kind = "bf16_tflops (burst)" if timed_s < 2.0 else "bf16_tflops_sustained"
     att_tflops = flops / (att_ms * 1e-3) / 1e12
     sel_gbs = select_bytes(w) / (sel_ms * 1e-3) / 1e9
-    value = world * flops / (ms_max / args.steps * 1e-3) / 1e12
+    value = aggregate_tflops(flops, ms_max, args.steps, world)
     out = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
@@ -334,7 +346,7 @@ def run_ours(args, w, rank, world, device):
                             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": sel_gbs / peaks["hbm_gbs"],
                             "peak_source": f"{src} hbm_gbs",
                             "traffic": recorded_traffic("pool_kernel", w.name)},
-        "e2e": {"value": world * flops / (e2e_max * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_max,
+        "e2e": {"value": aggregate_tflops(flops, e2e_max, 1, world), "unit": "TFLOP/s", "ms_per_step": e2e_max,
                 "h2d_bytes_per_step": int(3 * q.numel() * 2),
                 "d2h_bytes_per_step": int(o.numel() * 2 + lse.numel() * 4)},
         "gpu_launches": 3 * args.steps,
