@@ -14,8 +14,8 @@ import torch
 
 from ._native import VsaShape, check, lib
 
-__all__ = ["make_shape", "tile_count", "select", "attn_fwd", "forward", "device_error",
-           "select_workspace_bytes"]
+__all__ = ["make_shape", "tile_count", "select", "attn_fwd", "forward", "forward_host",
+           "device_error", "select_workspace_bytes"]
 
 
 def make_shape(B: int, H: int, grid, d: int, tile) -> VsaShape:
@@ -96,6 +96,94 @@ def forward(q, k, v, grid, tile, topk: int, *, scale=None, stream=None):
     idx = select(q, k, grid, tile, topk, stream=stream)
     o, lse = attn_fwd(q, k, v, idx, grid, tile, scale=scale, stream=stream)
     return o, lse, idx
+
+
+class _HostPipeline:
+    """Device buffers, streams and events reused by forward_host for one shape."""
+
+    def __init__(self, chunk, N, d, nT, topk, device, ws_bytes):
+        mk = lambda *shape, dt=torch.bfloat16: [torch.empty(shape, dtype=dt, device=device) for _ in range(2)]
+        self.q, self.k, self.v, self.o = (mk(1, chunk, N, d) for _ in range(4))
+        self.lse = mk(1, chunk, N, dt=torch.float32)
+        self.idx = mk(1, chunk, nT, topk, dt=torch.int32)
+        self.ws = [torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device) for _ in range(2)]
+        self.s_in = torch.cuda.Stream(device)
+        self.s_comp = torch.cuda.Stream(device)
+        self.s_out = torch.cuda.Stream(device)
+        self.key = (chunk, N, d, nT, topk, device)
+
+
+_PIPE = {}
+
+
+def forward_host(q, k, v, grid, tile, topk: int, *, scale=None, chunk_heads: int = 4,
+                 out=None, lse=None, idx=None, device=None):
+    """Host-to-host forward: select + attention for pinned CPU tensors.
+
+    q, k, v: pinned CPU bfloat16 [B, H, N, d].  Returns (O, LSE, idx) in pinned
+    CPU tensors (allocated unless given).  The (batch, head) pairs are
+    processed in chunks of ``chunk_heads``: the upload of chunk c+1 and the
+    download of chunk c-1 overlap the kernels of chunk c (three streams,
+    double-buffered device memory).  Every chunk is one vsa_select and one
+    vsa_attn_fwd call with H = chunk.  The caller's current stream waits for
+    all of it, so work queued on it afterwards sees the outputs.
+    """
+    B, H, N, d = q.shape
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    for name, x in (("q", q), ("k", k), ("v", v)):
+        if x.is_cuda or x.dtype != torch.bfloat16 or not x.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CPU bfloat16 tensor (pinned for overlap)")
+    nT, _ = tile_count(grid, tile, d, B, H)
+    BH = B * H
+    chunk = max(1, min(chunk_heads, BH))
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16).pin_memory()
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+    if idx is None:
+        idx = torch.empty((B, H, nT, topk), dtype=torch.int32).pin_memory()
+    key = (chunk, N, d, nT, topk, device)
+    pipe = _PIPE.get(key)
+    if pipe is None:
+        pipe = _HostPipeline(chunk, N, d, nT, topk, device, select_workspace_bytes(1, chunk, grid, d, tile))
+        _PIPE.clear()
+        _PIPE[key] = pipe
+    caller = torch.cuda.current_stream(device)
+    for s_ in (pipe.s_in, pipe.s_comp, pipe.s_out):
+        s_.wait_stream(caller)
+    qf, kf, vf = (x.view(BH, N, d) for x in (q, k, v))
+    of, lf, xf = out.view(BH, N, d), lse.view(BH, N), idx.view(BH, nT, topk)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [None, None]
+    for c, h0 in enumerate(range(0, BH, chunk)):
+        nh = min(chunk, BH - h0)
+        b = c % 2
+        dq, dk, dv, do = (t[b][:, :nh] for t in (pipe.q, pipe.k, pipe.v, pipe.o))
+        dl, di = pipe.lse[b][:, :nh], pipe.idx[b][:, :nh]
+        with torch.cuda.stream(pipe.s_in):
+            if ev_out[b] is not None:          # buffer b's previous outputs are downloaded
+                pipe.s_in.wait_event(ev_out[b])
+            dq.copy_(qf[h0:h0 + nh].unsqueeze(0), non_blocking=True)
+            dk.copy_(kf[h0:h0 + nh].unsqueeze(0), non_blocking=True)
+            dv.copy_(vf[h0:h0 + nh].unsqueeze(0), non_blocking=True)
+            ev_in[b].record(pipe.s_in)
+        with torch.cuda.stream(pipe.s_comp):
+            pipe.s_comp.wait_event(ev_in[b])
+            select(dq, dk, grid, tile, topk, out=di, workspace=pipe.ws[b], stream=pipe.s_comp)
+            attn_fwd(dq, dk, dv, di, grid, tile, scale=scale, out=do, lse=dl, stream=pipe.s_comp)
+            ev_comp[b].record(pipe.s_comp)
+        with torch.cuda.stream(pipe.s_out):
+            pipe.s_out.wait_event(ev_comp[b])
+            of[h0:h0 + nh].unsqueeze(0).copy_(do, non_blocking=True)
+            lf[h0:h0 + nh].unsqueeze(0).copy_(dl, non_blocking=True)
+            xf[h0:h0 + nh].unsqueeze(0).copy_(di, non_blocking=True)
+            e = torch.cuda.Event()
+            e.record(pipe.s_out)
+            ev_out[b] = e
+    for s_ in (pipe.s_in, pipe.s_comp, pipe.s_out):
+        caller.wait_stream(s_)
+    return out, lse, idx
 
 
 def device_error(reset: bool = True) -> int:

@@ -8,11 +8,17 @@
 // [B*H, T, Hh, W, d], so a tile or half-tile is one box, zero-filled past the
 // grid edge).
 //
-// One CTA = one work unit with two "slots" of up to 128 query rows each.
-//   SHARED (tiles of 256 tokens, tt >= 2): the slots are the two t-halves of
-//     one query tile and share every K/V sub-block (a t-half of a kept tile).
-//   !SHARED (tiles of 64 or 128 tokens): the slots are two consecutive query
-//     tiles; a K/V sub-block packs 128 / vol kept tiles of one slot.
+// One CTA = one work unit with two "slots" of 128 query rows each.
+//   MODE_SHARED (tiles of 256 tokens, tt >= 2): the slots are the two t-halves
+//     of one query tile and share every K/V sub-block (a t-half of a kept tile).
+//   MODE_TILE (tiles of 128 tokens): each slot is one query tile; a K/V
+//     sub-block is one of its kept tiles.
+//   MODE_PAIR (tiles of 64 tokens): each slot stacks two neighbouring query
+//     tiles A (rows 0-63) and B (rows 64-127).  The slot walks the union of
+//     their kept lists, two 64-token tiles per K/V sub-block, and every row
+//     masks the tiles only the other query tile kept.  Neighbouring tiles of a
+//     video keep mostly the same tiles, so most of each 128-row MMA is useful
+//     work; at worst (disjoint lists) it is half, as with one padded tile.
 // Warp roles (384 threads): warps 0-3 softmax slot 0, warps 4-7 softmax slot 1
 // (thread = query row = TMEM lane), warp 8 TMA producer, warp 9 MMA issuer,
 // warps 10-11 idle.  The producer warpgroup gives registers to the softmax
@@ -56,6 +62,8 @@ constexpr int kExpPolyPer8 = VSA_EXP_POLY_PER8;
 constexpr bool kPackAlu = VSA_P_PACK_ALU != 0;
 constexpr uint32_t kErrBadIndex = 2u;
 
+enum : int { MODE_SHARED = 0, MODE_TILE = 1, MODE_PAIR = 2 };
+
 struct AttnArgs {
   Geom g;
   int topk;
@@ -64,7 +72,7 @@ struct AttnArgs {
   __nv_bfloat16* o;          // [B*H, N, d]
   float* lse;                // [B*H, N]
   unsigned int* err;         // device error word
-  int box_t;                 // t-extent of one TMA box (tt/2 when SHARED, else tt)
+  int box_t;                 // t-extent of one TMA box (tt/2 in MODE_SHARED, else tt)
 };
 
 template <int D>
@@ -77,11 +85,17 @@ struct AttnSmem {
   static constexpr int kV = 4 * kBufBytes;            // 2 buffers
   static constexpr int kBar = 6 * kBufBytes;
   static constexpr int kNumBars = 17;
-  static constexpr int kMisc = kBar + kNumBars * 8;
+  static constexpr int kMisc = kBar + kNumBars * 8;   // TMEM address, abort flag, union lengths
   static constexpr int kTiles = kMisc + 16;           // uint2 per tile: (bt, by | bx << 16)
-  static constexpr int kMaxTiles = 2048;
-  static constexpr int kTotal = kTiles + 8 * kMaxTiles;
-  static constexpr int kAlloc = kTotal + 1024;        // slack for 1024-byte alignment
+  // then, in MODE_PAIR only: membership bitmaps (4 x ceil(nT/32) words) and
+  // the two slots' union lists (2 x 2*topk entries of j | in_a << 16 | in_b << 17)
+  __host__ __device__ static int bitmap_off(int nT) { return kTiles + ((8 * nT + 15) & ~15); }
+  __host__ __device__ static int bitmap_words(int nT) { return (nT + 31) / 32; }
+  __host__ __device__ static int union_off(int nT) { return bitmap_off(nT) + ((16 * bitmap_words(nT) + 15) & ~15); }
+  __host__ __device__ static int total(int nT, int topk, bool pair) {
+    return pair ? union_off(nT) + 2 * 2 * topk * 4 : kTiles + 8 * nT;
+  }
+  __host__ __device__ static int alloc(int nT, int topk, bool pair) { return total(nT, topk, pair) + 1024; }
 };
 
 enum : int {
@@ -91,8 +105,10 @@ enum : int {
 
 struct Slot {
   bool active;
-  int bh, tile;          // head index (b*H + h) and query tile
-  int t0, y0, x0;        // origin of the slot's query box
+  int bh, tile;          // head index (b*H + h) and query tile (tile A in MODE_PAIR)
+  int t0, y0, x0;        // origin of the slot's (first) query box
+  bool has_b;            // MODE_PAIR: tile B = tile + 1 exists
+  int tb0, yb0, xb0;     // MODE_PAIR: origin of tile B
 };
 
 __device__ __forceinline__ int load_tile_index(const AttnArgs& a, const int32_t* row, int e,
@@ -105,10 +121,6 @@ __device__ __forceinline__ int load_tile_index(const AttnArgs& a, const int32_t*
   return j;
 }
 
-// K/V sub-block sequence of one query tile.
-//   SHARED: for each kept tile (ascending), its t-halves that hold any token.
-//   !SHARED: groups of P = 128 / vol kept tiles; a short last group repeats its
-//            last tile in the missing pieces (masked out).
 // Tile coordinates from the per-CTA table built at kernel start (one shared
 // memory load instead of integer divisions in every iteration).
 __device__ __forceinline__ TileCoord table_coord(const uint2* tab, int j) {
@@ -120,14 +132,33 @@ __device__ __forceinline__ TileCoord table_coord(const uint2* tab, int j) {
   return c;
 }
 
-template <bool SHARED>
+// One K/V piece of a sub-block: kept tile j, t offset of the box inside the
+// tile, whether it is real (false: padding that repeats a real tile, fully
+// masked), and which query tile of a MODE_PAIR slot kept it.
+struct Piece {
+  int j, toff;
+  bool real, in_a, in_b;
+};
+
+// K/V sub-block sequence of one slot.
+//   MODE_SHARED: for each kept tile (ascending), its t-halves that hold a token.
+//   MODE_TILE:   each kept tile.
+//   MODE_PAIR:   the ascending union of tile A's and tile B's kept lists (built
+//                in shared memory at kernel start), two tiles per sub-block (a
+//                short last sub-block is padded).
+template <int MODE>
 struct KvSeq {
-  const int32_t* row;
+  const int32_t* row;     // kept list of the slot's (first) query tile
+  const uint32_t* uni;    // MODE_PAIR: the slot's union list in shared memory
+  int ulen;               // MODE_PAIR: its length
   const uint2* tab;
   int pos, half;
 
-  __device__ void init(const AttnArgs& a, const uint2* table, int bh, int tile) {
+  __device__ void init(const AttnArgs& a, const uint2* table, int bh, int tile, const uint32_t* union_list = nullptr,
+                       int union_len = 0) {
     row = a.idx + (static_cast<size_t>(bh) * a.g.nT + tile) * a.topk;
+    uni = union_list;
+    ulen = union_len;
     tab = table;
     pos = 0;
     half = 0;
@@ -136,30 +167,37 @@ struct KvSeq {
     return static_cast<int>(tab[j].x) * a.g.tt + a.box_t < a.g.T;
   }
   __device__ int count(const AttnArgs& a) const {
-    if (!SHARED) {
-      const int P = kSubRows / a.g.vol;
-      return (a.topk + P - 1) / P;
-    }
+    if (MODE == MODE_TILE) return a.topk;
+    if (MODE == MODE_PAIR) return (ulen + 1) / 2;
     int n = 0;
     for (int e = 0; e < a.topk; ++e) n += 1 + (second_half(a, load_tile_index(a, row, e, false)) ? 1 : 0);
     return n;
   }
-  // Piece p of the current sub-block: tile j, t offset inside the tile, and
-  // whether it is a real piece (false: padding repeat of the last tile).
-  __device__ void piece(const AttnArgs& a, int p, bool report, int& j, int& toff, bool& real) const {
-    if (SHARED) {
-      j = load_tile_index(a, row, pos, report);
-      toff = half * a.box_t;
-      real = true;
+  // Piece p (0 or 1) of the current sub-block.
+  __device__ Piece piece(const AttnArgs& a, int p, bool report) const {
+    Piece pc;
+    if (MODE == MODE_SHARED) {
+      pc.j = load_tile_index(a, row, pos, report);
+      pc.toff = half * a.box_t;
+      pc.real = pc.in_a = pc.in_b = true;
+    } else if (MODE == MODE_TILE) {
+      pc.j = load_tile_index(a, row, pos, report);
+      pc.toff = 0;
+      pc.real = pc.in_a = pc.in_b = true;
     } else {
-      const int e = pos + p;
-      real = e < a.topk;
-      j = load_tile_index(a, row, real ? e : a.topk - 1, report && real);
-      toff = 0;
+      const int e = 2 * pos + p;
+      const bool real = e < ulen;
+      const uint32_t u = uni[real ? e : 2 * pos];   // padding repeats a real piece, all masked
+      pc.j = static_cast<int>(u & 0xffffu);
+      pc.toff = 0;
+      pc.real = real;
+      pc.in_a = real && ((u >> 16) & 1u);
+      pc.in_b = real && ((u >> 17) & 1u);
     }
+    return pc;
   }
   __device__ void advance(const AttnArgs& a) {
-    if (SHARED) {
+    if (MODE == MODE_SHARED) {
       if (half == 0 && second_half(a, load_tile_index(a, row, pos, false))) {
         half = 1;
       } else {
@@ -167,15 +205,64 @@ struct KvSeq {
         ++pos;
       }
     } else {
-      pos += kSubRows / a.g.vol;
+      ++pos;
     }
   }
 };
 
-template <int D, bool SHARED>
+// One warp builds a MODE_PAIR slot's union list: membership bitmaps of the two
+// kept lists, then the set tiles in ascending order with per-list flags
+// (prefix counts across the warp give each tile its position).  Returns the
+// union length (valid in every lane).
+__device__ __forceinline__ int build_union(const AttnArgs& a, const int32_t* row_a, bool has_b, uint32_t* bm_a,
+                                           uint32_t* bm_b, uint32_t* out) {
+  const int lane = threadIdx.x % 32;
+  const int nw = (a.g.nT + 31) / 32;
+  for (int w = lane; w < nw; w += 32) {
+    bm_a[w] = 0u;
+    bm_b[w] = 0u;
+  }
+  __syncwarp();
+  for (int e = lane; e < a.topk; e += 32) {
+    const int ja = load_tile_index(a, row_a, e, true);
+    atomicOr(bm_a + (ja >> 5), 1u << (ja & 31));
+    if (has_b) {
+      const int jb = load_tile_index(a, row_a + a.topk, e, true);
+      atomicOr(bm_b + (jb >> 5), 1u << (jb & 31));
+    }
+  }
+  __syncwarp();
+  int base = 0;
+  for (int w0 = 0; w0 < nw; w0 += 32) {
+    const int w = w0 + lane;
+    const uint32_t ua = (w < nw) ? bm_a[w] : 0u;
+    const uint32_t ub = (w < nw) ? bm_b[w] : 0u;
+    uint32_t u = ua | ub;
+    const int cnt = __popc(u);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int pos = base + incl - cnt;
+    while (u) {
+      const int b = __ffs(u) - 1;
+      u &= u - 1;
+      out[pos++] = static_cast<uint32_t>(32 * w + b) | (((ua >> b) & 1u) << 16) | (((ub >> b) & 1u) << 17);
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  return base;
+}
+
+template <int D, int MODE>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+  constexpr bool SHARED = MODE == MODE_SHARED;
+  constexpr bool PAIR = MODE == MODE_PAIR;
+  constexpr int P = PAIR ? 2 : 1;                            // pieces per K/V sub-block
   using L = AttnSmem<D>;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -185,11 +272,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sp + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sp + L::kMisc + 4);
   uint2* tile_tab = reinterpret_cast<uint2*>(sp + L::kTiles);
+  int* union_len = reinterpret_cast<int*>(sp + L::kMisc + 8);          // [2]
+  uint32_t* bitmaps = reinterpret_cast<uint32_t*>(sp + L::bitmap_off(a.g.nT));
+  uint32_t* unions = reinterpret_cast<uint32_t*>(sp + L::union_off(a.g.nT));
   auto bar = [&](int id) -> uint32_t { return sBar + 8u * static_cast<uint32_t>(id); };
 
   const Geom& g = a.g;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int P = SHARED ? 1 : kSubRows / g.vol;             // pieces per sub-block
   const int box_rows = SHARED ? kSubRows : g.vol;          // rows per TMA box
   const uint32_t box_bytes = static_cast<uint32_t>(box_rows) * 128u;
 
@@ -199,16 +288,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   for (int h = 0; h < 2; ++h) {
     int bh, tile, toff;
     bool act;
+    bool has_b = false;
     if (SHARED) {
       bh = blockIdx.x / g.nT;
       tile = blockIdx.x % g.nT;
       toff = h * a.box_t;
       act = true;
-    } else {
+    } else if (MODE == MODE_TILE) {
       const long long gidx = 2ll * blockIdx.x + h;
       act = gidx < static_cast<long long>(g.B) * g.H * g.nT;
       bh = act ? static_cast<int>(gidx / g.nT) : 0;
       tile = act ? static_cast<int>(gidx % g.nT) : 0;
+      toff = 0;
+    } else {
+      const int npair = (g.nT + 1) / 2;
+      const long long gp = 2ll * blockIdx.x + h;
+      act = gp < static_cast<long long>(g.B) * g.H * npair;
+      bh = act ? static_cast<int>(gp / npair) : 0;
+      tile = act ? 2 * static_cast<int>(gp % npair) : 0;
+      has_b = act && tile + 1 < g.nT;
       toff = 0;
     }
     const TileCoord c = tile_coord(g, tile);
@@ -218,10 +316,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     slot[h].y0 = c.by * g.th;
     slot[h].x0 = c.bx * g.tw;
     slot[h].active = act && slot[h].t0 < g.T;
+    slot[h].has_b = has_b;
+    const TileCoord cb = tile_coord(g, has_b ? tile + 1 : tile);
+    slot[h].tb0 = cb.bt * g.tt;
+    slot[h].yb0 = cb.by * g.th;
+    slot[h].xb0 = cb.bx * g.tw;
   }
   const int last_active = slot[1].active ? 1 : 0;
 
-  // ---- setup: tile table, barriers, zero padding rows of Q, TMEM allocation
+  // ---- setup: tile table, barriers, zero rows of a missing tile B, TMEM
   for (int j = threadIdx.x; j < g.nT; j += kAttnThreads) {
     const TileCoord c = tile_coord(g, j);
     tile_tab[j] = make_uint2(static_cast<uint32_t>(c.bt),
@@ -235,15 +338,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (!SHARED && g.vol < kSlotRows) {
-    // rows [vol, 128) of the Q buffers are never loaded; make them zeros
-    for (int s = 0; s < 2; ++s)
+  if (PAIR && (warp == 10 || warp == 11)) {
+    // warp 10 builds slot 0's union list, warp 11 slot 1's
+    const int h = warp - 10;
+    const Slot& sl = h ? slot[1] : slot[0];
+    int len = 0;
+    if (sl.active) {
+      const int32_t* row_a = a.idx + (static_cast<size_t>(sl.bh) * g.nT + sl.tile) * a.topk;
+      const int nw = L::bitmap_words(g.nT);
+      len = build_union(a, row_a, sl.has_b, bitmaps + 2 * h * nw, bitmaps + (2 * h + 1) * nw,
+                        unions + h * 2 * a.topk);
+    }
+    if (lane == 0) union_len[h] = len;
+  }
+  if (PAIR) {
+    // a slot without tile B (odd tile count) computes rows 64-127 from zeros
+    for (int h = 0; h < 2; ++h) {
+      if (!slot[h].active || slot[h].has_b) continue;
       for (int sl = 0; sl < L::kSlabs; ++sl) {
-        uint4* p = reinterpret_cast<uint4*>(sp + L::kQ + s * L::kBufBytes + sl * L::kSlabBytes +
-                                            g.vol * 128);
-        const int n16 = (kSlotRows - g.vol) * 128 / 16;
-        for (int e = threadIdx.x; e < n16; e += kAttnThreads) p[e] = make_uint4(0, 0, 0, 0);
+        uint4* q4 = reinterpret_cast<uint4*>(sp + L::kQ + h * L::kBufBytes + sl * L::kSlabBytes + 64 * 128);
+        for (int e = threadIdx.x; e < 64 * 128 / 16; e += kAttnThreads) q4[e] = make_uint4(0, 0, 0, 0);
       }
+    }
     fence_proxy_async_smem();
   }
   if (warp == 9) {
@@ -260,9 +376,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  KvSeq<SHARED> seq;
-  seq.init(a, tile_tab, slot[0].bh, slot[0].tile);
-
   if (warp >= 8) {
     setmaxnreg_dec<kProducerRegs>();
   }
@@ -272,40 +385,49 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       bool ok = true;
       for (int h = 0; h < 2; ++h) {
         if (!slot[h].active) continue;
-        mbar_arrive_expect_tx(bar(BAR_Q_FULL + h), L::kSlabs * box_bytes);
-        for (int sl = 0; sl < L::kSlabs; ++sl)
+        const int nbox = (PAIR && slot[h].has_b) ? 2 : 1;
+        mbar_arrive_expect_tx(bar(BAR_Q_FULL + h), static_cast<uint32_t>(nbox * L::kSlabs) * box_bytes);
+        for (int sl = 0; sl < L::kSlabs; ++sl) {
           tma_load_5d(sQ + h * L::kBufBytes + sl * L::kSlabBytes, &tmQ, bar(BAR_Q_FULL + h), sl * 64,
                       slot[h].x0, slot[h].y0, slot[h].t0, slot[h].bh);
+          if (nbox == 2)
+            tma_load_5d(sQ + h * L::kBufBytes + sl * L::kSlabBytes + box_bytes, &tmQ, bar(BAR_Q_FULL + h),
+                        sl * 64, slot[h].xb0, slot[h].yb0, slot[h].tb0, slot[h].bh);
+        }
       }
-      KvSeq<SHARED> sq[2];
-      sq[0].init(a, tile_tab, slot[0].bh, slot[0].tile);
-      sq[1].init(a, tile_tab, slot[1].bh, slot[1].tile);
-      const int n = sq[0].count(a);
+      KvSeq<MODE> sq[2];
+      int n[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        sq[h].init(a, tile_tab, slot[h].bh, slot[h].tile, unions + h * 2 * a.topk, union_len[h]);
+        n[h] = slot[h].active ? sq[h].count(a) : 0;
+      }
+      const int n_max = SHARED ? n[0] : max(n[0], n[1]);
       int last_use[2][2] = {{-1, -1}, {-1, -1}};   // [K/V][stage]: last phase issued
-      for (int it = 0; it < n && ok; ++it) {
+      for (int it = 0; it < n_max && ok; ++it) {
         for (int kv = 0; kv < 2 && ok; ++kv) {         // K first, then V
           const CUtensorMap* tm = kv == 0 ? &tmK : &tmV;
           const uint32_t buf0 = kv == 0 ? sK : sV;
           const int full = kv == 0 ? BAR_K_FULL : BAR_V_FULL;
           const int empty = kv == 0 ? BAR_K_EMPTY : BAR_V_EMPTY;
+#pragma unroll
           for (int h = 0; h < (SHARED ? 1 : 2); ++h) {
-            if (!slot[h].active) continue;
+            if (!ok || it >= n[h]) continue;
             const int st = SHARED ? (it & 1) : h;
             const int use = SHARED ? (it >> 1) : it;
             if (use > 0 && !mbar_wait(bar(empty + st), (use - 1) & 1, abort_flag, a.err)) {
               ok = false;
-              break;
+              continue;
             }
             mbar_arrive_expect_tx(bar(full + st), static_cast<uint32_t>(P * L::kSlabs) * box_bytes);
             last_use[kv][st] = use;
+#pragma unroll
             for (int p = 0; p < P; ++p) {
-              int j, toff;
-              bool real;
-              sq[h].piece(a, p, kv == 0, j, toff, real);
-              const TileCoord c = table_coord(tile_tab, j);
+              const Piece pc = sq[h].piece(a, p, kv == 0);
+              const TileCoord c = table_coord(tile_tab, pc.j);
               for (int sl = 0; sl < L::kSlabs; ++sl)
                 tma_load_5d(buf0 + st * L::kBufBytes + sl * L::kSlabBytes + p * box_bytes, tm,
-                            bar(full + st), sl * 64, c.bx * g.tw, c.by * g.th, c.bt * g.tt + toff,
+                            bar(full + st), sl * 64, c.bx * g.tw, c.by * g.th, c.bt * g.tt + pc.toff,
                             slot[h].bh);
             }
           }
@@ -326,7 +448,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(kSlotRows, kSubRows, false);
       constexpr uint32_t idPV = idesc_bf16_f32(kSlotRows, D, true);
-      const int n = seq.count(a);
+      int n[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        KvSeq<MODE> sq;
+        sq.init(a, tile_tab, slot[h].bh, slot[h].tile, unions + h * 2 * a.topk, union_len[h]);
+        n[h] = slot[h].active ? sq.count(a) : 0;
+      }
       bool ok = true;
 #pragma unroll
       for (int h = 0; h < 2; ++h)
@@ -351,13 +479,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       };
 
-      for (int it = 0; it < n && ok; ++it) {
-        #pragma unroll
+      // iteration it of slot h: PV_h(it-1) then S_h(it); one step past the
+      // slot's last sub-block, only the final PV and the O_FULL commit.
+      const int n_max = max(n[0], n[1]);
+      for (int it = 0; it <= n_max && ok; ++it) {
+#pragma unroll
         for (int h = 0; h < 2; ++h) {
-          if (!ok || !slot[h].active) continue;
+          if (!ok || !slot[h].active || it > n[h]) continue;
           const int kst = SHARED ? (it & 1) : h;
           const int kpar = SHARED ? ((it >> 1) & 1) : (it & 1);
-          if (!mbar_wait(bar(BAR_K_FULL + kst), kpar, abort_flag, a.err)) { ok = false; continue; }
+          if (it < n[h] && !mbar_wait(bar(BAR_K_FULL + kst), kpar, abort_flag, a.err)) { ok = false; continue; }
           if (it > 0) {
             const int vst = SHARED ? ((it - 1) & 1) : h;
             const int vpar = SHARED ? (((it - 1) >> 1) & 1) : ((it - 1) & 1);
@@ -365,6 +496,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 !mbar_wait(bar(BAR_V_FULL + vst), vpar, abort_flag, a.err)) { ok = false; continue; }
             tc_fence_after();
             issue_pv(h, vst, it - 1 > 0);
+            if (it == n[h]) {
+              mma_commit(bar(BAR_O_FULL + h));
+              continue;
+            }
             if (!SHARED || h == last_active) mma_commit(bar(BAR_V_EMPTY + vst));
           }
           tc_fence_after();
@@ -372,18 +507,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           mma_commit(bar(BAR_S_FULL + h));
           if (!SHARED || h == last_active) mma_commit(bar(BAR_K_EMPTY + kst));
         }
-      }
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (!ok || !slot[h].active) continue;
-        const int it = n - 1;
-        const int vst = SHARED ? (it & 1) : h;
-        const int vpar = SHARED ? ((it >> 1) & 1) : (it & 1);
-        if (!mbar_wait(bar(BAR_P_FULL + h), it & 1, abort_flag, a.err) ||
-            !mbar_wait(bar(BAR_V_FULL + vst), vpar, abort_flag, a.err)) { ok = false; continue; }
-        tc_fence_after();
-        issue_pv(h, vst, it > 0);
-        mma_commit(bar(BAR_O_FULL + h));
       }
       // Drain: every MMA issued above has finished before TMEM is freed.
       mma_commit(bar(BAR_DRAIN));
@@ -400,9 +523,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     me.active = h ? slot[1].active : slot[0].active;
     me.bh = h ? slot[1].bh : slot[0].bh;
     me.tile = h ? slot[1].tile : slot[0].tile;
-    me.t0 = h ? slot[1].t0 : slot[0].t0;
-    me.y0 = h ? slot[1].y0 : slot[0].y0;
-    me.x0 = h ? slot[1].x0 : slot[0].x0;
+    me.has_b = h ? slot[1].has_b : slot[0].has_b;
+    // MODE_PAIR: rows 64-127 (warps 2-3 of the warpgroup) belong to tile B
+    const bool in_b = PAIR && r >= 64;
+    me.t0 = in_b ? (h ? slot[1].tb0 : slot[0].tb0) : (h ? slot[1].t0 : slot[0].t0);
+    me.y0 = in_b ? (h ? slot[1].yb0 : slot[0].yb0) : (h ? slot[1].y0 : slot[0].y0);
+    me.x0 = in_b ? (h ? slot[1].xb0 : slot[0].xb0) : (h ? slot[1].x0 : slot[0].x0);
     if (me.active) {
       const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
       const uint32_t tS = tmem + lane_base + 128u * h;
@@ -413,53 +539,53 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       bool row_valid;
       int tok_t, tok_y, tok_x;
       {
-        const int rr = r;
+        const int rr = PAIR ? (r & 63) : r;
         const int lt = rr >> lg_yx, ly = (rr >> g.lg_tw) & (g.th - 1), lx = rr & (g.tw - 1);
         tok_t = me.t0 + lt;
         tok_y = me.y0 + ly;
         tok_x = me.x0 + lx;
         row_valid = rr < box_rows && tok_t < g.T && tok_y < g.Hh && tok_x < g.W &&
-                    lt < (SHARED ? a.box_t : g.tt);
+                    lt < (SHARED ? a.box_t : g.tt) && (!in_b || me.has_b);
       }
 
-      KvSeq<SHARED> sq;
-      sq.init(a, tile_tab, me.bh, me.tile);
+      KvSeq<MODE> sq;
+      sq.init(a, tile_tab, me.bh, me.tile, unions + h * 2 * a.topk, union_len[h]);
       const int n = sq.count(a);
       float m = -INFINITY, l = 0.f;
       bool ok = true;
       for (int it = 0; it < n; ++it) {
-        // validity of the sub-block's 128 key columns (only needed at grid edges)
+        // Which key columns count for this warp's rows: columns [0, 64) are
+        // piece 0 and [64, 128) piece 1 (one 128-column piece outside
+        // MODE_PAIR).  use0/use1: the piece was kept by this row's query tile
+        // (warp-uniform); a piece that is not used contributes P = 0 without
+        // any exponential.  Partial tiles at the grid edge need a column mask.
         uint32_t mw[4] = {~0u, ~0u, ~0u, ~0u};
-        bool full = true;
+        bool use0 = true, use1 = true, geo_full = true;
         {
-          // extents of the (at most two) pieces, kept in scalars so that no
-          // array is indexed at run time
           int vt0 = 0, vy0 = 0, vx0 = 0, vt1 = 0, vy1 = 0, vx1 = 0;
-          bool real0 = false, real1 = false;
 #pragma unroll
-          for (int p = 0; p < 2; ++p) {
-            if (p < P) {
-              int j, toff;
-              bool real;
-              sq.piece(a, p, false, j, toff, real);
-              const TileCoord c = table_coord(tile_tab, j);
-              int et, ey, ex;
-              tile_extent(g, c, et, ey, ex);
-              const int vt = SHARED ? min(a.box_t, et - toff) : et;
-              full = full && real && vt == (SHARED ? a.box_t : g.tt) && ey == g.th && ex == g.tw;
-              if (p == 0) { vt0 = vt; vy0 = ey; vx0 = ex; real0 = real; }
-              else        { vt1 = vt; vy1 = ey; vx1 = ex; real1 = real; }
-            }
+          for (int p = 0; p < P; ++p) {
+            const Piece pc = sq.piece(a, p, false);
+            const TileCoord c = table_coord(tile_tab, pc.j);
+            int et, ey, ex;
+            tile_extent(g, c, et, ey, ex);
+            const int vt = SHARED ? min(a.box_t, et - pc.toff) : et;
+            const bool use = pc.real && (in_b ? pc.in_b : pc.in_a);
+            const bool gfull = vt == (SHARED ? a.box_t : g.tt) && ey == g.th && ex == g.tw;
+            geo_full = geo_full && (!use || gfull);
+            if (p == 0) { vt0 = vt; vy0 = ey; vx0 = ex; use0 = use; }
+            else        { vt1 = vt; vy1 = ey; vx1 = ex; use1 = use; }
           }
-          if (!full) {
+          if (!PAIR) use1 = use0;
+          if (!geo_full) {
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
               const int col = 32 * w + lane;
-              const bool second = !SHARED && col >= g.vol;
+              const bool second = PAIR && col >= g.vol;
               const int rr = second ? col - g.vol : col;
               const int lt = rr >> lg_yx, ly = (rr >> g.lg_tw) & (g.th - 1), lx = rr & (g.tw - 1);
-              const bool v = second ? (real1 && lt < vt1 && ly < vy1 && lx < vx1)
-                                    : (real0 && lt < vt0 && ly < vy0 && lx < vx0);
+              const bool v = second ? (use1 && lt < vt1 && ly < vy1 && lx < vx1)
+                                    : (use0 && lt < vt0 && ly < vy0 && lx < vx0);
               mw[w] = __ballot_sync(0xffffffffu, v);
             }
           }
@@ -478,49 +604,63 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
         tmem_wait_ld();
 
-        if (!full) {
+        if (!geo_full) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             if (!((mw[c >> 5] >> (c & 31)) & 1u)) s[c] = __float_as_uint(-INFINITY);
         }
-        // row max as a tree of 8 independent chains of 3-input max (short depth)
-        float mx8[8];
+        // row max over the used halves, each a tree of 4 chains of 3-input max
+        float mxh[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(s[e]);
+        for (int hf = 0; hf < 2; ++hf) {
+          if (!(hf ? use1 : use0)) continue;
+          float mx4[4];
 #pragma unroll
-        for (int c = 8; c < 128; c += 2)
-          mx8[(c >> 1) & 7] = fmax3(mx8[(c >> 1) & 7], __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
-        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
-        const float mx_s = mx * a.scale_log2;
+          for (int e = 0; e < 4; ++e) mx4[e] = __uint_as_float(s[64 * hf + e]);
+#pragma unroll
+          for (int c = 64 * hf + 4; c < 64 * hf + 64; c += 2)
+            mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+          mxh[hf] = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        }
+        const float mx_s = fmaxf(mxh[0], mxh[1]) * a.scale_log2;
 
-        // lazy rescale: move the reference max only when it grew by > 2^8
+        // lazy rescale: move the reference max only when it grew by > 2^8.  A
+        // row may see no valid key in a sub-block (mx = -inf, MODE_PAIR); its
+        // reference stays -inf until one arrives, with 0 used in the exponent.
         float alpha = 1.f;
-        if (it == 0) {
-          m = mx_s;
-        } else if (mx_s > m + kRescaleLog2) {
-          alpha = ex2_approx(m - mx_s);
+        if (mx_s > m + kRescaleLog2) {
+          alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - mx_s);
           m = mx_s;
           l *= alpha;
         }
-        const bool rescale = __any_sync(0xffffffffu, alpha != 1.f);
+        const bool rescale = __any_sync(0xffffffffu, alpha != 1.f) && it > 0;
+        const float m_use = (m == -INFINITY) ? 0.f : m;
         // P = 2^(scale*log2(e)*S - m) on pairs of columns; row sum in 4 packed chains
         const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2);
-        const uint64_t nm2 = f2_pack(-m, -m);
+        const uint64_t nm2 = f2_pack(-m_use, -m_use);
         uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), sc2, nm2);
-          float p0, p1;
-          if ((c & 7) < kExpPolyPer8) {
-            exp2_poly_pair(x2, p0, p1);
-          } else {
-            float x0, x1;
-            f2_unpack(x2, x0, x1);
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
+        for (int hf = 0; hf < 2; ++hf) {
+          if (!(hf ? use1 : use0)) {
+#pragma unroll
+            for (int c = 32 * hf; c < 32 * hf + 32; ++c) s[c] = 0u;     // P = 0
+            continue;
           }
-          ls2[c & 3] = f2_add(ls2[c & 3], f2_pack(p0, p1));
-          s[c] = kPackAlu ? pack_bf16x2_alu(p0, p1) : pack_bf16x2(p0, p1);
+#pragma unroll
+          for (int c = 32 * hf; c < 32 * hf + 32; ++c) {
+            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), sc2, nm2);
+            float p0, p1;
+            if ((c & 7) < kExpPolyPer8) {
+              exp2_poly_pair(x2, p0, p1);
+            } else {
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+            ls2[c & 3] = f2_add(ls2[c & 3], f2_pack(p0, p1));
+            s[c] = kPackAlu ? pack_bf16x2_alu(p0, p1) : pack_bf16x2(p0, p1);
+          }
         }
         {
           float a0, a1;

@@ -21,6 +21,7 @@ __device__ unsigned int g_device_error = 0u;
 
 constexpr int kMaxTiles = 1536;          // score rows of one CTA must fit in shared memory
 constexpr int kMaxDevices = 64;
+constexpr int kMaxSmemPerBlock = 232448;  // opt-in dynamic shared memory per CTA on sm_100
 
 // -------------------------------------------------------------- validation
 static int make_geom(const vsa_shape* s, Geom* g) {
@@ -117,16 +118,19 @@ static int launch_select(const Geom& g, const void* q, const void* k, int topk, 
   return g.nT <= 256 ? launch_score<D, 8>(g, topk, idx, ws, st) : launch_score<D, 16>(g, topk, idx, ws, st);
 }
 
-template <int D, bool SHARED>
+template <int D, int MODE>
 static int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnArgs& a,
                        cudaStream_t st) {
-  const int smem = AttnSmem<D>::kAlloc;
-  if (cudaFuncSetAttribute(attn_fwd_kernel<D, SHARED>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+  const int smem = AttnSmem<D>::alloc(a.g.nT, a.topk, MODE == MODE_PAIR);
+  if (cudaFuncSetAttribute(attn_fwd_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return VSA_ERR_CUDA;
-  const long long tiles = 1ll * a.g.B * a.g.H * a.g.nT;
-  const long long grid = SHARED ? tiles : (tiles + 1) / 2;
-  attn_fwd_kernel<D, SHARED><<<static_cast<unsigned>(grid), kAttnThreads, smem, st>>>(mq, mk, mv, a);
+  const long long BH = 1ll * a.g.B * a.g.H;
+  long long grid;
+  if (MODE == MODE_SHARED) grid = BH * a.g.nT;                             // one tile, two t-halves
+  else if (MODE == MODE_TILE) grid = (BH * a.g.nT + 1) / 2;                // two tiles
+  else grid = (BH * ((a.g.nT + 1) / 2) + 1) / 2;                           // two pairs of tiles
+  attn_fwd_kernel<D, MODE><<<static_cast<unsigned>(grid), kAttnThreads, smem, st>>>(mq, mk, mv, a);
   return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 
@@ -224,6 +228,10 @@ int vsa_attn_fwd(const vsa_shape* shape, const void* q, const void* k, const voi
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
       (reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u))
     return VSA_ERR_ALIGNMENT;
+  const int mode = g.vol == 256 ? MODE_SHARED : (g.vol == 128 ? MODE_TILE : MODE_PAIR);
+  const int smem = g.d == 128 ? AttnSmem<128>::alloc(g.nT, topk, mode == MODE_PAIR)
+                              : AttnSmem<64>::alloc(g.nT, topk, mode == MODE_PAIR);
+  if (smem > kMaxSmemPerBlock) return VSA_ERR_TOO_LARGE;
   if ((rc = check_arch()) != VSA_OK) return rc;
 
   const bool shared = (g.vol == 256);
@@ -242,9 +250,14 @@ int vsa_attn_fwd(const vsa_shape* shape, const void* q, const void* k, const voi
       (rc = encode_qkv_map(&mv, v, g, a.box_t)) != VSA_OK)
     return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (g.d == 128)
-    return shared ? launch_attn<128, true>(mq, mk, mv, a, st) : launch_attn<128, false>(mq, mk, mv, a, st);
-  return shared ? launch_attn<64, true>(mq, mk, mv, a, st) : launch_attn<64, false>(mq, mk, mv, a, st);
+  if (g.d == 128) {
+    if (mode == MODE_SHARED) return launch_attn<128, MODE_SHARED>(mq, mk, mv, a, st);
+    if (mode == MODE_TILE) return launch_attn<128, MODE_TILE>(mq, mk, mv, a, st);
+    return launch_attn<128, MODE_PAIR>(mq, mk, mv, a, st);
+  }
+  if (mode == MODE_SHARED) return launch_attn<64, MODE_SHARED>(mq, mk, mv, a, st);
+  if (mode == MODE_TILE) return launch_attn<64, MODE_TILE>(mq, mk, mv, a, st);
+  return launch_attn<64, MODE_PAIR>(mq, mk, mv, a, st);
 }
 
 int vsa_device_error(uint32_t* code, int32_t reset) {

@@ -68,7 +68,8 @@ typedef enum vsa_status {
   VSA_ERR_WORKSPACE = 5,    /* workspace NULL or smaller than required         */
   VSA_ERR_ARCH = 6,         /* current device is not sm_100                    */
   VSA_ERR_CUDA = 7,         /* a CUDA runtime/driver call failed               */
-  VSA_ERR_TOO_LARGE = 8     /* more than 1536 tiles per head, or B*H > 65535   */
+  VSA_ERR_TOO_LARGE = 8     /* more than 1536 tiles per head, B*H > 65535, or
+                               (64-token tiles) topk too large for shared memory */
 } vsa_status;
 
 /* Tile count of a shape (FastVideo VSA guide, "Wan top-k behavior": num_blocks).

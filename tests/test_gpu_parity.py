@@ -182,3 +182,18 @@ def test_full_size_sweep_all_tiles_is_dense():
         e = np.abs(og[0, bh][rows] - Od)
         assert e.max() <= gu.O_MAX_ABS and e.mean() <= gu.O_MEAN_ABS
         assert np.abs(lg[0, bh][rows] - Ld).max() <= gu.LSE_ABS
+
+
+@pytest.mark.parametrize("chunk", [1, 2, 5])
+def test_forward_host_matches_device_path(chunk):
+    """The pipelined host-to-host call gives the device path's bits."""
+    w = Workload("host_pipe", 2, 3, (9, 20, 20), 128, (4, 8, 8), 5)
+    (q, k, v), (qd, kd, vd) = gu.inputs(w, seed=6)
+    o_ref, l_ref, i_ref = api.forward(qd, kd, vd, w.grid, w.tile, w.topk)
+    hq, hk, hv = (qd.cpu().pin_memory(), kd.cpu().pin_memory(), vd.cpu().pin_memory())
+    o, l, i = api.forward_host(hq, hk, hv, w.grid, w.tile, w.topk, chunk_heads=chunk)
+    torch.cuda.synchronize()
+    gu.assert_no_device_error()
+    assert torch.equal(i, i_ref.cpu())
+    assert torch.equal(o.view(torch.int16), o_ref.cpu().view(torch.int16))
+    assert torch.equal(l, l_ref.cpu())
