@@ -30,6 +30,13 @@ SMALL = [
     Workload("ragged64_d64", 1, 3, (5, 9, 11), 64, (4, 4, 4), 6),
     Workload("vol128", 2, 1, (6, 12, 20), 128, (2, 8, 8), 4),
     Workload("topk1", 1, 2, (9, 20, 20), 128, (4, 8, 8), 1),
+    # 64-token tiles, odd tile count per head: the last pair has no tile B
+    Workload("pair_odd", 1, 3, (4, 4, 20), 128, (4, 4, 4), 3),
+    # 64-token tiles with structured inputs: neighbouring tiles share kept tiles
+    Workload("pair_field", 1, 2, (8, 12, 20), 128, (4, 4, 4), 7, "field"),
+    # 256-token tiles split along t with tt = 2 and with tt = 8
+    Workload("shared_tt2", 1, 2, (7, 16, 24), 128, (2, 8, 16), 5),
+    Workload("shared_tt8", 1, 2, (13, 8, 12), 64, (8, 4, 8), 4),
 ]
 
 
