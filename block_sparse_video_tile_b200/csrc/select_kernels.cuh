@@ -246,8 +246,13 @@ __global__ void __launch_bounds__(kScoreThreads) score_topk_kernel(Geom g, const
   __syncthreads();
 
   const int warp = threadIdx.x / 32;
-  for (int r = warp; r < nrows; r += kScoreThreads / 32)
-    bsearch_topk_row<MAXE>(keys + r * nT, nT, topk, idx + (static_cast<size_t>(bh) * nT + row0 + r) * topk);
+  for (int r = warp; r < nrows; r += kScoreThreads / 32) {
+    int32_t* out = idx + (static_cast<size_t>(bh) * nT + row0 + r) * topk;
+    if (MAXE > 24 && nT <= 32 * 24)   // fewer keys per lane: a shorter unrolled count loop
+      bsearch_topk_row<(MAXE > 24 ? 24 : MAXE)>(keys + r * nT, nT, topk, out);
+    else
+      bsearch_topk_row<MAXE>(keys + r * nT, nT, topk, out);
+  }
 }
 
 template <int D, int R>
