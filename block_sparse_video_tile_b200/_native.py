@@ -24,8 +24,11 @@ EXPORTS = ("vsa_tile_count", "vsa_select_workspace_bytes", "vsa_select", "vsa_se
 SELECT_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
+DTYPE_BF16, DTYPE_F16 = 0, 1
+
+
 class VsaShape(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int32) for n in ("B", "H", "T", "Hh", "W", "d", "tt", "th", "tw")]
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "H", "T", "Hh", "W", "d", "tt", "th", "tw", "dtype")]
 
 
 class VsaError(RuntimeError):

@@ -1,7 +1,7 @@
 """Python entry points over the C ABI, taking torch tensors.
 
 PyTorch provides device memory and the current stream; the work is done by
-libvsa's kernels.  Layouts (see include/vsa.h): Q, K, V, O bfloat16
+libvsa's kernels.  Layouts (see include/vsa.h): Q, K, V, O bfloat16 or float16
 [B, H, N, d] contiguous with raster token order over the latent grid (T, Hh, W);
 idx int32 [B, H, nT, topk]; LSE float32 [B, H, N].
 """
@@ -12,16 +12,19 @@ import math
 
 import torch
 
-from ._native import VsaShape, check, lib
+from ._native import DTYPE_BF16, DTYPE_F16, VsaShape, check, lib
 
 __all__ = ["make_shape", "tile_count", "select", "attn_fwd", "forward", "forward_host",
            "device_error", "select_workspace_bytes"]
 
 
-def make_shape(B: int, H: int, grid, d: int, tile) -> VsaShape:
+_DTYPES = {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_F16}
+
+
+def make_shape(B: int, H: int, grid, d: int, tile, dtype=torch.bfloat16) -> VsaShape:
     T, Hh, W = grid
     tt, th, tw = tile
-    return VsaShape(B, H, T, Hh, W, d, tt, th, tw)
+    return VsaShape(B, H, T, Hh, W, d, tt, th, tw, _DTYPES.get(dtype, -1))
 
 
 def tile_count(grid, tile, d: int = 128, B: int = 1, H: int = 1):
@@ -38,9 +41,11 @@ def select_workspace_bytes(B, H, grid, d, tile) -> int:
     return int(lib().vsa_select_workspace_bytes(ctypes.byref(shp)))
 
 
-def _check_qkv(name, x, B, H, N, d):
-    if not (x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous()):
-        raise ValueError(f"{name} must be a contiguous CUDA bfloat16 tensor")
+def _check_qkv(name, x, B, H, N, d, dtype=None):
+    if not (x.is_cuda and x.dtype in _DTYPES and x.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous CUDA bfloat16 or float16 tensor")
+    if dtype is not None and x.dtype != dtype:
+        raise ValueError(f"{name} is {x.dtype}, expected {dtype} like q")
     if tuple(x.shape) != (B, H, N, d):
         raise ValueError(f"{name} has shape {tuple(x.shape)}, expected {(B, H, N, d)}")
 
@@ -55,8 +60,8 @@ def select(q: torch.Tensor, k: torch.Tensor, grid, tile, topk: int, *, out=None,
     """Top-k key tiles per query tile: int32 [B, H, nT, topk], ascending."""
     B, H, N, d = q.shape
     _check_qkv("q", q, B, H, N, d)
-    _check_qkv("k", k, B, H, N, d)
-    shp = make_shape(B, H, grid, d, tile)
+    _check_qkv("k", k, B, H, N, d, q.dtype)
+    shp = make_shape(B, H, grid, d, tile, q.dtype)
     nT, _ = tile_count(grid, tile, d, B, H)
     if out is None:
         out = torch.empty((B, H, nT, topk), dtype=torch.int32, device=q.device)
@@ -74,7 +79,7 @@ def attn_fwd(q, k, v, idx, grid, tile, *, scale: float | None = None, out=None, 
     """Block-sparse attention over the kept tiles: (O bf16 [B,H,N,d], LSE f32 [B,H,N])."""
     B, H, N, d = q.shape
     for name, x in (("q", q), ("k", k), ("v", v)):
-        _check_qkv(name, x, B, H, N, d)
+        _check_qkv(name, x, B, H, N, d, q.dtype)
     if not (idx.is_cuda and idx.dtype == torch.int32 and idx.is_contiguous() and idx.dim() == 4):
         raise ValueError("idx must be a contiguous CUDA int32 tensor [B, H, nT, topk]")
     topk = idx.shape[-1]
@@ -84,7 +89,9 @@ def attn_fwd(q, k, v, idx, grid, tile, *, scale: float | None = None, out=None, 
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    shp = make_shape(B, H, grid, d, tile)
+    shp = make_shape(B, H, grid, d, tile, q.dtype)
+    if out.dtype != q.dtype:
+        raise ValueError("out must have the dtype of q")
     check("vsa_attn_fwd", lib().vsa_attn_fwd(
         ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(), int(topk),
         float(scale), out.data_ptr(), lse.data_ptr(), _stream(stream)))
@@ -101,8 +108,8 @@ def forward(q, k, v, grid, tile, topk: int, *, scale=None, stream=None):
 class _HostPipeline:
     """Device buffers, streams and events reused by forward_host for one shape."""
 
-    def __init__(self, chunk, N, d, nT, topk, device, ws_bytes):
-        mk = lambda *shape, dt=torch.bfloat16: [torch.empty(shape, dtype=dt, device=device) for _ in range(2)]
+    def __init__(self, chunk, N, d, nT, topk, device, ws_bytes, dtype):
+        mk = lambda *shape, dt=dtype: [torch.empty(shape, dtype=dt, device=device) for _ in range(2)]
         self.q, self.k, self.v, self.o = (mk(1, chunk, N, d) for _ in range(4))
         self.lse = mk(1, chunk, N, dt=torch.float32)
         self.idx = mk(1, chunk, nT, topk, dt=torch.int32)
@@ -110,7 +117,7 @@ class _HostPipeline:
         self.s_in = torch.cuda.Stream(device)
         self.s_comp = torch.cuda.Stream(device)
         self.s_out = torch.cuda.Stream(device)
-        self.key = (chunk, N, d, nT, topk, device)
+        self.key = (chunk, N, d, nT, topk, device, dtype)
 
 
 _PIPE = {}
@@ -131,21 +138,23 @@ def forward_host(q, k, v, grid, tile, topk: int, *, scale=None, chunk_heads: int
     B, H, N, d = q.shape
     device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
     for name, x in (("q", q), ("k", k), ("v", v)):
-        if x.is_cuda or x.dtype != torch.bfloat16 or not x.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous CPU bfloat16 tensor (pinned for overlap)")
+        if x.is_cuda or x.dtype != q.dtype or q.dtype not in _DTYPES or not x.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CPU bfloat16/float16 tensor like q "
+                             "(pinned for overlap)")
     nT, _ = tile_count(grid, tile, d, B, H)
     BH = B * H
     chunk = max(1, min(chunk_heads, BH))
     if out is None:
-        out = torch.empty((B, H, N, d), dtype=torch.bfloat16).pin_memory()
+        out = torch.empty((B, H, N, d), dtype=q.dtype).pin_memory()
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
     if idx is None:
         idx = torch.empty((B, H, nT, topk), dtype=torch.int32).pin_memory()
-    key = (chunk, N, d, nT, topk, device)
+    key = (chunk, N, d, nT, topk, device, q.dtype)
     pipe = _PIPE.get(key)
     if pipe is None:
-        pipe = _HostPipeline(chunk, N, d, nT, topk, device, select_workspace_bytes(1, chunk, grid, d, tile))
+        pipe = _HostPipeline(chunk, N, d, nT, topk, device, select_workspace_bytes(1, chunk, grid, d, tile),
+                             q.dtype)
         _PIPE.clear()
         _PIPE[key] = pipe
     caller = torch.cuda.current_stream(device)

@@ -69,7 +69,7 @@ struct AttnArgs {
   int topk;
   float scale_log2;          // softmax_scale * log2(e)
   const int32_t* idx;        // [B*H, nT, topk]
-  __nv_bfloat16* o;          // [B*H, N, d]
+  uint16_t* o;               // [B*H, N, d], bf16 or fp16 like the inputs
   float* lse;                // [B*H, N]
   unsigned int* err;         // device error word
   int box_t;                 // t-extent of one TMA box (tt/2 in MODE_SHARED, else tt)
@@ -256,7 +256,7 @@ __device__ __forceinline__ int build_union(const AttnArgs& a, const int32_t* row
   return base;
 }
 
-template <int D, int MODE>
+template <int D, int MODE, bool F16>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
@@ -446,8 +446,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   } else if (warp == 9) {
     // ====================================================== MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(kSlotRows, kSubRows, false);
-      constexpr uint32_t idPV = idesc_bf16_f32(kSlotRows, D, true);
+      constexpr uint32_t idS = idesc_f16kind_f32(kSlotRows, kSubRows, false, F16);
+      constexpr uint32_t idPV = idesc_f16kind_f32(kSlotRows, D, true, F16);
       int n[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -659,7 +659,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               p1 = ex2_approx(x1);
             }
             ls2[c & 3] = f2_add(ls2[c & 3], f2_pack(p0, p1));
-            s[c] = kPackAlu ? pack_bf16x2_alu(p0, p1) : pack_bf16x2(p0, p1);
+            s[c] = (kPackAlu && !F16) ? pack_bf16x2_alu(p0, p1) : pack_elem2<F16>(p0, p1);
           }
         }
         {
@@ -693,7 +693,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const float inv_l = 1.f / l;
         const size_t N = static_cast<size_t>(g.T) * g.Hh * g.W;
         const size_t n_tok = (static_cast<size_t>(tok_t) * g.Hh + tok_y) * g.W + tok_x;
-        __nv_bfloat16* orow = a.o + (static_cast<size_t>(me.bh) * N + n_tok) * D;
+        uint16_t* orow = a.o + (static_cast<size_t>(me.bh) * N + n_tok) * D;
 #pragma unroll
         for (int c4 = 0; c4 < D / 32; ++c4) {
           uint32_t ov[32];
@@ -703,7 +703,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             uint32_t pk[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e)
-              pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l, __uint_as_float(ov[2 * e + 1]) * inv_l);
+              pk[e] = pack_elem2<F16>(__uint_as_float(ov[2 * e]) * inv_l, __uint_as_float(ov[2 * e + 1]) * inv_l);
             // streaming stores: O is not read again by this kernel, so it
             // should not sit dirty in L2 for whatever kernel runs next
             uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c4);

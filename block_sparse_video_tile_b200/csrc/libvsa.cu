@@ -30,6 +30,7 @@ static int make_geom(const vsa_shape* s, Geom* g) {
       s->th <= 0 || s->tw <= 0)
     return VSA_ERR_INVALID_ARG;
   if (s->d != 64 && s->d != 128) return VSA_ERR_UNSUPPORTED;
+  if (s->dtype != VSA_DTYPE_BF16 && s->dtype != VSA_DTYPE_F16) return VSA_ERR_UNSUPPORTED;
   const int lt = ilog2_exact(s->tt), ly = ilog2_exact(s->th), lx = ilog2_exact(s->tw);
   if (lt < 0 || ly < 0 || lx < 0) return VSA_ERR_UNSUPPORTED;
   if (s->tt > 256 || s->th > 256 || s->tw > 256) return VSA_ERR_UNSUPPORTED;
@@ -40,6 +41,7 @@ static int make_geom(const vsa_shape* s, Geom* g) {
   g->tt = s->tt; g->th = s->th; g->tw = s->tw;
   g->lg_tt = lt; g->lg_th = ly; g->lg_tw = lx;
   g->vol = vol;
+  g->f16 = s->dtype == VSA_DTYPE_F16 ? 1 : 0;
   g->nTt = ceil_div(s->T, s->tt);
   g->nTy = ceil_div(s->Hh, s->th);
   g->nTx = ceil_div(s->W, s->tw);
@@ -100,29 +102,29 @@ static int launch_score(const Geom& g, int topk, int32_t* idx, const float* ws, 
                                                                                                : VSA_ERR_CUDA;
 }
 
-template <int D>
+template <int D, bool F16>
 static int launch_select(const Geom& g, const void* q, const void* k, int topk, int32_t* idx, float* ws,
                          cudaStream_t st) {
   CUtensorMap mq, mk;
   int rc;
-  if ((rc = encode_qkv_map(&mq, q, g, g.tt)) != VSA_OK || (rc = encode_qkv_map(&mk, k, g, g.tt)) != VSA_OK)
+  if ((rc = encode_qkv_map(&mq, q, g, g.tt, F16)) != VSA_OK || (rc = encode_qkv_map(&mk, k, g, g.tt, F16)) != VSA_OK)
     return rc;
   unsigned int* err = device_error_ptr();
   if (err == nullptr) return VSA_ERR_CUDA;
   const size_t psmem = pool_smem_bytes<D>(g);
-  if (cudaFuncSetAttribute(pool_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(pool_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(psmem)) != cudaSuccess)
     return VSA_ERR_CUDA;
-  pool_kernel<D><<<dim3(g.nT, g.B * g.H, 2), kPoolThreads, psmem, st>>>(mq, mk, g, ws, err);
+  pool_kernel<D, F16><<<dim3(g.nT, g.B * g.H, 2), kPoolThreads, psmem, st>>>(mq, mk, g, ws, err);
   if (cudaGetLastError() != cudaSuccess) return VSA_ERR_CUDA;
   return g.nT <= 256 ? launch_score<D, 8>(g, topk, idx, ws, st) : launch_score<D, 16>(g, topk, idx, ws, st);
 }
 
-template <int D, int MODE>
+template <int D, int MODE, bool F16>
 static int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnArgs& a,
                        cudaStream_t st) {
   const int smem = AttnSmem<D>::alloc(a.g.nT, a.topk, MODE == MODE_PAIR);
-  if (cudaFuncSetAttribute(attn_fwd_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+  if (cudaFuncSetAttribute(attn_fwd_kernel<D, MODE, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return VSA_ERR_CUDA;
   const long long BH = 1ll * a.g.B * a.g.H;
@@ -130,7 +132,7 @@ static int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   if (MODE == MODE_SHARED) grid = BH * a.g.nT;                             // one tile, two t-halves
   else if (MODE == MODE_TILE) grid = (BH * a.g.nT + 1) / 2;                // two tiles
   else grid = (BH * ((a.g.nT + 1) / 2) + 1) / 2;                           // two pairs of tiles
-  attn_fwd_kernel<D, MODE><<<static_cast<unsigned>(grid), kAttnThreads, smem, st>>>(mq, mk, mv, a);
+  attn_fwd_kernel<D, MODE, F16><<<static_cast<unsigned>(grid), kAttnThreads, smem, st>>>(mq, mk, mv, a);
   return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 
@@ -154,6 +156,27 @@ static int select_scratch_ptr(float** out) {
   }
   *out = cached[dev];
   return VSA_OK;
+}
+
+template <bool F16>
+static int dispatch_attn(int d, int mode, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         const AttnArgs& a, cudaStream_t st) {
+  if (d == 128) {
+    if (mode == MODE_SHARED) return launch_attn<128, MODE_SHARED, F16>(mq, mk, mv, a, st);
+    if (mode == MODE_TILE) return launch_attn<128, MODE_TILE, F16>(mq, mk, mv, a, st);
+    return launch_attn<128, MODE_PAIR, F16>(mq, mk, mv, a, st);
+  }
+  if (mode == MODE_SHARED) return launch_attn<64, MODE_SHARED, F16>(mq, mk, mv, a, st);
+  if (mode == MODE_TILE) return launch_attn<64, MODE_TILE, F16>(mq, mk, mv, a, st);
+  return launch_attn<64, MODE_PAIR, F16>(mq, mk, mv, a, st);
+}
+
+static int dispatch_select(const Geom& g, const void* q, const void* k, int topk, int32_t* idx, float* ws,
+                           cudaStream_t st) {
+  if (g.d == 128) return g.f16 ? launch_select<128, true>(g, q, k, topk, idx, ws, st)
+                               : launch_select<128, false>(g, q, k, topk, idx, ws, st);
+  return g.f16 ? launch_select<64, true>(g, q, k, topk, idx, ws, st)
+               : launch_select<64, false>(g, q, k, topk, idx, ws, st);
 }
 
 }  // namespace vsa
@@ -195,8 +218,7 @@ int vsa_select(const vsa_shape* shape, const void* q, const void* k, int32_t top
   if ((rc = check_arch()) != VSA_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* ws = static_cast<float*>(workspace);
-  return g.d == 128 ? launch_select<128>(g, q, k, topk, idx_out, ws, st)
-                    : launch_select<64>(g, q, k, topk, idx_out, ws, st);
+  return dispatch_select(g, q, k, topk, idx_out, ws, st);
 }
 
 int vsa_select_noalloc(const vsa_shape* shape, const void* q, const void* k, int32_t topk, int32_t* idx_out,
@@ -212,8 +234,7 @@ int vsa_select_noalloc(const vsa_shape* shape, const void* q, const void* k, int
   float* ws = nullptr;
   if ((rc = select_scratch_ptr(&ws)) != VSA_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return g.d == 128 ? launch_select<128>(g, q, k, topk, idx_out, ws, st)
-                    : launch_select<64>(g, q, k, topk, idx_out, ws, st);
+  return dispatch_select(g, q, k, topk, idx_out, ws, st);
 }
 
 int vsa_attn_fwd(const vsa_shape* shape, const void* q, const void* k, const void* v, const int32_t* idx,
@@ -240,24 +261,19 @@ int vsa_attn_fwd(const vsa_shape* shape, const void* q, const void* k, const voi
   a.topk = topk;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
   a.idx = idx;
-  a.o = static_cast<__nv_bfloat16*>(o);
+  a.o = static_cast<uint16_t*>(o);
   a.lse = lse;
   a.err = device_error_ptr();
   a.box_t = shared ? g.tt / 2 : g.tt;
   if (a.err == nullptr) return VSA_ERR_CUDA;
   CUtensorMap mq, mk, mv;
-  if ((rc = encode_qkv_map(&mq, q, g, a.box_t)) != VSA_OK || (rc = encode_qkv_map(&mk, k, g, a.box_t)) != VSA_OK ||
-      (rc = encode_qkv_map(&mv, v, g, a.box_t)) != VSA_OK)
+  const bool f16 = g.f16 != 0;
+  if ((rc = encode_qkv_map(&mq, q, g, a.box_t, f16)) != VSA_OK ||
+      (rc = encode_qkv_map(&mk, k, g, a.box_t, f16)) != VSA_OK ||
+      (rc = encode_qkv_map(&mv, v, g, a.box_t, f16)) != VSA_OK)
     return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (g.d == 128) {
-    if (mode == MODE_SHARED) return launch_attn<128, MODE_SHARED>(mq, mk, mv, a, st);
-    if (mode == MODE_TILE) return launch_attn<128, MODE_TILE>(mq, mk, mv, a, st);
-    return launch_attn<128, MODE_PAIR>(mq, mk, mv, a, st);
-  }
-  if (mode == MODE_SHARED) return launch_attn<64, MODE_SHARED>(mq, mk, mv, a, st);
-  if (mode == MODE_TILE) return launch_attn<64, MODE_TILE>(mq, mk, mv, a, st);
-  return launch_attn<64, MODE_PAIR>(mq, mk, mv, a, st);
+  return f16 ? dispatch_attn<true>(g.d, mode, mq, mk, mv, a, st) : dispatch_attn<false>(g.d, mode, mq, mk, mv, a, st);
 }
 
 int vsa_device_error(uint32_t* code, int32_t reset) {

@@ -33,7 +33,7 @@ constexpr int kPoolThreads = 256;
 // zeros and add nothing to the sums.  Threads then sum 16-byte chunks down the
 // rows in a fixed order (deterministic) and divide by the tile's valid count.
 // Dynamic shared memory: box (slabs x vol x 128 B, 1024-aligned) | partial sums | mbarrier.
-template <int D>
+template <int D, bool F16>
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                             const __grid_constant__ CUtensorMap tmK, Geom g,
                                                             float* __restrict__ pooled, unsigned int* err) {
@@ -76,10 +76,10 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __grid_constan
 #pragma unroll 4
     for (int r = rg; r < vol; r += RP) {
       const uint4 u = *reinterpret_cast<const uint4*>(slab + r * 128 + (((cc % 8) ^ (r & 7)) << 4));
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(h2[e]);
+        const float2 f = unpack_elem2<F16>(w4[e]);
         acc[2 * e] += f.x;
         acc[2 * e + 1] += f.y;
       }

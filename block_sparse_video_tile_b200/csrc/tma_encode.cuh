@@ -35,7 +35,7 @@ inline EncodeTiledFn get_encode_fn() {
 
 // [B*H, T, Hh, W, d] bf16 viewed as a 5-D tensor (d innermost); box = 64
 // channels x (tw, th, box_t) tokens, 128-byte swizzle, zero fill past edges.
-inline int encode_qkv_map(CUtensorMap* m, const void* ptr, const Geom& g, int box_t) {
+inline int encode_qkv_map(CUtensorMap* m, const void* ptr, const Geom& g, int box_t, bool f16 = false) {
   EncodeTiledFn fn = get_encode_fn();
   if (fn == nullptr) return VSA_ERR_CUDA;
   const cuuint64_t e = 2;
@@ -46,7 +46,7 @@ inline int encode_qkv_map(CUtensorMap* m, const void* ptr, const Geom& g, int bo
   cuuint32_t box[5] = {64u, static_cast<cuuint32_t>(g.tw), static_cast<cuuint32_t>(g.th),
                        static_cast<cuuint32_t>(box_t), 1u};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box, estr,
+  CUresult r = fn(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? VSA_OK : VSA_ERR_CUDA;

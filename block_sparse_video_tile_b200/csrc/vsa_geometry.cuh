@@ -21,6 +21,7 @@ struct Geom {
   int nTt, nTy, nTx, nT;  // tiles per axis and in total
   int lg_tt, lg_th, lg_tw;  // log2 of the (power-of-two) tile extents
   int vol;                  // tt * th * tw
+  int f16;                  // element type: 0 bfloat16, 1 float16
 };
 
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }

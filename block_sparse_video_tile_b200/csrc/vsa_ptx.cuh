@@ -9,6 +9,7 @@
 
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace vsa {
 
@@ -204,12 +205,13 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
-// Instruction descriptor for kind::f16 with bf16 A/B and f32 accumulate.
-// b_mn_major: B operand stored with N contiguous (e.g. V as [kv][d]).
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
+// Instruction descriptor for kind::f16 with bf16 (or fp16: f16 = true) A/B
+// and f32 accumulate.  b_mn_major: B operand stored with N contiguous (e.g. V
+// as [kv][d]).  A and B always have the same type.
+__host__ __device__ constexpr uint32_t idesc_f16kind_f32(int M, int N, bool b_mn_major, bool f16) {
   return (1u << 4)                       // D format f32
-         | (1u << 7)                     // A format bf16
-         | (1u << 10)                    // B format bf16
+         | ((f16 ? 0u : 1u) << 7)        // A format: 0 fp16, 1 bf16
+         | ((f16 ? 0u : 1u) << 10)       // B format: same as A
          | ((b_mn_major ? 1u : 0u) << 16)
          | (static_cast<uint32_t>(N >> 3) << 17)
          | (static_cast<uint32_t>(M >> 4) << 24);
@@ -303,9 +305,38 @@ __device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
   return __byte_perm(a, b, 0x7632);
 }
 
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
+  return idesc_f16kind_f32(M, N, b_mn_major, false);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Two float32 -> the 16-bit element type of the inputs (bf16 or fp16), packed.
+template <bool F16>
+__device__ __forceinline__ uint32_t pack_elem2(float lo, float hi);
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <>
+__device__ __forceinline__ uint32_t pack_elem2<false>(float lo, float hi) {
+  return pack_bf16x2(lo, hi);
+}
+template <>
+__device__ __forceinline__ uint32_t pack_elem2<true>(float lo, float hi) {
+  return pack_f16x2(lo, hi);
+}
+
+// Two packed 16-bit elements (bf16 or fp16) -> float2.
+template <bool F16>
+__device__ __forceinline__ float2 unpack_elem2(uint32_t v) {
+  if (F16) return __half22float2(*reinterpret_cast<const __half2*>(&v));
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v));
 }
 
 }  // namespace vsa

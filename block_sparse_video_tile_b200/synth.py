@@ -27,7 +27,7 @@ from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["f32_to_bf16_bits", "bf16_bits_to_f32", "make_qkv", "N_SINUSOIDS"]
+__all__ = ["f32_to_bf16_bits", "f32_to_f16_bits", "bf16_bits_to_f32", "make_qkv", "N_SINUSOIDS"]
 
 N_SINUSOIDS = 8
 
@@ -37,6 +37,11 @@ def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
     rounding = np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))
     return ((u + rounding) >> np.uint32(16)).astype(np.uint16)
+
+
+def f32_to_f16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to IEEE half precision (nearest, ties to even); return the bits."""
+    return np.ascontiguousarray(x, dtype=np.float32).astype(np.float16).view(np.uint16)
 
 
 def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
@@ -74,8 +79,9 @@ def _field_head(freq: np.ndarray, phase: np.ndarray, grid: tuple) -> np.ndarray:
 
 
 def make_qkv(B: int, H: int, grid: tuple, d: int, seed: int = 0,
-             kind: str = "normal"):
-    """Return (q, k, v) as uint16 bfloat16-bit arrays of shape [B, H, N, d].
+             kind: str = "normal", dtype: str = "bf16"):
+    """Return (q, k, v) as uint16 arrays of shape [B, H, N, d] holding bfloat16
+    bit patterns (dtype "bf16") or IEEE half-precision ones ("f16").
 
     Values are drawn head by head in (b, h) order within each tensor; a
     Generator fills consecutive draws from one stream, so this equals drawing
@@ -85,11 +91,12 @@ def make_qkv(B: int, H: int, grid: tuple, d: int, seed: int = 0,
     N = T * Hh * W
     rng = np.random.Generator(np.random.PCG64(seed))
     out = [np.empty((B, H, N, d), dtype=np.uint16) for _ in range(3)]
+    to_bits = f32_to_f16_bits if dtype == "f16" else f32_to_bf16_bits
     if kind == "normal":
         for x in out:
             for b in range(B):
                 for h in range(H):
-                    x[b, h] = f32_to_bf16_bits(rng.standard_normal((N, d), dtype=np.float32))
+                    x[b, h] = to_bits(rng.standard_normal((N, d), dtype=np.float32))
         return tuple(out)
     if kind == "field":
         freq, phase = _field_params(rng, B, H, d)
@@ -98,9 +105,9 @@ def make_qkv(B: int, H: int, grid: tuple, d: int, seed: int = 0,
                 for h in range(H):
                     fld = _field_head(freq[b, h], phase[b, h], grid)
                     noise = rng.standard_normal((N, d), dtype=np.float32)
-                    x[b, h] = f32_to_bf16_bits(fld + np.float32(0.5) * noise)
+                    x[b, h] = to_bits(fld + np.float32(0.5) * noise)
         for b in range(B):
             for h in range(H):
-                out[2][b, h] = f32_to_bf16_bits(rng.standard_normal((N, d), dtype=np.float32))
+                out[2][b, h] = to_bits(rng.standard_normal((N, d), dtype=np.float32))
         return tuple(out)
     raise ValueError(f"unknown input kind {kind!r}")

@@ -33,6 +33,7 @@ class Workload:
     tile: tuple
     topk: int
     kind: str = "normal"
+    dtype: str = "bf16"        # element type of Q, K, V, O: "bf16" or "f16"
 
     @property
     def N(self) -> int:

@@ -14,7 +14,8 @@
  * Conventions shared by every call
  * --------------------------------
  * Tensors are dense, row-major, on the current CUDA device:
- *   Q, K, V, O : bfloat16 [B, H, N, d], N = T*Hh*W, token n = (t*Hh + y)*W + x
+ *   Q, K, V, O : bfloat16 or float16 (vsa_shape.dtype) [B, H, N, d],
+ *                N = T*Hh*W, token n = (t*Hh + y)*W + x
  *                (raster order over the grid; no permutation to tile order is
  *                 needed -- the kernels evaluate the tile index map themselves,
  *                 as the fastbsa page's "How it works" describes)
@@ -26,7 +27,8 @@
  * their missing tokens are left out of pooling and of the softmax.  Tile
  * j = (bt * ceil(Hh/th) + by) * ceil(W/tw) + bx (raster over tile coordinates).
  *
- * Supported: d in {64, 128}; tt, th, tw powers of two with tt*th*tw in
+ * Supported: bf16 or fp16 inputs (O has the input type; pooling, scores,
+ * softmax and accumulation are float32); d in {64, 128}; tt, th, tw powers of two with tt*th*tw in
  * {64, 128, 256} (the guide's 4x4x4 = 64 and 4x8x8 = 256 blocks), and tt >= 2
  * when tt*th*tw = 256; H_q = H_kv; non-causal self-attention, no mask.
  * Inputs must be finite (NaN/Inf give unspecified results, never a fault).
@@ -56,14 +58,21 @@ typedef struct vsa_shape {
   int32_t T, Hh, W;      /* post-patch latent grid                            */
   int32_t d;             /* head dimension: 64 or 128                         */
   int32_t tt, th, tw;    /* tile extents along T, Hh, W                        */
+  int32_t dtype;         /* element type of Q, K, V, O: VSA_DTYPE_BF16 (0, the
+                            default of a zeroed struct) or VSA_DTYPE_F16      */
 } vsa_shape;
+
+/* Element types (FastVideo VSA guide, "Verify routing and fallback": the
+ * Wan route takes FP16 or BF16 tensors). */
+#define VSA_DTYPE_BF16 0
+#define VSA_DTYPE_F16 1
 
 typedef enum vsa_status {
   VSA_OK = 0,
   VSA_ERR_INVALID_ARG = 1,  /* NULL pointer, non-positive extent, bad scale    */
   VSA_ERR_TOPK_RANGE = 2,   /* topk <= 0 or topk > nT (guide: topk must be
                                positive; topk > num_blocks is invalid)         */
-  VSA_ERR_UNSUPPORTED = 3,  /* d or tile shape outside the supported set       */
+  VSA_ERR_UNSUPPORTED = 3,  /* d, dtype or tile shape outside the supported set */
   VSA_ERR_ALIGNMENT = 4,    /* a tensor pointer not 16-byte aligned            */
   VSA_ERR_WORKSPACE = 5,    /* workspace NULL or smaller than required         */
   VSA_ERR_ARCH = 6,         /* current device is not sm_100                    */
@@ -83,7 +92,7 @@ size_t vsa_select_workspace_bytes(const vsa_shape* shape);
 
 /* Tile selection (FastVideo VSA guide intro and "Wan top-k behavior"; fastbsa
  * page "How it works": selection kept on chip, no score matrix in HBM).
- *   q, k      : device bfloat16 [B, H, N, d], 16-byte aligned
+ *   q, k      : device [B, H, N, d] of shape->dtype, 16-byte aligned
  *   topk      : kept key tiles per query tile, 1 <= topk <= nT
  *               (topk == nT keeps every tile: the dense case)
  *   idx_out   : device int32 [B, H, nT, topk]; row i gets the topk tiles j with
@@ -124,12 +133,12 @@ int vsa_select_noalloc(const vsa_shape* shape, const void* q, const void* k, int
 /* Block-sparse attention forward (FastVideo VSA guide intro: attention only
  * against the selected top-k blocks; "Verify routing and fallback": scale
  * head_size ** -0.5 by default, non-causal, no mask).
- *   q, k, v       : device bfloat16 [B, H, N, d], 16-byte aligned
+ *   q, k, v       : device [B, H, N, d] of shape->dtype, 16-byte aligned
  *   idx           : device int32 [B, H, nT, topk], ascending distinct tiles
  *                   (as vsa_select writes them); an entry outside [0, nT)
  *                   raises a device error and is read as tile 0 instead
  *   softmax_scale : > 0 and finite; pass d ** -0.5 for the standard scale
- *   o             : device bfloat16 [B, H, N, d] out, 16-byte aligned
+ *   o             : device [B, H, N, d] out, same type as q, 16-byte aligned
  *   lse           : device float32 [B, H, N] out, natural log
  * For every token n of query tile i: O[n] = softmax_m(scale * Q[n].K[m]) V[m]
  * over the valid tokens m of the tiles idx[i, :]; LSE[n] = log of the

@@ -3,8 +3,8 @@
 TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import this module:
 only the tests, the package's smoke check and the benchmark's CPU-baseline leg
 call it.  It shares no code with the CUDA library (its own geometry, its own
-pooling, scoring, selection and softmax), and takes its inputs as bfloat16 bit
-patterns widened exactly to float64.
+pooling, scoring, selection and softmax), and takes its inputs as bfloat16 or
+float16 bit patterns widened exactly to float64.
 
 What it computes, and where the pages fix each step:
 
@@ -48,6 +48,16 @@ def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
     """Widen bfloat16 bit patterns (uint16) exactly to float64."""
     u32 = bits.astype(np.uint32) << np.uint32(16)
     return u32.view(np.float32).astype(np.float64)
+
+
+def f16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Widen IEEE half-precision bit patterns (uint16) exactly to float64."""
+    return np.ascontiguousarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
+def widen(bits: np.ndarray, dtype: str = "bf16") -> np.ndarray:
+    """Exact float64 values of 16-bit inputs ("bf16" or "f16" bit patterns)."""
+    return f16_to_f64(bits) if dtype == "f16" else bf16_to_f64(bits)
 
 
 # ------------------------------------------------------------------- geometry
@@ -126,7 +136,7 @@ def select_head(Q: np.ndarray, K: np.ndarray, grid, tile, topk: int):
     return idx, s, near
 
 
-def select(q_bits, k_bits, grid, tile, topk: int):
+def select(q_bits, k_bits, grid, tile, topk: int, dtype: str = "bf16"):
     """All (b, h): idx [B, H, nT, topk], scores [B, H, nT, nT], near_tie [B, H, nT]."""
     B, H = q_bits.shape[:2]
     nT = num_tiles(grid, tile)
@@ -136,7 +146,7 @@ def select(q_bits, k_bits, grid, tile, topk: int):
     for b in range(B):
         for h in range(H):
             idx[b, h], sc[b, h], near[b, h] = select_head(
-                bf16_to_f64(q_bits[b, h]), bf16_to_f64(k_bits[b, h]), grid, tile, topk)
+                widen(q_bits[b, h], dtype), widen(k_bits[b, h], dtype), grid, tile, topk)
     return idx, sc, near
 
 

@@ -20,8 +20,9 @@ O_MEAN_ABS = 2e-3
 LSE_ABS = 1e-3
 
 
-def to_dev(bits: np.ndarray) -> torch.Tensor:
-    return torch.from_numpy(np.ascontiguousarray(bits)).view(torch.bfloat16).cuda()
+def to_dev(bits: np.ndarray, dtype: str = "bf16") -> torch.Tensor:
+    t = torch.float16 if dtype == "f16" else torch.bfloat16
+    return torch.from_numpy(np.ascontiguousarray(bits)).view(t).cuda()
 
 
 _CACHE = {}
@@ -30,13 +31,13 @@ _CACHE = {}
 def inputs(w, seed=0):
     """((q, k, v) host bf16 bits, (q, k, v) device bf16); the last two input
     sets are kept so that tests on the same workload do not redraw them."""
-    key = (w.B, w.H, w.grid, w.d, w.kind, seed)
+    key = (w.B, w.H, w.grid, w.d, w.kind, seed, w.dtype)
     if key not in _CACHE:
         if len(_CACHE) >= 2:
             _CACHE.pop(next(iter(_CACHE)))
-        _CACHE[key] = synth.make_qkv(w.B, w.H, w.grid, w.d, seed=seed, kind=w.kind)
+        _CACHE[key] = synth.make_qkv(w.B, w.H, w.grid, w.d, seed=seed, kind=w.kind, dtype=w.dtype)
     q, k, v = _CACHE[key]
-    return (q, k, v), tuple(to_dev(x) for x in (q, k, v))
+    return (q, k, v), tuple(to_dev(x, w.dtype) for x in (q, k, v))
 
 
 def oracle_scores(q, k, w):
@@ -45,7 +46,7 @@ def oracle_scores(q, k, w):
     out = []
     for b in range(B):
         for h in range(H):
-            Q, K = vo.bf16_to_f64(q[b, h]), vo.bf16_to_f64(k[b, h])
+            Q, K = vo.widen(q[b, h], w.dtype), vo.widen(k[b, h], w.dtype)
             out.append(vo.tile_scores(vo.pool(Q, w.grid, w.tile), vo.pool(K, w.grid, w.tile)))
     nT = out[0].shape[0]
     return np.stack(out).reshape(B, H, nT, nT)
@@ -82,7 +83,7 @@ def check_attention(o_gpu, lse_gpu, q, k, v, w, idx, scale, tiles=None):
     for b, h, i in tiles:
         by_head.setdefault((b, h), []).append(i)
     for (b, h), ts in by_head.items():
-        Q, K, V = (vo.bf16_to_f64(x[b, h]) for x in (q, k, v))
+        Q, K, V = (vo.widen(x[b, h], w.dtype) for x in (q, k, v))
         O, L = vo.attend_head(Q, K, V, w.grid, w.tile, idx[b, h], scale, query_tiles=ts)
         rows = np.concatenate([toks[i] for i in ts])
         errs.append(np.abs(o_gpu[b, h][rows] - O[rows]))

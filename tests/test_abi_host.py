@@ -7,6 +7,7 @@ import re
 
 import numpy as np
 import pytest
+import torch
 
 from block_sparse_video_tile_b200 import _native, api
 from block_sparse_video_tile_b200.workloads import ALL
@@ -53,6 +54,7 @@ def test_tile_count_matches_oracle(name):
 @pytest.mark.parametrize("kw,status", [
     (dict(d=96), 3), (dict(d=0), 1), (dict(tile=(3, 8, 8)), 3), (dict(tile=(1, 16, 16)), 3),
     (dict(tile=(4, 8, 16)), 3), (dict(grid=(0, 22, 40)), 1), (dict(tile=(8, 8, 8)), 3),
+    (dict(dtype=torch.float32), 3),
 ])
 def test_unsupported_shapes(kw, status):
     args = dict(B=1, H=1, grid=(31, 22, 40), d=128, tile=(4, 8, 8))
@@ -118,3 +120,10 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
     assert L.vsa_select_noalloc(ctypes.byref(big), 256, 512, 4, 1024, None) == 5
     assert L.vsa_select_noalloc(ctypes.byref(small), 256, 512, 0, 1024, None) == 2
     assert L.vsa_select_noalloc(ctypes.byref(small), 8, 512, 4, 1024, None) == 4
+
+
+def test_f16_shape_accepted():
+    shp = api.make_shape(1, 2, (31, 22, 40), 128, (4, 8, 8), torch.float16)
+    assert shp.dtype == _native.DTYPE_F16
+    n = ctypes.c_int32()
+    assert _native.lib().vsa_tile_count(ctypes.byref(shp), ctypes.byref(n), None) == 0 and n.value == 120

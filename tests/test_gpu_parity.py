@@ -37,6 +37,10 @@ SMALL = [
     # 256-token tiles split along t with tt = 2 and with tt = 8
     Workload("shared_tt2", 1, 2, (7, 16, 24), 128, (2, 8, 16), 5),
     Workload("shared_tt8", 1, 2, (13, 8, 12), 64, (8, 4, 8), 4),
+    # float16 inputs (the Wan route takes FP16 or BF16) in each kernel mode
+    Workload("f16_shared", 1, 2, (9, 20, 20), 128, (4, 8, 8), 5, dtype="f16"),
+    Workload("f16_tile_d64", 2, 1, (6, 12, 20), 64, (2, 8, 8), 4, dtype="f16"),
+    Workload("f16_pair", 1, 2, (6, 10, 14), 128, (4, 4, 4), 5, "field", dtype="f16"),
 ]
 
 
@@ -87,7 +91,7 @@ def test_all_tiles_equal_dense(w):
     og, lg = o.float().cpu().numpy(), lse.cpu().numpy()
     for b in range(w.B):
         for h in range(w.H):
-            Od, Ld = vo.dense_bruteforce(*(vo.bf16_to_f64(x[b, h]) for x in (q, k, v)), scale)
+            Od, Ld = vo.dense_bruteforce(*(vo.widen(x[b, h], w.dtype) for x in (q, k, v)), scale)
             e = np.abs(og[b, h] - Od)
             assert e.max() <= gu.O_MAX_ABS and e.mean() <= gu.O_MEAN_ABS
             assert np.abs(lg[b, h] - Ld).max() <= gu.LSE_ABS
@@ -129,7 +133,7 @@ def test_bad_topk_raises():
 
 
 # ----------------------------------------------------------- full-size workloads
-FULL = [WAN5B, WAN14B, LONGCAT]
+FULL = [WAN5B, WAN14B, LONGCAT, WAN5B.with_(name="wan5b_f16", dtype="f16")]
 
 
 def _sample_tiles(w, rng, n_heads=2, n_tiles=4):
@@ -184,7 +188,7 @@ def test_full_size_sweep_all_tiles_is_dense():
     scale = w.d ** -0.5
     for bh in (0, 17):
         rows = np.concatenate([[0, w.N - 1], rng.choice(w.N, 30, replace=False)])
-        Q, K, V = (vo.bf16_to_f64(x[0, bh]) for x in (q, k, v))
+        Q, K, V = (vo.widen(x[0, bh], w.dtype) for x in (q, k, v))
         Od, Ld = vo.dense_bruteforce(Q[rows], K, V, scale)
         e = np.abs(og[0, bh][rows] - Od)
         assert e.max() <= gu.O_MAX_ABS and e.mean() <= gu.O_MEAN_ABS

@@ -297,3 +297,14 @@ def test_workload_table():
     for w in ALL.values():
         if w.name.startswith("sweep"):
             assert vo.num_tiles(w.grid, w.tile) == 120 and w.topk in (8, 16, 32, 64, 120)
+
+
+def test_f16_widening_textbook_values():
+    """IEEE binary16 encodings: 1.0, -2.0, the largest finite 65504, the
+    smallest subnormal 2^-24, and round-to-nearest-even at a tie."""
+    bits = np.array([0x3C00, 0xC000, 0x7BFF, 0x0001, 0x3555], dtype=np.uint16)
+    np.testing.assert_array_equal(vo.f16_to_f64(bits)[:4], [1.0, -2.0, 65504.0, 2.0 ** -24])
+    assert abs(vo.f16_to_f64(bits)[4] - 1 / 3) < 2 ** -11
+    # 1 + 2^-11 lies halfway between 1 and 1 + 2^-10: ties round to the even one (1.0)
+    assert synth.f32_to_f16_bits(np.array([1 + 2 ** -11], np.float32))[0] == 0x3C00
+    assert synth.f32_to_f16_bits(np.array([1 + 3 * 2 ** -11], np.float32))[0] == 0x3C02
