@@ -23,7 +23,7 @@
 // (thread = query row = TMEM lane), warp 8 TMA producer, warp 9 MMA issuer,
 // warps 10-11 idle.  The producer warpgroup gives registers to the softmax
 // warpgroups (setmaxnreg): 2*128*208 + 128*80 = 63488 <= 384*168, the launch budget.
-// TMEM (512 columns): S_h at [128h, 128h+128), P_h (bf16 pairs) aliases the
+// TMEM (512 columns): S_h at [128h, 128h+128), P_h (16-bit pairs) aliases the
 // first 64 columns of S_h, O_h at [256 + 128h, ...).  The MMA warp issues, per
 // K/V sub-block: PV_0(prev), S_0(cur), PV_1(prev), S_1(cur); tcgen05.mma ops
 // from one thread execute in issue order, so S_h(cur) overwrites P_h(prev)
@@ -687,7 +687,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_arrive(bar(BAR_P_FULL + h));
       }
 
-      // ---- epilogue: O / l -> bf16, LSE
+      // ---- epilogue: O / l -> the input type, LSE
       if (ok && __all_sync(0xffffffffu, mbar_wait(bar(BAR_O_FULL + h), 0, abort_flag, a.err))) {
         tc_fence_after();
         const float inv_l = 1.f / l;
