@@ -353,7 +353,7 @@ def run_ours(args, w, rank, world, device):
         "config": {"workload": describe(w), "parallelism": f"replicas x{world} (heads shard, no exchange)",
                    "l2": "inputs 3 x %.1f MB > 126 MB L2; no flush" % (w.B * w.H * w.N * w.d * 2 / 1e6),
                    "inputs": ("structured field + noise (torch, on device)" if w.kind == "field"
-                              else "N(0,1) (torch, on device)") + ", rounded to bf16"},
+                              else "N(0,1) (torch, on device)") + f", rounded to {w.dtype}"},
         "select_ms": sel_ms, "attend_ms": att_ms,
         "attend_tflops_exact": att_tflops,
         "attend_tflops_nominal": nominal_flops(w) / (att_ms * 1e-3) / 1e12,
@@ -362,7 +362,7 @@ def run_ours(args, w, rank, world, device):
                      "peak": tensor_peak, "unit": "TFLOP/s", "frac": att_tflops / tensor_peak,
                      "peak_source": f"{src} {peak_kind}",
                      "traffic": recorded_traffic("attn_fwd_kernel", w.name)},
-        "select_roofline": {"kernels": "pool_kernel + score_topk_kernel", "bound": "hbm", "achieved": sel_gbs,
+        "select_roofline": {"kernels": "pool_kernel + " + ("score_topk_kernel" if 256 < nT <= 768 else "score_topk_narrow_kernel"), "bound": "hbm", "achieved": sel_gbs,
                             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": sel_gbs / peaks["hbm_gbs"],
                             "peak_source": f"{src} hbm_gbs",
                             "traffic": recorded_traffic("pool_kernel", w.name)},

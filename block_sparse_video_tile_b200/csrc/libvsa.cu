@@ -78,19 +78,25 @@ static unsigned int* device_error_ptr() {
   return static_cast<unsigned int*>(p);
 }
 
-// Score + top-k grid: 8 query tiles per CTA up to 256 tiles per head, else
-// 16 (more reuse of each staged key-mean chunk).
-template <int D, int R>
-static int launch_score(const Geom& g, int topk, int32_t* idx, const float* ws, cudaStream_t st) {
-  const size_t smem = score_smem_bytes<D, R>(g);
-  if (cudaFuncSetAttribute(score_topk_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
+// Score + top-k grid, launched as a programmatic dependent of the pooling
+// grid: its CTAs may start while pooling drains; griddepcontrol.wait holds
+// them until the pooled means are complete.  Heads of kNarrowMaxTiles + 1 ..
+// kWideMaxTiles tiles take the wide kernel (32 query tiles per CTA); smaller
+// heads (little score work, more CTAs) and larger ones (key rows that would
+// not fit beside the wide ring) take the narrow kernel (16).
+template <int D>
+static int launch_score(const Geom& g, int topk, int32_t* idx, const float* means, unsigned int* err,
+                        cudaStream_t st) {
+  const bool wide = g.nT > kNarrowMaxTiles && g.nT <= kWideMaxTiles;
+  const size_t smem = wide ? score_smem_bytes<D>(g) : score_narrow_smem_bytes<D>(g);
+  const void* fn = wide ? reinterpret_cast<const void*>(score_topk_kernel<D>)
+                        : reinterpret_cast<const void*>(score_topk_narrow_kernel<D>);
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
     return VSA_ERR_CUDA;
-  // programmatic dependent launch: the grid may start while pooling drains;
-  // its griddepcontrol.wait holds it until the pooled means are complete
+  const int rows = wide ? kWideRows : kNarrowRows;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(ceil_div(g.nT, R), g.B * g.H);
-  cfg.blockDim = dim3(kScoreThreads);
+  cfg.gridDim = dim3(ceil_div(g.nT, rows), g.B * g.H);
+  cfg.blockDim = dim3(wide ? kWideThreads : kNarrowThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -98,12 +104,13 @@ static int launch_score(const Geom& g, int topk, int32_t* idx, const float* ws, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, score_topk_kernel<D, R>, g, ws, topk, idx) == cudaSuccess ? VSA_OK
-                                                                                               : VSA_ERR_CUDA;
+  const cudaError_t e = wide ? cudaLaunchKernelEx(&cfg, score_topk_kernel<D>, g, means, topk, idx)
+                             : cudaLaunchKernelEx(&cfg, score_topk_narrow_kernel<D>, g, means, topk, idx);
+  return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 
 template <int D, bool F16>
-static int launch_select(const Geom& g, const void* q, const void* k, int topk, int32_t* idx, float* ws,
+static int launch_select(const Geom& g, const void* q, const void* k, int topk, int32_t* idx, void* ws,
                          cudaStream_t st) {
   CUtensorMap mq, mk;
   int rc;
@@ -111,13 +118,14 @@ static int launch_select(const Geom& g, const void* q, const void* k, int topk, 
     return rc;
   unsigned int* err = device_error_ptr();
   if (err == nullptr) return VSA_ERR_CUDA;
+  float* means = static_cast<float*>(ws);
   const size_t psmem = pool_smem_bytes<D>(g);
   if (cudaFuncSetAttribute(pool_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(psmem)) != cudaSuccess)
     return VSA_ERR_CUDA;
-  pool_kernel<D, F16><<<dim3(g.nT, g.B * g.H, 2), kPoolThreads, psmem, st>>>(mq, mk, g, ws, err);
+  pool_kernel<D, F16><<<dim3(g.nT, g.B * g.H, 2), kPoolThreads, psmem, st>>>(mq, mk, g, means, err);
   if (cudaGetLastError() != cudaSuccess) return VSA_ERR_CUDA;
-  return g.nT <= 256 ? launch_score<D, 8>(g, topk, idx, ws, st) : launch_score<D, 16>(g, topk, idx, ws, st);
+  return launch_score<D>(g, topk, idx, means, err, st);
 }
 
 template <int D, int MODE, bool F16>
@@ -171,7 +179,7 @@ static int dispatch_attn(int d, int mode, const CUtensorMap& mq, const CUtensorM
   return launch_attn<64, MODE_PAIR, F16>(mq, mk, mv, a, st);
 }
 
-static int dispatch_select(const Geom& g, const void* q, const void* k, int topk, int32_t* idx, float* ws,
+static int dispatch_select(const Geom& g, const void* q, const void* k, int topk, int32_t* idx, void* ws,
                            cudaStream_t st) {
   if (g.d == 128) return g.f16 ? launch_select<128, true>(g, q, k, topk, idx, ws, st)
                                : launch_select<128, false>(g, q, k, topk, idx, ws, st);
@@ -202,7 +210,7 @@ int vsa_tile_count(const vsa_shape* shape, int32_t* num_tiles, int32_t* tiles_pe
 size_t vsa_select_workspace_bytes(const vsa_shape* shape) {
   Geom g;
   if (make_geom(shape, &g) != VSA_OK) return 0;
-  return sizeof(float) * 2ull * g.B * g.H * g.nT * g.d;
+  return select_workspace_bytes(g);
 }
 
 int vsa_select(const vsa_shape* shape, const void* q, const void* k, int32_t topk, int32_t* idx_out,
@@ -217,8 +225,7 @@ int vsa_select(const vsa_shape* shape, const void* q, const void* k, int32_t top
   if (workspace == nullptr || workspace_bytes < vsa_select_workspace_bytes(shape)) return VSA_ERR_WORKSPACE;
   if ((rc = check_arch()) != VSA_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float* ws = static_cast<float*>(workspace);
-  return dispatch_select(g, q, k, topk, idx_out, ws, st);
+  return dispatch_select(g, q, k, topk, idx_out, workspace, st);
 }
 
 int vsa_select_noalloc(const vsa_shape* shape, const void* q, const void* k, int32_t topk, int32_t* idx_out,

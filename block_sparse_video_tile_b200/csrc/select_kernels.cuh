@@ -7,11 +7,16 @@
 // shared memory instead of round-tripping a score matrix through HBM.
 //
 // Two kernels:
-//   pool_kernel   HBM-bound: reads every Q and K byte once, writes the per-tile
-//                 means (float32 [2, B*H, nT, d]) to the caller's workspace.
-//   score_topk_kernel: per (head, block of query tiles) computes the score
-//                 rows into shared memory (float32 FMA in a fixed order) and
-//                 selects each row's top-k exactly; writes ascending idx.
+//   pool_kernel        HBM-bound: reads every Q and K byte once and writes the
+//                      per-tile float32 means, transposed, to the caller's
+//                      workspace: [2, B*H, d, ldT] (Q, then K), ldT = nT
+//                      rounded up to 4.
+//   score_topk_kernel  per (head, block of R query tiles): the R x nT score
+//                      rows in shared memory (float32 FMA, channels summed in
+//                      ascending order) and each row's exact top-k; writes
+//                      ascending idx.  Launched as a programmatic dependent of
+//                      the pooling grid, so its launch overlaps the pooling
+//                      tail; it waits for the pooled means before reading them.
 #pragma once
 
 #include <cstdint>
@@ -26,6 +31,112 @@ namespace vsa {
 
 constexpr int kPoolThreads = 256;
 
+// Row stride (floats) of the transposed tile means.
+__host__ __device__ inline int means_ld(int nT) { return (nT + 3) & ~3; }
+
+inline size_t select_workspace_bytes(const Geom& g) {
+  return sizeof(float) * 2ull * g.B * g.H * g.d * means_ld(g.nT);
+}
+
+// Larger float -> larger unsigned key (total order; -0 < +0, scores are
+// canonicalised so -0 does not occur).
+__device__ __forceinline__ uint32_t order_key(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Exact top-k of NR rows of order keys by one warp, keys held in registers
+// (lane l holds tiles l, l + 32, ...).  The topk-th largest key T of a row is
+// found bit by bit from the top: T keeps a bit when at least topk keys are
+// >= T with that bit set (a warp-wide count per bit, no shared-memory
+// atomics).  Bits on which all keys of the row agree are decided without
+// counting, and the search stops once exactly topk keys are >= T.  The rows
+// advance together, so their warp reductions overlap.  Every key above T is
+// taken, then the keys equal to T in ascending tile order until topk are
+// taken (ties go to the lower tile index); indices are written in ascending
+// order.  Order keys of finite scores are never 0, so 0 marks padding slots.
+// Rows r < nrow are kr + r * kst, written to out + r * topk.
+template <int MAXE, int NR>
+__device__ __forceinline__ void bsearch_topk_rows(const uint32_t* kr, int kst, int nrow, int nT, int topk,
+                                                  int32_t* out) {
+  const int lane = threadIdx.x % 32;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  uint32_t key[NR][MAXE];
+  uint32_t T[NR];
+  int bit[NR];
+#pragma unroll
+  for (int r = 0; r < NR; ++r) {
+    uint32_t kand = 0xffffffffu, kor = 0u;
+#pragma unroll
+    for (int e = 0; e < MAXE; ++e) {
+      const int j = lane + 32 * e;
+      key[r][e] = (r < nrow && j < nT) ? kr[r * kst + j] : 0u;
+      if (j < nT) {
+        kand &= key[r][e];
+        kor |= key[r][e];
+      }
+    }
+    kand = __reduce_and_sync(0xffffffffu, kand);
+    kor = __reduce_or_sync(0xffffffffu, kor);
+    const int common = __clz(kand ^ kor);        // leading bits shared by all keys (32: all equal)
+    T[r] = common == 0 ? 0u : (kand & (0xffffffffu << (32 - common)));
+    bit[r] = r < nrow ? 31 - common : -1;        // next bit to decide; -1: done
+  }
+  for (;;) {
+    bool any = false;
+    uint32_t c[NR];
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      c[r] = 0;
+      if (bit[r] >= 0) {
+        any = true;
+        const uint32_t cand = T[r] | (1u << bit[r]);
+        uint32_t p[4] = {0u, 0u, 0u, 0u};   // four independent chains of adds
+#pragma unroll
+        for (int e = 0; e < MAXE; ++e) p[e & 3] += (key[r][e] >= cand) ? 1u : 0u;
+        c[r] = (p[0] + p[1]) + (p[2] + p[3]);
+      }
+    }
+    if (!any) break;
+#pragma unroll
+    for (int r = 0; r < NR; ++r) c[r] = __reduce_add_sync(0xffffffffu, c[r]);
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      if (bit[r] < 0) continue;
+      const uint32_t cand = T[r] | (1u << bit[r]);
+      --bit[r];
+      if (c[r] >= static_cast<uint32_t>(topk)) {
+        T[r] = cand;
+        // exactly topk keys are >= T: they are the answer whatever the lower bits
+        if (c[r] == static_cast<uint32_t>(topk)) bit[r] = -1;
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < NR; ++r) {
+    if (r >= nrow) break;
+    uint32_t gt = 0;
+#pragma unroll
+    for (int e = 0; e < MAXE; ++e) gt += (key[r][e] > T[r]) ? 1u : 0u;
+    gt = __reduce_add_sync(0xffffffffu, gt);
+    const int want_eq = topk - static_cast<int>(gt);
+    int base = 0, eq_seen = 0;
+    int32_t* o = out + static_cast<size_t>(r) * topk;
+#pragma unroll
+    for (int e = 0; e < MAXE; ++e) {
+      if (32 * e >= nT) break;
+      const bool gtb = key[r][e] > T[r];
+      const bool eqb = key[r][e] == T[r];
+      const uint32_t eqm = __ballot_sync(0xffffffffu, eqb);
+      const bool take = gtb || (eqb && eq_seen + __popc(eqm & lt_mask) < want_eq);
+      const uint32_t tm = __ballot_sync(0xffffffffu, take);
+      if (take) o[base + __popc(tm & lt_mask)] = lane + 32 * e;
+      base += __popc(tm);
+      eq_seen += __popc(eqm);
+    }
+  }
+}
+
 // One CTA per (tile j, head bh, tensor z in {Q, K}).  The whole tile is one
 // 5-D TMA box per 64-channel slab (the same [B*H, T, Hh, W, d] view the
 // attend kernel uses), so a 256-token tile of d = 128 puts 64 KB in flight
@@ -36,7 +147,7 @@ constexpr int kPoolThreads = 256;
 template <int D, bool F16>
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                             const __grid_constant__ CUtensorMap tmK, Geom g,
-                                                            float* __restrict__ pooled, unsigned int* err) {
+                                                            float* __restrict__ means, unsigned int* err) {
   constexpr int kSlabs = D / 64;
   constexpr int TPR = D / 8;                 // threads per row (one 16-byte chunk each)
   constexpr int RP = kPoolThreads / TPR;     // row groups
@@ -91,11 +202,13 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __grid_constan
   int vt, vy, vx;
   tile_extent(g, c, vt, vy, vx);
   const float cnt = static_cast<float>(vt * vy * vx);
+  const int ld = means_ld(g.nT);
+  float* mz = means + (static_cast<size_t>(z) * g.B * g.H + bh) * D * ld;
   for (int col = threadIdx.x; col < D; col += kPoolThreads) {
     float sum = 0.f;
 #pragma unroll 8
     for (int i = 0; i < RP; ++i) sum += part[i * D + col];
-    pooled[((static_cast<size_t>(z) * g.B * g.H + bh) * g.nT + j) * D + col] = sum / cnt;
+    mz[static_cast<size_t>(col) * ld + j] = sum / cnt;
   }
 }
 
@@ -104,162 +217,267 @@ inline size_t pool_smem_bytes(const Geom& g) {
   return static_cast<size_t>(D / 64) * g.vol * 128 + (kPoolThreads / (D / 8)) * D * 4 + 16 + 1024;
 }
 
-constexpr int kScoreThreads = 256;  // 8 warps
+// ------------------------------------------------------------ score + top-k
+// Shared-memory traffic bounds the score phase: a 16-byte shared load is
+// served one 8-lane quarter-warp at a time, so each costs at least four
+// shared-memory cycles even when lanes read the same address.  A thread block
+// of m x n scores per thread needs (m + n) such cycles per warp and channel
+// for 32 m n FMAs, and the SM retires 128 FMAs per shared-memory cycle: the
+// 8 x 8 block of the wide kernel balances the two (4 x 4 would run at half
+// the FMA rate).
 
-// Larger float -> larger unsigned key (total order; -0 < +0, scores are
-// canonicalised so -0 does not occur).
-__device__ __forceinline__ uint32_t order_key(float f) {
-  const uint32_t b = __float_as_uint(f);
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-
-// Exact top-k of one row of order keys by one warp, keys held in registers
-// (lane l holds tiles l, l + 32, ...).  The topk-th largest key T is found
-// bit by bit from the top: T keeps a bit when at least topk keys are >= T
-// with that bit set (a warp-wide count per bit, no shared-memory atomics).
-// Every key above T is taken, then the keys equal to T in ascending tile
-// order until topk are taken (ties go to the lower tile index); indices are
-// written in ascending order.  Order keys of finite scores are never 0, so 0
-// marks the padding slots.
-template <int MAXE>
-__device__ __forceinline__ void bsearch_topk_row(const uint32_t* kr, int nT, int topk, int32_t* out) {
-  const int lane = threadIdx.x % 32;
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  uint32_t key[MAXE];
-#pragma unroll
-  for (int e = 0; e < MAXE; ++e) {
-    const int j = lane + 32 * e;
-    key[e] = (j < nT) ? kr[j] : 0u;
-  }
-  uint32_t T = 0;
-  for (int b = 31; b >= 0; --b) {
-    const uint32_t cand = T | (1u << b);
-    uint32_t c = 0;
-#pragma unroll
-    for (int e = 0; e < MAXE; ++e) c += (key[e] >= cand) ? 1u : 0u;
-    c = __reduce_add_sync(0xffffffffu, c);
-    if (c >= static_cast<uint32_t>(topk)) T = cand;
-  }
-  uint32_t gt = 0;
-#pragma unroll
-  for (int e = 0; e < MAXE; ++e) gt += (key[e] > T) ? 1u : 0u;
-  gt = __reduce_add_sync(0xffffffffu, gt);
-  const int want_eq = topk - static_cast<int>(gt);
-  int base = 0, eq_seen = 0;
-#pragma unroll
-  for (int e = 0; e < MAXE; ++e) {
-    if (32 * e >= nT) break;
-    const bool gtb = key[e] > T;
-    const bool eqb = key[e] == T;
-    const uint32_t eqm = __ballot_sync(0xffffffffu, eqb);
-    const bool take = gtb || (eqb && eq_seen + __popc(eqm & lt_mask) < want_eq);
-    const uint32_t tm = __ballot_sync(0xffffffffu, take);
-    if (take) out[base + __popc(tm & lt_mask)] = lane + 32 * e;
-    base += __popc(tm);
-    eq_seen += __popc(eqm);
+// One warp per row picks each row's top-k from the order keys in shared memory.
+__device__ __forceinline__ void topk_rows(const uint32_t* keys, int kst, int nT, int nrows, int topk,
+                                          int32_t* out_rows, int warps) {
+  const int warp = threadIdx.x / 32;
+  for (int r = warp; r < nrows; r += warps) {
+    const uint32_t* kr = keys + r * kst;
+    int32_t* out = out_rows + static_cast<size_t>(r) * topk;
+    if (nT <= 32 * 8)
+      bsearch_topk_rows<8, 1>(kr, kst, 1, nT, topk, out);
+    else if (nT <= 32 * 12)
+      bsearch_topk_rows<12, 1>(kr, kst, 1, nT, topk, out);
+    else if (nT <= 32 * 16)
+      bsearch_topk_rows<16, 1>(kr, kst, 1, nT, topk, out);
+    else if (nT <= 32 * 24)
+      bsearch_topk_rows<24, 1>(kr, kst, 1, nT, topk, out);
+    else
+      bsearch_topk_rows<48, 1>(kr, kst, 1, nT, topk, out);
   }
 }
 
-// Tile scores and top-k.  One CTA takes R query tiles of one head (R = 8 when
-// the head has at most 256 tiles, else 16).  Their pooled Q means and the
-// pooled K means, in chunks of up to 64 key tiles (rows padded to d + 4
-// floats), are copied to shared memory with vector loads.  Thread t =
-// (quarter, j) forms, for key tile j of the chunk and all R query tiles, the
-// partial dot product over its quarter of the d channels: the padded rows make
-// the key reads of a quarter-warp hit 8 different bank groups, and the query
-// reads are warp-wide broadcasts.  The four partial sums are added in a fixed
-// order (deterministic); the score rows stay in shared memory as order keys,
-// and one warp per row selects its top-k.  Shared memory stays under 76 KB
-// for up to 256 tiles, so three CTAs fit on an SM.
-// Dynamic shared memory: qb[R][D] | kb[min(nT,64)][D+4] | part[4][R][64] | keys[R][nT]
-constexpr int kScoreChunk = 64;
-constexpr int kScoreSplit = kScoreThreads / kScoreChunk;   // d split in 4 parts
+// Wide kernel (heads of kNarrowMaxTiles + 1 .. kWideMaxTiles tiles): one CTA per (block of 32
+// query tiles, head), 8 warps.  Per pass of 512 key tiles, warp w takes key
+// tiles 64w .. 64w + 63 of the pass against all 32 query tiles; lane
+// (qg = lane / 8, kg = lane % 8) holds the 8 x 8 block of query tiles
+// {4qg .. 4qg+3, 16+4qg .. 16+4qg+3} x key tiles {4kg .. 4kg+3, 32+4kg ..
+// 32+4kg+3} of the warp's 64, so each 16-byte load of a quarter-warp covers
+// 128 contiguous bytes (no bank conflicts).  Key means stream through shared
+// memory in slices of 16 channels x 512 key tiles on a 3-deep cp.async ring
+// (one barrier per slice).  Warps whose key tiles lie past nT skip the math.
+// Each score adds its channels in ascending order (deterministic); scores
+// become order keys in shared memory, never written to HBM.
+// Dynamic shared memory: qT [D][32] | ring [3][16][512] | keys [32][nT].
+constexpr int kWideRows = 32;
+constexpr int kWideKeys = 512;
+constexpr int kWideSlice = 16;
+constexpr int kWideStages = 3;
+constexpr int kWideThreads = 256;
+constexpr int kWideMaxTiles = 768;
+constexpr int kNarrowMaxTiles = 256;   // below this the narrow kernel is used too (more, shorter CTAs)
 
-template <int D, int R>
-__global__ void __launch_bounds__(kScoreThreads) score_topk_kernel(Geom g, const float* __restrict__ pooled,
-                                                                   int topk, int32_t* __restrict__ idx) {
-  constexpr int KS = D + 4;                 // padded key-mean row (floats)
-  constexpr int C4 = D / 4;
-  constexpr int PART4 = D / 4 / kScoreSplit;  // float4 chunks per part of a row
-  constexpr int MAXE = (R == 8) ? 8 : 48;   // keys per lane in the top-k (nT <= 256 / <= 1536)
+template <int D>
+__global__ void __launch_bounds__(kWideThreads) score_topk_kernel(Geom g, const float* __restrict__ means, int topk,
+                                                                  int32_t* __restrict__ idx) {
+  constexpr int SPP = D / kWideSlice;      // stages per pass
+  constexpr int SLICE = kWideSlice * kWideKeys;
+  constexpr int R = kWideRows;
   // the pooled means are written by the previous grid: wait for it
   asm volatile("griddepcontrol.wait;" ::: "memory");
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int nT = g.nT;
-  const int chunk = min(nT, kScoreChunk);
-  float* qb = reinterpret_cast<float*>(smem_raw);
-  float* kb = qb + R * D;
-  float* part = kb + chunk * KS;
-  uint32_t* keys = reinterpret_cast<uint32_t*>(part + kScoreSplit * R * kScoreChunk);
-
+  float* qT = reinterpret_cast<float*>(smem_raw);
+  float* ring = qT + D * R;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(ring + kWideStages * SLICE);
+  const int nT = g.nT, ld = means_ld(nT);
   const int bh = blockIdx.y;
   const int row0 = blockIdx.x * R;
   const int nrows = min(R, nT - row0);
   const size_t BH = static_cast<size_t>(g.B) * g.H;
-  const float4* qp = reinterpret_cast<const float4*>(pooled + (static_cast<size_t>(bh) * nT + row0) * D);
-  const float4* kp = reinterpret_cast<const float4*>(pooled + ((BH + bh) * nT) * D);
+  const float* mq = means + static_cast<size_t>(bh) * D * ld;
+  const float* mk = means + (BH + bh) * D * ld;
+  const int nstage = ceil_div(nT, kWideKeys) * SPP;
 
+  // query means (joined to the first cp.async group); float4s past the row are zero
+  for (int f = threadIdx.x; f < D * R / 4; f += kWideThreads) {
+    const int c = f / (R / 4), r4 = f % (R / 4);
+    const int row = row0 + 4 * r4;
+    const bool in = row < ld;
+    cp_async16(smem_u32(qT + c * R + 4 * r4),
+               in ? static_cast<const void*>(mq + static_cast<size_t>(c) * ld + row) : static_cast<const void*>(mq),
+               in ? 16u : 0u);
+  }
+  // stage st = (pass st / SPP, channel slice st % SPP) -> ring slot st % 3; one group per call
+  auto issue = [&](int st) {
+    if (st < nstage) {
+      const int kc0 = (st / SPP) * kWideKeys, c0 = (st % SPP) * kWideSlice;
+      float* dst = ring + (st % kWideStages) * SLICE;
 #pragma unroll 4
-  for (int e = threadIdx.x; e < R * C4; e += kScoreThreads)
-    reinterpret_cast<float4*>(qb)[e] = (e / C4 < nrows) ? __ldg(qp + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-
-  const int j = threadIdx.x % kScoreChunk;
-  const int quarter = threadIdx.x / kScoreChunk;
-  for (int c0 = 0; c0 < nT; c0 += kScoreChunk) {
-    const int ncol = min(kScoreChunk, nT - c0);
-    if (c0 > 0) __syncthreads();   // the previous chunk's partial sums are consumed
-#pragma unroll 8
-    for (int e = threadIdx.x; e < ncol * C4; e += kScoreThreads) {
-      const int r = e / C4, c = e % C4;
-      *reinterpret_cast<float4*>(kb + r * KS + 4 * c) = __ldg(kp + static_cast<size_t>(c0) * C4 + e);
+      for (int f = threadIdx.x; f < SLICE / 4; f += kWideThreads) {
+        const int c = f / (kWideKeys / 4), k4 = f % (kWideKeys / 4);
+        const int key = kc0 + 4 * k4;
+        const bool in = key < ld;
+        cp_async16(smem_u32(dst + c * kWideKeys + 4 * k4),
+                   in ? static_cast<const void*>(mk + static_cast<size_t>(c0 + c) * ld + key)
+                      : static_cast<const void*>(mk),
+                   in ? 16u : 0u);
+      }
     }
-    __syncthreads();
-    if (j < ncol) {
-      float acc[R];
+    cp_async_commit();
+  };
 #pragma unroll
-      for (int r = 0; r < R; ++r) acc[r] = 0.f;
-      const float4* krow = reinterpret_cast<const float4*>(kb + j * KS) + quarter * PART4;
-      const float4* qrow = reinterpret_cast<const float4*>(qb) + quarter * PART4;
-#pragma unroll 4
-      for (int i = 0; i < PART4; ++i) {
-        const float4 kv = krow[i];
+  for (int st = 0; st < kWideStages - 1; ++st) issue(st);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int qg = lane / 8, kg = lane % 8;
+  float acc[8][8];
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const float4 qv = qrow[r * C4 + i];
-          acc[r] = fmaf(qv.x, kv.x, acc[r]);
-          acc[r] = fmaf(qv.y, kv.y, acc[r]);
-          acc[r] = fmaf(qv.z, kv.z, acc[r]);
-          acc[r] = fmaf(qv.w, kv.w, acc[r]);
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+
+  for (int st = 0; st < nstage; ++st) {
+    cp_async_wait<kWideStages - 2>();
+    __syncthreads();                 // slice st visible; slot of slice st-1 free
+    issue(st + kWideStages - 1);
+    const int sl = st % SPP;
+    const int kw0 = (st / SPP) * kWideKeys + 64 * warp;   // the warp's first key tile
+    if (kw0 < nT) {
+      const float* kb = ring + (st % kWideStages) * SLICE + 64 * warp + 4 * kg;
+      const float* qb = qT + sl * kWideSlice * R + 4 * qg;
+#pragma unroll
+      for (int c = 0; c < kWideSlice; ++c) {
+        const float4 q0 = *reinterpret_cast<const float4*>(qb + c * R);
+        const float4 q1 = *reinterpret_cast<const float4*>(qb + c * R + 16);
+        const float4 k0 = *reinterpret_cast<const float4*>(kb + c * kWideKeys);
+        const float4 k1 = *reinterpret_cast<const float4*>(kb + c * kWideKeys + 32);
+        const float qa[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+        const float ka[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(qa[i], ka[j], acc[i][j]);
+      }
+    }
+    if (sl == SPP - 1) {             // end of a pass: scores -> order keys
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int row = (i < 4 ? 0 : 16) + 4 * qg + (i & 3);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int key = kw0 + (j < 4 ? 0 : 32) + 4 * kg + (j & 3);
+          if (row < nrows && key < nT) keys[row * nT + key] = order_key(acc[i][j] + 0.f);
+          acc[i][j] = 0.f;
         }
       }
-#pragma unroll
-      for (int r = 0; r < R; ++r) part[(quarter * R + r) * kScoreChunk + j] = acc[r];
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < R * ncol; e += kScoreThreads) {
-      const int r = e / ncol, c = e % ncol;
-      const float sc = (part[r * kScoreChunk + c] + part[(R + r) * kScoreChunk + c]) +
-                       (part[(2 * R + r) * kScoreChunk + c] + part[(3 * R + r) * kScoreChunk + c]);
-      keys[r * nT + c0 + c] = order_key(sc + 0.f);
     }
   }
+  cp_async_wait<0>();
   __syncthreads();
-
-  const int warp = threadIdx.x / 32;
-  for (int r = warp; r < nrows; r += kScoreThreads / 32) {
-    int32_t* out = idx + (static_cast<size_t>(bh) * nT + row0 + r) * topk;
-    if (MAXE > 24 && nT <= 32 * 24)   // fewer keys per lane: a shorter unrolled count loop
-      bsearch_topk_row<(MAXE > 24 ? 24 : MAXE)>(keys + r * nT, nT, topk, out);
-    else
-      bsearch_topk_row<MAXE>(keys + r * nT, nT, topk, out);
-  }
+  topk_rows(keys, nT, nT, nrows, topk, idx + (static_cast<size_t>(bh) * nT + row0) * topk, kWideThreads / 32);
 }
 
-template <int D, int R>
+template <int D>
 inline size_t score_smem_bytes(const Geom& g) {
-  const size_t chunk = static_cast<size_t>(min(g.nT, kScoreChunk));
-  return sizeof(float) * (static_cast<size_t>(R) * D + chunk * (D + 4) + kScoreSplit * static_cast<size_t>(R) * kScoreChunk) +
-         sizeof(uint32_t) * (static_cast<size_t>(R) * g.nT);
+  return sizeof(float) * (static_cast<size_t>(D) * kWideRows + kWideStages * kWideSlice * kWideKeys) +
+         sizeof(uint32_t) * static_cast<size_t>(kWideRows) * g.nT;
+}
+
+// Narrow kernel (heads of at most kNarrowMaxTiles tiles, and of more than
+// kWideMaxTiles, whose 32 key rows would not fit beside the wide ring): one
+// CTA per (block of 16 query tiles,
+// head), 8 warps; lane (qg, kg) of warp w holds the 4 x 4 block of query
+// tiles 4qg .. 4qg+3 x key tiles 32w + 4kg .. 32w + 4kg + 3 of a pass of 256
+// key tiles.  Key means stream in slices of 16 channels x 256 key tiles on a
+// 4-deep cp.async ring.  Same summation order and selection as the wide kernel.
+// Dynamic shared memory: qT [D][16] | ring [4][16][256] | keys [16][nT].
+constexpr int kNarrowRows = 16;
+constexpr int kNarrowKeys = 256;
+constexpr int kNarrowSlice = 16;
+constexpr int kNarrowStages = 4;
+constexpr int kNarrowThreads = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kNarrowThreads) score_topk_narrow_kernel(Geom g, const float* __restrict__ means,
+                                                                           int topk, int32_t* __restrict__ idx) {
+  constexpr int SPP = D / kNarrowSlice;
+  constexpr int SLICE = kNarrowSlice * kNarrowKeys;
+  constexpr int R = kNarrowRows;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float* qT = reinterpret_cast<float*>(smem_raw);
+  float* ring = qT + D * R;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(ring + kNarrowStages * SLICE);
+  const int nT = g.nT, ld = means_ld(nT);
+  const int bh = blockIdx.y;
+  const int row0 = blockIdx.x * R;
+  const int nrows = min(R, nT - row0);
+  const size_t BH = static_cast<size_t>(g.B) * g.H;
+  const float* mq = means + static_cast<size_t>(bh) * D * ld;
+  const float* mk = means + (BH + bh) * D * ld;
+  const int nstage = ceil_div(nT, kNarrowKeys) * SPP;
+
+  for (int f = threadIdx.x; f < D * R / 4; f += kNarrowThreads) {
+    const int c = f / (R / 4), r4 = f % (R / 4);
+    const int row = row0 + 4 * r4;
+    const bool in = row < ld;
+    cp_async16(smem_u32(qT + c * R + 4 * r4),
+               in ? static_cast<const void*>(mq + static_cast<size_t>(c) * ld + row) : static_cast<const void*>(mq),
+               in ? 16u : 0u);
+  }
+  auto issue = [&](int st) {
+    if (st < nstage) {
+      const int kc0 = (st / SPP) * kNarrowKeys, c0 = (st % SPP) * kNarrowSlice;
+      float* dst = ring + (st % kNarrowStages) * SLICE;
+      for (int f = threadIdx.x; f < SLICE / 4; f += kNarrowThreads) {
+        const int c = f / (kNarrowKeys / 4), k4 = f % (kNarrowKeys / 4);
+        const int key = kc0 + 4 * k4;
+        const bool in = key < ld;
+        cp_async16(smem_u32(dst + c * kNarrowKeys + 4 * k4),
+                   in ? static_cast<const void*>(mk + static_cast<size_t>(c0 + c) * ld + key)
+                      : static_cast<const void*>(mk),
+                   in ? 16u : 0u);
+      }
+    }
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int st = 0; st < kNarrowStages - 1; ++st) issue(st);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int qg = lane / 8, kg = lane % 8;
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  for (int st = 0; st < nstage; ++st) {
+    cp_async_wait<kNarrowStages - 2>();
+    __syncthreads();
+    issue(st + kNarrowStages - 1);
+    const int sl = st % SPP;
+    const float* kb = ring + (st % kNarrowStages) * SLICE + 32 * warp + 4 * kg;
+    const float* qb = qT + sl * kNarrowSlice * R + 4 * qg;
+#pragma unroll
+    for (int c = 0; c < kNarrowSlice; ++c) {
+      const float4 qv = *reinterpret_cast<const float4*>(qb + c * R);
+      const float4 kv = *reinterpret_cast<const float4*>(kb + c * kNarrowKeys);
+      const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
+      const float ka[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(qa[i], ka[j], acc[i][j]);
+    }
+    if (sl == SPP - 1) {
+      const int kc0 = (st / SPP) * kNarrowKeys + 32 * warp + 4 * kg;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (4 * qg + i < nrows && kc0 + j < nT) keys[(4 * qg + i) * nT + kc0 + j] = order_key(acc[i][j] + 0.f);
+          acc[i][j] = 0.f;
+        }
+    }
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  topk_rows(keys, nT, nT, nrows, topk, idx + (static_cast<size_t>(bh) * nT + row0) * topk, kNarrowThreads / 32);
+}
+
+template <int D>
+inline size_t score_narrow_smem_bytes(const Geom& g) {
+  return sizeof(float) * (static_cast<size_t>(D) * kNarrowRows + kNarrowStages * kNarrowSlice * kNarrowKeys) +
+         sizeof(uint32_t) * static_cast<size_t>(kNarrowRows) * g.nT;
 }
 
 }  // namespace vsa

@@ -86,8 +86,10 @@ typedef enum vsa_status {
  * Host only; touches no device. */
 int vsa_tile_count(const vsa_shape* shape, int32_t* num_tiles, int32_t* tiles_per_axis);
 
-/* Bytes of device workspace vsa_select needs for `shape` (pooled Q and K tile
- * means, float32 [2, B, H, nT, d]).  Returns 0 for an invalid shape. */
+/* Bytes of device workspace vsa_select needs for `shape`: the pooled Q and K
+ * tile means, float32 [2, B, H, d, ldT] with ldT = nT rounded up to a
+ * multiple of 4 (channel-major, so the score kernel reads contiguous tile
+ * rows).  Returns 0 for an invalid shape. */
 size_t vsa_select_workspace_bytes(const vsa_shape* shape);
 
 /* Tile selection (FastVideo VSA guide intro and "Wan top-k behavior"; fastbsa
@@ -116,7 +118,8 @@ int vsa_select(const vsa_shape* shape, const void* q, const void* k, int32_t top
  * own pool, code running inside a region where allocation is forbidden, or a
  * plugin with no allocator handle.  This call itself allocates nothing (no
  * cudaMalloc, no cudaFree, no allocating library routine).
- *   - The scratch needs 2*B*H*nT*d*4 bytes; larger shapes are rejected with
+ *   - The scratch needs vsa_select_workspace_bytes(shape) bytes (about
+ *     2*B*H*nT*d*4); larger shapes are rejected with
  *     VSA_ERR_WORKSPACE before anything is launched.
  *   - The first call on a device (with that device current) looks up the
  *     scratch array's device address; make that first call before any CUDA

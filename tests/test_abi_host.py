@@ -48,7 +48,9 @@ def test_tile_count_matches_oracle(name):
     n, per = api.tile_count(w.grid, w.tile, w.d, w.B, w.H)
     assert n == vo.num_tiles(w.grid, w.tile)
     assert per == vo.tiles_per_axis(w.grid, w.tile)
-    assert api.select_workspace_bytes(w.B, w.H, w.grid, w.d, w.tile) == 4 * 2 * w.B * w.H * n * w.d
+    # transposed float32 tile means [2, B*H, d, nT rounded up to 4]
+    ldT = -(-n // 4) * 4
+    assert api.select_workspace_bytes(w.B, w.H, w.grid, w.d, w.tile) == 4 * 2 * w.B * w.H * w.d * ldT
 
 
 @pytest.mark.parametrize("kw,status", [

@@ -138,7 +138,7 @@ FULL = [WAN5B, WAN14B, LONGCAT, WAN5B.with_(name="wan5b_f16", dtype="f16")]
 
 def _sample_tiles(w, rng, n_heads=2, n_tiles=4):
     nT = vo.num_tiles(w.grid, w.tile)
-    heads = sorted(rng.choice(w.B * w.H, n_heads, replace=False).tolist())
+    heads = sorted(rng.choice(w.B * w.H, min(n_heads, w.B * w.H), replace=False).tolist())
     out = []
     for bh in heads:
         b, h = divmod(bh, w.H)
@@ -165,6 +165,22 @@ def _full_case(w, seed=0, topks=None):
 
 @pytest.mark.parametrize("w", FULL, ids=lambda w: w.name)
 def test_full_size(w):
+    rep = _full_case(w)
+    print(w.name, rep)
+
+
+# Heads of up to 768 tiles take the wide score kernel (768: its largest head),
+# larger ones the narrow kernel, up to the 1536-tile limit; ragged on every axis.
+MANY_TILES = [
+    Workload("tiles768", 1, 1, (15, 47, 63), 64, (4, 4, 4), 48, "field"),
+    Workload("tiles960", 1, 2, (19, 45, 62), 64, (4, 4, 4), 60, "field"),
+    Workload("tiles1536", 1, 1, (23, 61, 62), 64, (4, 4, 4), 96),
+]
+
+
+@pytest.mark.parametrize("w", MANY_TILES, ids=lambda w: w.name)
+def test_many_tiles(w):
+    assert vo.num_tiles(w.grid, w.tile) == int(w.name[5:])
     rep = _full_case(w)
     print(w.name, rep)
 
