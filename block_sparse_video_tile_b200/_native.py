@@ -19,16 +19,19 @@ STATUS = {
 }
 DEVERR = {0: "none", 1: "wait timeout", 2: "tile index out of range"}
 
-EXPORTS = ("vsa_tile_count", "vsa_select_workspace_bytes", "vsa_select", "vsa_select_noalloc",
-           "vsa_attn_fwd", "vsa_device_error", "vsa_status_string")
+EXPORTS = ("vsa_tile_count", "vsa_kv_tile_count", "vsa_topk_from_sparsity", "vsa_select_workspace_bytes",
+           "vsa_select", "vsa_select_noalloc", "vsa_attn_fwd", "vsa_device_error", "vsa_status_string")
 SELECT_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 DTYPE_BF16, DTYPE_F16 = 0, 1
+LAYOUT_BHND, LAYOUT_BNHD = 0, 1
 
 
 class VsaShape(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int32) for n in ("B", "H", "T", "Hh", "W", "d", "tt", "th", "tw", "dtype")]
+    """vsa_shape: zero key/value fields mean "the query grid / tile"."""
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "H", "T", "Hh", "W", "d", "tt", "th", "tw", "dtype", "layout",
+                                              "Tk", "Hk", "Wk", "tk", "hk", "wk")]
 
 
 class VsaError(RuntimeError):
@@ -52,6 +55,10 @@ def lib() -> ctypes.CDLL:
         P, S, I32, SZ = ctypes.c_void_p, ctypes.POINTER(VsaShape), ctypes.c_int32, ctypes.c_size_t
         L.vsa_tile_count.argtypes = [S, ctypes.POINTER(I32), ctypes.POINTER(I32)]
         L.vsa_tile_count.restype = ctypes.c_int
+        L.vsa_kv_tile_count.argtypes = [S, ctypes.POINTER(I32), ctypes.POINTER(I32)]
+        L.vsa_kv_tile_count.restype = ctypes.c_int
+        L.vsa_topk_from_sparsity.argtypes = [S, ctypes.c_float, ctypes.POINTER(I32)]
+        L.vsa_topk_from_sparsity.restype = ctypes.c_int
         L.vsa_select_workspace_bytes.argtypes = [S]
         L.vsa_select_workspace_bytes.restype = SZ
         L.vsa_select.argtypes = [S, P, P, I32, P, P, SZ, P]

@@ -1,9 +1,11 @@
 """Python entry points over the C ABI, taking torch tensors.
 
 PyTorch provides device memory and the current stream; the work is done by
-libvsa's kernels.  Layouts (see include/vsa.h): Q, K, V, O bfloat16 or float16
-[B, H, N, d] contiguous with raster token order over the latent grid (T, Hh, W);
-idx int32 [B, H, nT, topk]; LSE float32 [B, H, N].
+libvsa's kernels.  Layouts (see include/vsa.h): Q, K, V, O bfloat16 or float16,
+contiguous, either "bhnd" = [B, H, N, d] or "bnhd" = [B, N, H, d], with raster
+token order over the latent grid (T, Hh, W); idx int32 [B, H, nTq, topk];
+LSE float32 [B, H, Nq].  Keys and values may have their own grid and tile
+(grid_k, tile_k; by default the query's) with the same tile volume.
 """
 from __future__ import annotations
 
@@ -12,42 +14,81 @@ import math
 
 import torch
 
-from ._native import DTYPE_BF16, DTYPE_F16, VsaShape, check, lib
+from ._native import DTYPE_BF16, DTYPE_F16, LAYOUT_BHND, LAYOUT_BNHD, VsaShape, check, lib
 
-__all__ = ["make_shape", "tile_count", "select", "attn_fwd", "forward", "forward_host",
-           "device_error", "select_workspace_bytes"]
+__all__ = ["make_shape", "tile_count", "kv_tile_count", "topk_from_sparsity", "select", "attn_fwd", "forward",
+           "forward_host", "device_error", "select_workspace_bytes"]
 
 
 _DTYPES = {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_F16}
+_LAYOUTS = {"bhnd": LAYOUT_BHND, "bnhd": LAYOUT_BNHD}
 
 
-def make_shape(B: int, H: int, grid, d: int, tile, dtype=torch.bfloat16) -> VsaShape:
+def make_shape(B: int, H: int, grid, d: int, tile, dtype=torch.bfloat16, *, layout: str = "bhnd",
+               grid_k=None, tile_k=None) -> VsaShape:
     T, Hh, W = grid
     tt, th, tw = tile
-    return VsaShape(B, H, T, Hh, W, d, tt, th, tw, _DTYPES.get(dtype, -1))
+    Tk, Hk, Wk = grid_k if grid_k is not None else (0, 0, 0)
+    tk, hk, wk = tile_k if tile_k is not None else (0, 0, 0)
+    return VsaShape(B, H, T, Hh, W, d, tt, th, tw, _DTYPES.get(dtype, -1), _LAYOUTS.get(layout, -1),
+                    Tk, Hk, Wk, tk, hk, wk)
 
 
-def tile_count(grid, tile, d: int = 128, B: int = 1, H: int = 1):
-    """(num_tiles, (tiles along T, Hh, W)) -- host only."""
-    shp = make_shape(B, H, grid, d, tile)
+def _count(fn, shp):
     n = ctypes.c_int32()
     per = (ctypes.c_int32 * 3)()
-    check("vsa_tile_count", lib().vsa_tile_count(ctypes.byref(shp), ctypes.byref(n), per))
+    check(fn, getattr(lib(), fn)(ctypes.byref(shp), ctypes.byref(n), per))
     return n.value, (per[0], per[1], per[2])
 
 
-def select_workspace_bytes(B, H, grid, d, tile) -> int:
-    shp = make_shape(B, H, grid, d, tile)
+def tile_count(grid, tile, d: int = 128, B: int = 1, H: int = 1):
+    """(num query tiles, (tiles along T, Hh, W)) -- host only."""
+    return _count("vsa_tile_count", make_shape(B, H, grid, d, tile))
+
+
+def kv_tile_count(grid, tile, grid_k=None, tile_k=None, d: int = 128, B: int = 1, H: int = 1):
+    """(num key/value tiles, (tiles along T, Hh, W)) -- host only."""
+    return _count("vsa_kv_tile_count", make_shape(B, H, grid, d, tile, grid_k=grid_k, tile_k=tile_k))
+
+
+def topk_from_sparsity(grid, tile, sparsity: float, grid_k=None, tile_k=None, d: int = 128) -> int:
+    """Kept key/value tiles per query tile for a sparsity: round((1 - sparsity) * nTk), in [1, nTk]."""
+    shp = make_shape(1, 1, grid, d, tile, grid_k=grid_k, tile_k=tile_k)
+    k = ctypes.c_int32()
+    check("vsa_topk_from_sparsity", lib().vsa_topk_from_sparsity(ctypes.byref(shp), float(sparsity),
+                                                                  ctypes.byref(k)))
+    return k.value
+
+
+def select_workspace_bytes(B, H, grid, d, tile, grid_k=None, tile_k=None) -> int:
+    shp = make_shape(B, H, grid, d, tile, grid_k=grid_k, tile_k=tile_k)
     return int(lib().vsa_select_workspace_bytes(ctypes.byref(shp)))
 
 
-def _check_qkv(name, x, B, H, N, d, dtype=None):
+def _dims(x, layout):
+    """(B, H, N, d) of a tensor in the given layout."""
+    if x.dim() != 4:
+        raise ValueError(f"expected a 4-D tensor, got shape {tuple(x.shape)}")
+    if layout == "bhnd":
+        return tuple(x.shape)
+    if layout == "bnhd":
+        B, N, H, d = x.shape
+        return B, H, N, d
+    raise ValueError(f"layout must be 'bhnd' or 'bnhd', got {layout!r}")
+
+
+def _check_qkv(name, x, want, layout, dtype=None):
     if not (x.is_cuda and x.dtype in _DTYPES and x.is_contiguous()):
         raise ValueError(f"{name} must be a contiguous CUDA bfloat16 or float16 tensor")
     if dtype is not None and x.dtype != dtype:
         raise ValueError(f"{name} is {x.dtype}, expected {dtype} like q")
-    if tuple(x.shape) != (B, H, N, d):
-        raise ValueError(f"{name} has shape {tuple(x.shape)}, expected {(B, H, N, d)}")
+    got = _dims(x, layout)
+    if got != tuple(want):
+        raise ValueError(f"{name} has (B, H, N, d) = {got} in layout {layout}, expected {tuple(want)}")
+
+
+def _grid_tokens(grid) -> int:
+    return grid[0] * grid[1] * grid[2]
 
 
 def _stream(stream) -> int:
@@ -55,13 +96,14 @@ def _stream(stream) -> int:
     return s.cuda_stream
 
 
-def select(q: torch.Tensor, k: torch.Tensor, grid, tile, topk: int, *, out=None,
-           workspace=None, stream=None) -> torch.Tensor:
-    """Top-k key tiles per query tile: int32 [B, H, nT, topk], ascending."""
-    B, H, N, d = q.shape
-    _check_qkv("q", q, B, H, N, d)
-    _check_qkv("k", k, B, H, N, d, q.dtype)
-    shp = make_shape(B, H, grid, d, tile, q.dtype)
+def select(q: torch.Tensor, k: torch.Tensor, grid, tile, topk: int, *, grid_k=None, tile_k=None,
+           layout: str = "bhnd", out=None, workspace=None, stream=None) -> torch.Tensor:
+    """Top-k key tiles per query tile: int32 [B, H, nTq, topk], ascending."""
+    B, H, Nq, d = _dims(q, layout)
+    Nk = _grid_tokens(grid_k if grid_k is not None else grid)
+    _check_qkv("q", q, (B, H, _grid_tokens(grid), d), layout)
+    _check_qkv("k", k, (B, H, Nk, d), layout, q.dtype)
+    shp = make_shape(B, H, grid, d, tile, q.dtype, layout=layout, grid_k=grid_k, tile_k=tile_k)
     nT, _ = tile_count(grid, tile, d, B, H)
     if out is None:
         out = torch.empty((B, H, nT, topk), dtype=torch.int32, device=q.device)
@@ -74,22 +116,24 @@ def select(q: torch.Tensor, k: torch.Tensor, grid, tile, topk: int, *, out=None,
     return out
 
 
-def attn_fwd(q, k, v, idx, grid, tile, *, scale: float | None = None, out=None, lse=None,
-             stream=None):
-    """Block-sparse attention over the kept tiles: (O bf16 [B,H,N,d], LSE f32 [B,H,N])."""
-    B, H, N, d = q.shape
-    for name, x in (("q", q), ("k", k), ("v", v)):
-        _check_qkv(name, x, B, H, N, d, q.dtype)
+def attn_fwd(q, k, v, idx, grid, tile, *, grid_k=None, tile_k=None, layout: str = "bhnd",
+             scale: float | None = None, out=None, lse=None, stream=None):
+    """Block-sparse attention over the kept tiles: (O like q, LSE f32 [B, H, Nq])."""
+    B, H, Nq, d = _dims(q, layout)
+    Nk = _grid_tokens(grid_k if grid_k is not None else grid)
+    _check_qkv("q", q, (B, H, _grid_tokens(grid), d), layout)
+    for name, x in (("k", k), ("v", v)):
+        _check_qkv(name, x, (B, H, Nk, d), layout, q.dtype)
     if not (idx.is_cuda and idx.dtype == torch.int32 and idx.is_contiguous() and idx.dim() == 4):
-        raise ValueError("idx must be a contiguous CUDA int32 tensor [B, H, nT, topk]")
+        raise ValueError("idx must be a contiguous CUDA int32 tensor [B, H, nTq, topk]")
     topk = idx.shape[-1]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
-        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    shp = make_shape(B, H, grid, d, tile, q.dtype)
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    shp = make_shape(B, H, grid, d, tile, q.dtype, layout=layout, grid_k=grid_k, tile_k=tile_k)
     if out.dtype != q.dtype:
         raise ValueError("out must have the dtype of q")
     check("vsa_attn_fwd", lib().vsa_attn_fwd(
@@ -98,10 +142,17 @@ def attn_fwd(q, k, v, idx, grid, tile, *, scale: float | None = None, out=None, 
     return out, lse
 
 
-def forward(q, k, v, grid, tile, topk: int, *, scale=None, stream=None):
-    """select + attn_fwd: (O, LSE, idx)."""
-    idx = select(q, k, grid, tile, topk, stream=stream)
-    o, lse = attn_fwd(q, k, v, idx, grid, tile, scale=scale, stream=stream)
+def forward(q, k, v, grid, tile, topk: int | None = None, *, sparsity: float | None = None, grid_k=None,
+            tile_k=None, layout: str = "bhnd", scale=None, stream=None):
+    """select + attn_fwd: (O, LSE, idx).  Give topk, or sparsity (the fraction
+    of key/value tiles left out, as in the fastbsa page's "Use" example)."""
+    if (topk is None) == (sparsity is None):
+        raise ValueError("give exactly one of topk and sparsity")
+    if topk is None:
+        topk = topk_from_sparsity(grid, tile, sparsity, grid_k, tile_k, _dims(q, layout)[3])
+    kw = dict(grid_k=grid_k, tile_k=tile_k, layout=layout, stream=stream)
+    idx = select(q, k, grid, tile, topk, **kw)
+    o, lse = attn_fwd(q, k, v, idx, grid, tile, scale=scale, **kw)
     return o, lse, idx
 
 

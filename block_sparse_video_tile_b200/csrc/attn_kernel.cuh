@@ -65,14 +65,14 @@ constexpr uint32_t kErrBadIndex = 2u;
 enum : int { MODE_SHARED = 0, MODE_TILE = 1, MODE_PAIR = 2 };
 
 struct AttnArgs {
-  Geom g;
+  Geom gq, gk;               // query side, key/value side (same tile volume)
   int topk;
   float scale_log2;          // softmax_scale * log2(e)
-  const int32_t* idx;        // [B*H, nT, topk]
-  uint16_t* o;               // [B*H, N, d], bf16 or fp16 like the inputs
-  float* lse;                // [B*H, N]
+  const int32_t* idx;        // [B*H, nTq, topk], entries in [0, nTk)
+  uint16_t* o;               // Q's layout, bf16 or fp16 like the inputs
+  float* lse;                // [B*H, Nq]
   unsigned int* err;         // device error word
-  int box_t;                 // t-extent of one TMA box (tt/2 in MODE_SHARED, else tt)
+  int box_tq, box_tk;        // t-extent of one TMA box per side (tt/2 in MODE_SHARED, else tt)
 };
 
 template <int D>
@@ -114,7 +114,7 @@ struct Slot {
 __device__ __forceinline__ int load_tile_index(const AttnArgs& a, const int32_t* row, int e,
                                                bool report) {
   int j = __ldg(row + e);
-  if (j < 0 || j >= a.g.nT) {
+  if (j < 0 || j >= a.gk.nT) {
     if (report) atomicCAS(a.err, 0u, kErrBadIndex);
     j = 0;
   }
@@ -156,7 +156,7 @@ struct KvSeq {
 
   __device__ void init(const AttnArgs& a, const uint2* table, int bh, int tile, const uint32_t* union_list = nullptr,
                        int union_len = 0) {
-    row = a.idx + (static_cast<size_t>(bh) * a.g.nT + tile) * a.topk;
+    row = a.idx + (static_cast<size_t>(bh) * a.gq.nT + tile) * a.topk;
     uni = union_list;
     ulen = union_len;
     tab = table;
@@ -164,7 +164,7 @@ struct KvSeq {
     half = 0;
   }
   __device__ bool second_half(const AttnArgs& a, int j) const {
-    return static_cast<int>(tab[j].x) * a.g.tt + a.box_t < a.g.T;
+    return static_cast<int>(tab[j].x) * a.gk.tt + a.box_tk < a.gk.T;
   }
   __device__ int count(const AttnArgs& a) const {
     if (MODE == MODE_TILE) return a.topk;
@@ -178,7 +178,7 @@ struct KvSeq {
     Piece pc;
     if (MODE == MODE_SHARED) {
       pc.j = load_tile_index(a, row, pos, report);
-      pc.toff = half * a.box_t;
+      pc.toff = half * a.box_tk;
       pc.real = pc.in_a = pc.in_b = true;
     } else if (MODE == MODE_TILE) {
       pc.j = load_tile_index(a, row, pos, report);
@@ -217,7 +217,7 @@ struct KvSeq {
 __device__ __forceinline__ int build_union(const AttnArgs& a, const int32_t* row_a, bool has_b, uint32_t* bm_a,
                                            uint32_t* bm_b, uint32_t* out) {
   const int lane = threadIdx.x % 32;
-  const int nw = (a.g.nT + 31) / 32;
+  const int nw = (a.gk.nT + 31) / 32;
   for (int w = lane; w < nw; w += 32) {
     bm_a[w] = 0u;
     bm_b[w] = 0u;
@@ -273,13 +273,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sp + L::kMisc + 4);
   uint2* tile_tab = reinterpret_cast<uint2*>(sp + L::kTiles);
   int* union_len = reinterpret_cast<int*>(sp + L::kMisc + 8);          // [2]
-  uint32_t* bitmaps = reinterpret_cast<uint32_t*>(sp + L::bitmap_off(a.g.nT));
-  uint32_t* unions = reinterpret_cast<uint32_t*>(sp + L::union_off(a.g.nT));
+  uint32_t* bitmaps = reinterpret_cast<uint32_t*>(sp + L::bitmap_off(a.gk.nT));
+  uint32_t* unions = reinterpret_cast<uint32_t*>(sp + L::union_off(a.gk.nT));
   auto bar = [&](int id) -> uint32_t { return sBar + 8u * static_cast<uint32_t>(id); };
 
-  const Geom& g = a.g;
+  const Geom& g = a.gq;                                     // query side
+  const Geom& gk = a.gk;                                    // key/value side
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int box_rows = SHARED ? kSubRows : g.vol;          // rows per TMA box
+  const int box_rows = SHARED ? kSubRows : g.vol;          // rows per TMA box (equal volumes)
   const uint32_t box_bytes = static_cast<uint32_t>(box_rows) * 128u;
 
   // ---- work unit -> slots
@@ -292,7 +293,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (SHARED) {
       bh = blockIdx.x / g.nT;
       tile = blockIdx.x % g.nT;
-      toff = h * a.box_t;
+      toff = h * a.box_tq;
       act = true;
     } else if (MODE == MODE_TILE) {
       const long long gidx = 2ll * blockIdx.x + h;
@@ -325,8 +326,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int last_active = slot[1].active ? 1 : 0;
 
   // ---- setup: tile table, barriers, zero rows of a missing tile B, TMEM
-  for (int j = threadIdx.x; j < g.nT; j += kAttnThreads) {
-    const TileCoord c = tile_coord(g, j);
+  for (int j = threadIdx.x; j < gk.nT; j += kAttnThreads) {
+    const TileCoord c = tile_coord(gk, j);
     tile_tab[j] = make_uint2(static_cast<uint32_t>(c.bt),
                              static_cast<uint32_t>(c.by) | (static_cast<uint32_t>(c.bx) << 16));
   }
@@ -345,7 +346,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     int len = 0;
     if (sl.active) {
       const int32_t* row_a = a.idx + (static_cast<size_t>(sl.bh) * g.nT + sl.tile) * a.topk;
-      const int nw = L::bitmap_words(g.nT);
+      const int nw = L::bitmap_words(gk.nT);
       len = build_union(a, row_a, sl.has_b, bitmaps + 2 * h * nw, bitmaps + (2 * h + 1) * nw,
                         unions + h * 2 * a.topk);
     }
@@ -387,12 +388,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!slot[h].active) continue;
         const int nbox = (PAIR && slot[h].has_b) ? 2 : 1;
         mbar_arrive_expect_tx(bar(BAR_Q_FULL + h), static_cast<uint32_t>(nbox * L::kSlabs) * box_bytes);
+        const BoxCoord ca = box_coord(g, slot[h].bh, slot[h].t0, slot[h].y0, slot[h].x0);
+        const BoxCoord cb = box_coord(g, slot[h].bh, slot[h].tb0, slot[h].yb0, slot[h].xb0);
         for (int sl = 0; sl < L::kSlabs; ++sl) {
-          tma_load_5d(sQ + h * L::kBufBytes + sl * L::kSlabBytes, &tmQ, bar(BAR_Q_FULL + h), sl * 64,
-                      slot[h].x0, slot[h].y0, slot[h].t0, slot[h].bh);
+          tma_load_5d(sQ + h * L::kBufBytes + sl * L::kSlabBytes, &tmQ, bar(BAR_Q_FULL + h), sl * 64, ca.c1,
+                      ca.c2, ca.c3, ca.c4);
           if (nbox == 2)
             tma_load_5d(sQ + h * L::kBufBytes + sl * L::kSlabBytes + box_bytes, &tmQ, bar(BAR_Q_FULL + h),
-                        sl * 64, slot[h].xb0, slot[h].yb0, slot[h].tb0, slot[h].bh);
+                        sl * 64, cb.c1, cb.c2, cb.c3, cb.c4);
         }
       }
       KvSeq<MODE> sq[2];
@@ -425,10 +428,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             for (int p = 0; p < P; ++p) {
               const Piece pc = sq[h].piece(a, p, kv == 0);
               const TileCoord c = table_coord(tile_tab, pc.j);
+              const BoxCoord bc = box_coord(gk, slot[h].bh, c.bt * gk.tt + pc.toff, c.by * gk.th, c.bx * gk.tw);
               for (int sl = 0; sl < L::kSlabs; ++sl)
                 tma_load_5d(buf0 + st * L::kBufBytes + sl * L::kSlabBytes + p * box_bytes, tm,
-                            bar(full + st), sl * 64, c.bx * g.tw, c.by * g.th, c.bt * g.tt + pc.toff,
-                            slot[h].bh);
+                            bar(full + st), sl * 64, bc.c1, bc.c2, bc.c3, bc.c4);
             }
           }
         }
@@ -534,6 +537,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t tS = tmem + lane_base + 128u * h;
       const uint32_t tO = tmem + lane_base + 256u + 128u * h;
       const int lg_yx = g.lg_th + g.lg_tw;
+      const int lg_yx_k = gk.lg_th + gk.lg_tw;
 
       // which token this row is (if any)
       bool row_valid;
@@ -545,7 +549,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tok_y = me.y0 + ly;
         tok_x = me.x0 + lx;
         row_valid = rr < box_rows && tok_t < g.T && tok_y < g.Hh && tok_x < g.W &&
-                    lt < (SHARED ? a.box_t : g.tt) && (!in_b || me.has_b);
+                    lt < (SHARED ? a.box_tq : g.tt) && (!in_b || me.has_b);
       }
 
       KvSeq<MODE> sq;
@@ -568,10 +572,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const Piece pc = sq.piece(a, p, false);
             const TileCoord c = table_coord(tile_tab, pc.j);
             int et, ey, ex;
-            tile_extent(g, c, et, ey, ex);
-            const int vt = SHARED ? min(a.box_t, et - pc.toff) : et;
+            tile_extent(gk, c, et, ey, ex);
+            const int vt = SHARED ? min(a.box_tk, et - pc.toff) : et;
             const bool use = pc.real && (in_b ? pc.in_b : pc.in_a);
-            const bool gfull = vt == (SHARED ? a.box_t : g.tt) && ey == g.th && ex == g.tw;
+            const bool gfull = vt == (SHARED ? a.box_tk : gk.tt) && ey == gk.th && ex == gk.tw;
             geo_full = geo_full && (!use || gfull);
             if (p == 0) { vt0 = vt; vy0 = ey; vx0 = ex; use0 = use; }
             else        { vt1 = vt; vy1 = ey; vx1 = ex; use1 = use; }
@@ -581,9 +585,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
               const int col = 32 * w + lane;
-              const bool second = PAIR && col >= g.vol;
-              const int rr = second ? col - g.vol : col;
-              const int lt = rr >> lg_yx, ly = (rr >> g.lg_tw) & (g.th - 1), lx = rr & (g.tw - 1);
+              const bool second = PAIR && col >= gk.vol;
+              const int rr = second ? col - gk.vol : col;
+              const int lt = rr >> lg_yx_k, ly = (rr >> gk.lg_tw) & (gk.th - 1), lx = rr & (gk.tw - 1);
               const bool v = second ? (use1 && lt < vt1 && ly < vy1 && lx < vx1)
                                     : (use0 && lt < vt0 && ly < vy0 && lx < vx0);
               mw[w] = __ballot_sync(0xffffffffu, v);
@@ -693,7 +697,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const float inv_l = 1.f / l;
         const size_t N = static_cast<size_t>(g.T) * g.Hh * g.W;
         const size_t n_tok = (static_cast<size_t>(tok_t) * g.Hh + tok_y) * g.W + tok_x;
-        uint16_t* orow = a.o + (static_cast<size_t>(me.bh) * N + n_tok) * D;
+        uint16_t* orow = a.o + token_offset(g, me.bh, n_tok);
 #pragma unroll
         for (int c4 = 0; c4 < D / 32; ++c4) {
           uint32_t ov[32];

@@ -24,34 +24,52 @@ constexpr int kMaxDevices = 64;
 constexpr int kMaxSmemPerBlock = 232448;  // opt-in dynamic shared memory per CTA on sm_100
 
 // -------------------------------------------------------------- validation
-static int make_geom(const vsa_shape* s, Geom* g) {
-  if (s == nullptr) return VSA_ERR_INVALID_ARG;
-  if (s->B <= 0 || s->H <= 0 || s->T <= 0 || s->Hh <= 0 || s->W <= 0 || s->d <= 0 || s->tt <= 0 ||
-      s->th <= 0 || s->tw <= 0)
-    return VSA_ERR_INVALID_ARG;
-  if (s->d != 64 && s->d != 128) return VSA_ERR_UNSUPPORTED;
-  if (s->dtype != VSA_DTYPE_BF16 && s->dtype != VSA_DTYPE_F16) return VSA_ERR_UNSUPPORTED;
-  const int lt = ilog2_exact(s->tt), ly = ilog2_exact(s->th), lx = ilog2_exact(s->tw);
+// One side's grid and tile: positive extents, power-of-two tile extents with
+// a supported volume, tile counts and index ranges within the kernels' limits.
+static int side_geom(const vsa_shape* s, int T, int Hh, int W, int tt, int th, int tw, Geom* g) {
+  if (T <= 0 || Hh <= 0 || W <= 0 || tt <= 0 || th <= 0 || tw <= 0) return VSA_ERR_INVALID_ARG;
+  const int lt = ilog2_exact(tt), ly = ilog2_exact(th), lx = ilog2_exact(tw);
   if (lt < 0 || ly < 0 || lx < 0) return VSA_ERR_UNSUPPORTED;
-  if (s->tt > 256 || s->th > 256 || s->tw > 256) return VSA_ERR_UNSUPPORTED;
-  const int vol = s->tt * s->th * s->tw;
+  if (tt > 256 || th > 256 || tw > 256) return VSA_ERR_UNSUPPORTED;
+  const int vol = tt * th * tw;
   if (vol != 64 && vol != 128 && vol != 256) return VSA_ERR_UNSUPPORTED;
-  if (vol == 256 && s->tt < 2) return VSA_ERR_UNSUPPORTED;
-  g->B = s->B; g->H = s->H; g->T = s->T; g->Hh = s->Hh; g->W = s->W; g->d = s->d;
-  g->tt = s->tt; g->th = s->th; g->tw = s->tw;
+  if (vol == 256 && tt < 2) return VSA_ERR_UNSUPPORTED;
+  g->B = s->B; g->H = s->H; g->T = T; g->Hh = Hh; g->W = W; g->d = s->d;
+  g->tt = tt; g->th = th; g->tw = tw;
   g->lg_tt = lt; g->lg_th = ly; g->lg_tw = lx;
   g->vol = vol;
   g->f16 = s->dtype == VSA_DTYPE_F16 ? 1 : 0;
-  g->nTt = ceil_div(s->T, s->tt);
-  g->nTy = ceil_div(s->Hh, s->th);
-  g->nTx = ceil_div(s->W, s->tw);
+  g->layout = s->layout;
+  g->nTt = ceil_div(T, tt);
+  g->nTy = ceil_div(Hh, th);
+  g->nTx = ceil_div(W, tw);
   const long long nT = 1ll * g->nTt * g->nTy * g->nTx;
-  const long long N = 1ll * s->T * s->Hh * s->W;
+  const long long N = 1ll * T * Hh * W;
   const long long BH = 1ll * s->B * s->H;
   // grid-dimension and index limits of the kernels
-  if (nT > kMaxTiles || BH > 65535 || BH * nT > 0x7fffffffll || N * s->d * BH > (1ll << 40))
+  if (nT > kMaxTiles || BH > 65535 || BH * nT > 0x7fffffffll || N * s->d * BH > (1ll << 40) ||
+      1ll * s->B * T > 0x7fffffffll)
     return VSA_ERR_TOO_LARGE;
   g->nT = static_cast<int>(nT);
+  return VSA_OK;
+}
+
+// Query-side and key/value-side geometry of a shape (the key/value grid and
+// tile default to the query's when left zero).
+static int make_geoms(const vsa_shape* s, Geom* gq, Geom* gk) {
+  if (s == nullptr) return VSA_ERR_INVALID_ARG;
+  if (s->B <= 0 || s->H <= 0 || s->d <= 0) return VSA_ERR_INVALID_ARG;
+  if (s->d != 64 && s->d != 128) return VSA_ERR_UNSUPPORTED;
+  if (s->dtype != VSA_DTYPE_BF16 && s->dtype != VSA_DTYPE_F16) return VSA_ERR_UNSUPPORTED;
+  if (s->layout != VSA_LAYOUT_BHND && s->layout != VSA_LAYOUT_BNHD) return VSA_ERR_UNSUPPORTED;
+  int rc = side_geom(s, s->T, s->Hh, s->W, s->tt, s->th, s->tw, gq);
+  if (rc != VSA_OK) return rc;
+  const bool kgrid = s->Tk != 0 || s->Hk != 0 || s->Wk != 0;
+  const bool ktile = s->tk != 0 || s->hk != 0 || s->wk != 0;
+  rc = side_geom(s, kgrid ? s->Tk : s->T, kgrid ? s->Hk : s->Hh, kgrid ? s->Wk : s->W, ktile ? s->tk : s->tt,
+                 ktile ? s->hk : s->th, ktile ? s->wk : s->tw, gk);
+  if (rc != VSA_OK) return rc;
+  if (gq->vol != gk->vol) return VSA_ERR_UNSUPPORTED;
   return VSA_OK;
 }
 
@@ -85,17 +103,17 @@ static unsigned int* device_error_ptr() {
 // heads (little score work, more CTAs) and larger ones (key rows that would
 // not fit beside the wide ring) take the narrow kernel (16).
 template <int D>
-static int launch_score(const Geom& g, int topk, int32_t* idx, const float* means, unsigned int* err,
+static int launch_score(const Geom& gq, const Geom& gk, int topk, int32_t* idx, const float* means,
                         cudaStream_t st) {
-  const bool wide = g.nT > kNarrowMaxTiles && g.nT <= kWideMaxTiles;
-  const size_t smem = wide ? score_smem_bytes<D>(g) : score_narrow_smem_bytes<D>(g);
+  const bool wide = gk.nT > kNarrowMaxTiles && gk.nT <= kWideMaxTiles;
+  const size_t smem = wide ? score_smem_bytes<D>(gk) : score_narrow_smem_bytes<D>(gk);
   const void* fn = wide ? reinterpret_cast<const void*>(score_topk_kernel<D>)
                         : reinterpret_cast<const void*>(score_topk_narrow_kernel<D>);
   if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
     return VSA_ERR_CUDA;
   const int rows = wide ? kWideRows : kNarrowRows;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(ceil_div(g.nT, rows), g.B * g.H);
+  cfg.gridDim = dim3(ceil_div(gq.nT, rows), gq.B * gq.H);
   cfg.blockDim = dim3(wide ? kWideThreads : kNarrowThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -104,42 +122,43 @@ static int launch_score(const Geom& g, int topk, int32_t* idx, const float* mean
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = wide ? cudaLaunchKernelEx(&cfg, score_topk_kernel<D>, g, means, topk, idx)
-                             : cudaLaunchKernelEx(&cfg, score_topk_narrow_kernel<D>, g, means, topk, idx);
+  const cudaError_t e = wide ? cudaLaunchKernelEx(&cfg, score_topk_kernel<D>, gq, gk, means, topk, idx)
+                             : cudaLaunchKernelEx(&cfg, score_topk_narrow_kernel<D>, gq, gk, means, topk, idx);
   return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 
 template <int D, bool F16>
-static int launch_select(const Geom& g, const void* q, const void* k, int topk, int32_t* idx, void* ws,
+static int launch_select(const Geom& gq, const Geom& gk, const void* q, const void* k, int topk, int32_t* idx, void* ws,
                          cudaStream_t st) {
   CUtensorMap mq, mk;
   int rc;
-  if ((rc = encode_qkv_map(&mq, q, g, g.tt, F16)) != VSA_OK || (rc = encode_qkv_map(&mk, k, g, g.tt, F16)) != VSA_OK)
+  if ((rc = encode_qkv_map(&mq, q, gq, gq.tt, F16)) != VSA_OK || (rc = encode_qkv_map(&mk, k, gk, gk.tt, F16)) != VSA_OK)
     return rc;
   unsigned int* err = device_error_ptr();
   if (err == nullptr) return VSA_ERR_CUDA;
   float* means = static_cast<float*>(ws);
-  const size_t psmem = pool_smem_bytes<D>(g);
+  const size_t psmem = pool_smem_bytes<D>(gq);
   if (cudaFuncSetAttribute(pool_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(psmem)) != cudaSuccess)
     return VSA_ERR_CUDA;
-  pool_kernel<D, F16><<<dim3(g.nT, g.B * g.H, 2), kPoolThreads, psmem, st>>>(mq, mk, g, means, err);
+  pool_kernel<D, F16><<<dim3(max(gq.nT, gk.nT), gq.B * gq.H, 2), kPoolThreads, psmem, st>>>(mq, mk, gq, gk, means,
+                                                                                              err);
   if (cudaGetLastError() != cudaSuccess) return VSA_ERR_CUDA;
-  return launch_score<D>(g, topk, idx, means, err, st);
+  return launch_score<D>(gq, gk, topk, idx, means, st);
 }
 
 template <int D, int MODE, bool F16>
 static int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnArgs& a,
                        cudaStream_t st) {
-  const int smem = AttnSmem<D>::alloc(a.g.nT, a.topk, MODE == MODE_PAIR);
+  const int smem = AttnSmem<D>::alloc(a.gk.nT, a.topk, MODE == MODE_PAIR);
   if (cudaFuncSetAttribute(attn_fwd_kernel<D, MODE, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return VSA_ERR_CUDA;
-  const long long BH = 1ll * a.g.B * a.g.H;
+  const long long BH = 1ll * a.gq.B * a.gq.H;
   long long grid;
-  if (MODE == MODE_SHARED) grid = BH * a.g.nT;                             // one tile, two t-halves
-  else if (MODE == MODE_TILE) grid = (BH * a.g.nT + 1) / 2;                // two tiles
-  else grid = (BH * ((a.g.nT + 1) / 2) + 1) / 2;                           // two pairs of tiles
+  if (MODE == MODE_SHARED) grid = BH * a.gq.nT;                            // one tile, two t-halves
+  else if (MODE == MODE_TILE) grid = (BH * a.gq.nT + 1) / 2;               // two tiles
+  else grid = (BH * ((a.gq.nT + 1) / 2) + 1) / 2;                          // two pairs of tiles
   attn_fwd_kernel<D, MODE, F16><<<static_cast<unsigned>(grid), kAttnThreads, smem, st>>>(mq, mk, mv, a);
   return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
@@ -179,12 +198,22 @@ static int dispatch_attn(int d, int mode, const CUtensorMap& mq, const CUtensorM
   return launch_attn<64, MODE_PAIR, F16>(mq, mk, mv, a, st);
 }
 
-static int dispatch_select(const Geom& g, const void* q, const void* k, int topk, int32_t* idx, void* ws,
-                           cudaStream_t st) {
-  if (g.d == 128) return g.f16 ? launch_select<128, true>(g, q, k, topk, idx, ws, st)
-                               : launch_select<128, false>(g, q, k, topk, idx, ws, st);
-  return g.f16 ? launch_select<64, true>(g, q, k, topk, idx, ws, st)
-               : launch_select<64, false>(g, q, k, topk, idx, ws, st);
+static int dispatch_select(const Geom& gq, const Geom& gk, const void* q, const void* k, int topk, int32_t* idx,
+                           void* ws, cudaStream_t st) {
+  if (gq.d == 128) return gq.f16 ? launch_select<128, true>(gq, gk, q, k, topk, idx, ws, st)
+                                 : launch_select<128, false>(gq, gk, q, k, topk, idx, ws, st);
+  return gq.f16 ? launch_select<64, true>(gq, gk, q, k, topk, idx, ws, st)
+                : launch_select<64, false>(gq, gk, q, k, topk, idx, ws, st);
+}
+
+static int tile_count_of(const Geom& g, int32_t* num_tiles, int32_t* tiles_per_axis) {
+  *num_tiles = g.nT;
+  if (tiles_per_axis != nullptr) {
+    tiles_per_axis[0] = g.nTt;
+    tiles_per_axis[1] = g.nTy;
+    tiles_per_axis[2] = g.nTx;
+  }
+  return VSA_OK;
 }
 
 }  // namespace vsa
@@ -195,92 +224,110 @@ extern "C" {
 
 int vsa_tile_count(const vsa_shape* shape, int32_t* num_tiles, int32_t* tiles_per_axis) {
   if (num_tiles == nullptr) return VSA_ERR_INVALID_ARG;
-  Geom g;
-  const int rc = make_geom(shape, &g);
+  Geom gq, gk;
+  const int rc = make_geoms(shape, &gq, &gk);
+  return rc != VSA_OK ? rc : tile_count_of(gq, num_tiles, tiles_per_axis);
+}
+
+int vsa_kv_tile_count(const vsa_shape* shape, int32_t* num_tiles, int32_t* tiles_per_axis) {
+  if (num_tiles == nullptr) return VSA_ERR_INVALID_ARG;
+  Geom gq, gk;
+  const int rc = make_geoms(shape, &gq, &gk);
+  return rc != VSA_OK ? rc : tile_count_of(gk, num_tiles, tiles_per_axis);
+}
+
+int vsa_topk_from_sparsity(const vsa_shape* shape, float sparsity, int32_t* topk) {
+  if (topk == nullptr) return VSA_ERR_INVALID_ARG;
+  Geom gq, gk;
+  const int rc = make_geoms(shape, &gq, &gk);
   if (rc != VSA_OK) return rc;
-  *num_tiles = g.nT;
-  if (tiles_per_axis != nullptr) {
-    tiles_per_axis[0] = g.nTt;
-    tiles_per_axis[1] = g.nTy;
-    tiles_per_axis[2] = g.nTx;
-  }
+  if (!(sparsity >= 0.f && sparsity < 1.f)) return VSA_ERR_TOPK_RANGE;
+  const double keep = (1.0 - static_cast<double>(sparsity)) * gk.nT;
+  long long k = static_cast<long long>(std::floor(keep + 0.5));
+  if (k < 1) k = 1;
+  if (k > gk.nT) k = gk.nT;
+  *topk = static_cast<int32_t>(k);
   return VSA_OK;
 }
 
 size_t vsa_select_workspace_bytes(const vsa_shape* shape) {
-  Geom g;
-  if (make_geom(shape, &g) != VSA_OK) return 0;
-  return select_workspace_bytes(g);
+  Geom gq, gk;
+  if (make_geoms(shape, &gq, &gk) != VSA_OK) return 0;
+  return select_workspace_bytes(gq, gk);
 }
 
 int vsa_select(const vsa_shape* shape, const void* q, const void* k, int32_t topk, int32_t* idx_out,
                void* workspace, size_t workspace_bytes, void* stream) {
-  Geom g;
-  int rc = make_geom(shape, &g);
+  Geom gq, gk;
+  int rc = make_geoms(shape, &gq, &gk);
   if (rc != VSA_OK) return rc;
   if (q == nullptr || k == nullptr || idx_out == nullptr) return VSA_ERR_INVALID_ARG;
-  if (topk <= 0 || topk > g.nT) return VSA_ERR_TOPK_RANGE;
+  if (topk <= 0 || topk > gk.nT) return VSA_ERR_TOPK_RANGE;
   if (!aligned16(q) || !aligned16(k) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(idx_out) & 3u))
     return VSA_ERR_ALIGNMENT;
-  if (workspace == nullptr || workspace_bytes < vsa_select_workspace_bytes(shape)) return VSA_ERR_WORKSPACE;
+  if (workspace == nullptr || workspace_bytes < select_workspace_bytes(gq, gk)) return VSA_ERR_WORKSPACE;
   if ((rc = check_arch()) != VSA_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return dispatch_select(g, q, k, topk, idx_out, workspace, st);
+  return dispatch_select(gq, gk, q, k, topk, idx_out, workspace, st);
 }
 
 int vsa_select_noalloc(const vsa_shape* shape, const void* q, const void* k, int32_t topk, int32_t* idx_out,
                        void* stream) {
-  Geom g;
-  int rc = make_geom(shape, &g);
+  Geom gq, gk;
+  int rc = make_geoms(shape, &gq, &gk);
   if (rc != VSA_OK) return rc;
   if (q == nullptr || k == nullptr || idx_out == nullptr) return VSA_ERR_INVALID_ARG;
-  if (topk <= 0 || topk > g.nT) return VSA_ERR_TOPK_RANGE;
+  if (topk <= 0 || topk > gk.nT) return VSA_ERR_TOPK_RANGE;
   if (!aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(idx_out) & 3u)) return VSA_ERR_ALIGNMENT;
-  if (vsa_select_workspace_bytes(shape) > VSA_SELECT_NOALLOC_SCRATCH_BYTES) return VSA_ERR_WORKSPACE;
+  if (select_workspace_bytes(gq, gk) > VSA_SELECT_NOALLOC_SCRATCH_BYTES) return VSA_ERR_WORKSPACE;
   if ((rc = check_arch()) != VSA_OK) return rc;
   float* ws = nullptr;
   if ((rc = select_scratch_ptr(&ws)) != VSA_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return dispatch_select(g, q, k, topk, idx_out, ws, st);
+  return dispatch_select(gq, gk, q, k, topk, idx_out, ws, st);
 }
 
 int vsa_attn_fwd(const vsa_shape* shape, const void* q, const void* k, const void* v, const int32_t* idx,
                  int32_t topk, float softmax_scale, void* o, float* lse, void* stream) {
-  Geom g;
-  int rc = make_geom(shape, &g);
+  Geom gq, gk;
+  int rc = make_geoms(shape, &gq, &gk);
   if (rc != VSA_OK) return rc;
   if (q == nullptr || k == nullptr || v == nullptr || idx == nullptr || o == nullptr || lse == nullptr)
     return VSA_ERR_INVALID_ARG;
   if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return VSA_ERR_INVALID_ARG;
-  if (topk <= 0 || topk > g.nT) return VSA_ERR_TOPK_RANGE;
+  if (topk <= 0 || topk > gk.nT) return VSA_ERR_TOPK_RANGE;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
       (reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u))
     return VSA_ERR_ALIGNMENT;
-  const int mode = g.vol == 256 ? MODE_SHARED : (g.vol == 128 ? MODE_TILE : MODE_PAIR);
-  const int smem = g.d == 128 ? AttnSmem<128>::alloc(g.nT, topk, mode == MODE_PAIR)
-                              : AttnSmem<64>::alloc(g.nT, topk, mode == MODE_PAIR);
+  const int vol = gq.vol;                    // equal on both sides
+  const int mode = vol == 256 ? MODE_SHARED : (vol == 128 ? MODE_TILE : MODE_PAIR);
+  const int smem = gq.d == 128 ? AttnSmem<128>::alloc(gk.nT, topk, mode == MODE_PAIR)
+                               : AttnSmem<64>::alloc(gk.nT, topk, mode == MODE_PAIR);
   if (smem > kMaxSmemPerBlock) return VSA_ERR_TOO_LARGE;
   if ((rc = check_arch()) != VSA_OK) return rc;
 
-  const bool shared = (g.vol == 256);
+  const bool shared = (vol == 256);
   AttnArgs a;
-  a.g = g;
+  a.gq = gq;
+  a.gk = gk;
   a.topk = topk;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
   a.idx = idx;
   a.o = static_cast<uint16_t*>(o);
   a.lse = lse;
   a.err = device_error_ptr();
-  a.box_t = shared ? g.tt / 2 : g.tt;
+  a.box_tq = shared ? gq.tt / 2 : gq.tt;
+  a.box_tk = shared ? gk.tt / 2 : gk.tt;
   if (a.err == nullptr) return VSA_ERR_CUDA;
   CUtensorMap mq, mk, mv;
-  const bool f16 = g.f16 != 0;
-  if ((rc = encode_qkv_map(&mq, q, g, a.box_t, f16)) != VSA_OK ||
-      (rc = encode_qkv_map(&mk, k, g, a.box_t, f16)) != VSA_OK ||
-      (rc = encode_qkv_map(&mv, v, g, a.box_t, f16)) != VSA_OK)
+  const bool f16 = gq.f16 != 0;
+  if ((rc = encode_qkv_map(&mq, q, gq, a.box_tq, f16)) != VSA_OK ||
+      (rc = encode_qkv_map(&mk, k, gk, a.box_tk, f16)) != VSA_OK ||
+      (rc = encode_qkv_map(&mv, v, gk, a.box_tk, f16)) != VSA_OK)
     return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return f16 ? dispatch_attn<true>(g.d, mode, mq, mk, mv, a, st) : dispatch_attn<false>(g.d, mode, mq, mk, mv, a, st);
+  return f16 ? dispatch_attn<true>(gq.d, mode, mq, mk, mv, a, st)
+             : dispatch_attn<false>(gq.d, mode, mq, mk, mv, a, st);
 }
 
 int vsa_device_error(uint32_t* code, int32_t reset) {

@@ -8,10 +8,10 @@
 //
 // Two kernels:
 //   pool_kernel        HBM-bound: reads every Q and K byte once and writes the
-//                      per-tile float32 means, transposed, to the caller's
-//                      workspace: [2, B*H, d, ldT] (Q, then K), ldT = nT
-//                      rounded up to 4.
-//   score_topk_kernel  per (head, block of R query tiles): the R x nT score
+//                      per-tile float32 means, channel-major, to the caller's
+//                      workspace: Q means [B*H, d, ldq], then K means
+//                      [B*H, d, ldk] (ldq, ldk: nTq, nTk rounded up to 4).
+//   score_topk_kernel  per (head, block of R query tiles): the R x nTk score
 //                      rows in shared memory (float32 FMA, channels summed in
 //                      ascending order) and each row's exact top-k; writes
 //                      ascending idx.  Launched as a programmatic dependent of
@@ -34,8 +34,15 @@ constexpr int kPoolThreads = 256;
 // Row stride (floats) of the transposed tile means.
 __host__ __device__ inline int means_ld(int nT) { return (nT + 3) & ~3; }
 
-inline size_t select_workspace_bytes(const Geom& g) {
-  return sizeof(float) * 2ull * g.B * g.H * g.d * means_ld(g.nT);
+inline size_t select_workspace_bytes(const Geom& gq, const Geom& gk) {
+  return sizeof(float) * static_cast<size_t>(gq.B) * gq.H * gq.d * (means_ld(gq.nT) + means_ld(gk.nT));
+}
+
+// Start of head bh's means of side z (0: Q, 1: K) in the workspace.
+__host__ __device__ inline size_t means_offset(const Geom& gq, const Geom& gk, int z, int bh) {
+  const size_t BH = static_cast<size_t>(gq.B) * gq.H;
+  return z == 0 ? static_cast<size_t>(bh) * gq.d * means_ld(gq.nT)
+                : BH * gq.d * means_ld(gq.nT) + static_cast<size_t>(bh) * gk.d * means_ld(gk.nT);
 }
 
 // Larger float -> larger unsigned key (total order; -0 < +0, scores are
@@ -137,17 +144,19 @@ __device__ __forceinline__ void bsearch_topk_rows(const uint32_t* kr, int kst, i
   }
 }
 
-// One CTA per (tile j, head bh, tensor z in {Q, K}).  The whole tile is one
-// 5-D TMA box per 64-channel slab (the same [B*H, T, Hh, W, d] view the
-// attend kernel uses), so a 256-token tile of d = 128 puts 64 KB in flight
-// per CTA without using registers; positions past the grid edge arrive as
-// zeros and add nothing to the sums.  Threads then sum 16-byte chunks down the
-// rows in a fixed order (deterministic) and divide by the tile's valid count.
+// One CTA per (tile j, head bh, tensor z in {Q, K}), each side with its own
+// grid and tile (CTAs past a side's tile count exit).  The whole tile is one
+// 5-D TMA box per 64-channel slab (the same views the attend kernel uses), so
+// a 256-token tile of d = 128 puts 64 KB in flight per CTA without using
+// registers; positions past the y and x edges arrive as zeros, and rows past
+// the t edge are left out of the sums (in the [B, N, H, d] view they hold the
+// next batch's frames).  Threads sum 16-byte chunks down the rows in a fixed
+// order (deterministic) and divide by the tile's valid count.
 // Dynamic shared memory: box (slabs x vol x 128 B, 1024-aligned) | partial sums | mbarrier.
 template <int D, bool F16>
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __grid_constant__ CUtensorMap tmQ,
-                                                            const __grid_constant__ CUtensorMap tmK, Geom g,
-                                                            float* __restrict__ means, unsigned int* err) {
+                                                            const __grid_constant__ CUtensorMap tmK, Geom gq,
+                                                            Geom gk, float* __restrict__ means, unsigned int* err) {
   constexpr int kSlabs = D / 64;
   constexpr int TPR = D / 8;                 // threads per row (one 16-byte chunk each)
   constexpr int RP = kPoolThreads / TPR;     // row groups
@@ -155,22 +164,27 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __grid_constan
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* sp = smem_raw + (base - raw);
+  const int z = blockIdx.z;
+  const Geom& g = z == 0 ? gq : gk;
+  const int j = blockIdx.x;
+  if (j >= g.nT) return;
   const int vol = g.vol;
   const int box_bytes = vol * 128;
   float* part = reinterpret_cast<float*>(sp + kSlabs * box_bytes);     // [RP][D]
   const uint32_t bar = base + kSlabs * box_bytes + RP * D * 4;
 
-  const int j = blockIdx.x;
   const int bh = blockIdx.y;
-  const int z = blockIdx.z;
   const TileCoord c = tile_coord(g, j);
+  int vt, vy, vx;
+  tile_extent(g, c, vt, vy, vx);
   if (threadIdx.x == 0) {
     mbar_init(bar, 1);
     fence_mbar_init();
     mbar_arrive_expect_tx(bar, static_cast<uint32_t>(kSlabs * box_bytes));
+    const BoxCoord bc = box_coord(g, bh, c.bt * g.tt, c.by * g.th, c.bx * g.tw);
     for (int sl = 0; sl < kSlabs; ++sl)
       tma_load_5d(base + sl * box_bytes, z == 0 ? static_cast<const void*>(&tmQ) : static_cast<const void*>(&tmK),
-                  bar, sl * 64, c.bx * g.tw, c.by * g.th, c.bt * g.tt, bh);
+                  bar, sl * 64, bc.c1, bc.c2, bc.c3, bc.c4);
   }
   // let the score kernel's launch begin while this grid drains
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -183,9 +197,10 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __grid_constan
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  const int rows = vt * g.th * g.tw;          // rows of the box inside the t extent
   if (ok) {
 #pragma unroll 4
-    for (int r = rg; r < vol; r += RP) {
+    for (int r = rg; r < rows; r += RP) {
       const uint4 u = *reinterpret_cast<const uint4*>(slab + r * 128 + (((cc % 8) ^ (r & 7)) << 4));
       const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -199,11 +214,9 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __grid_constan
 #pragma unroll
   for (int e = 0; e < 8; ++e) part[rg * D + cc * 8 + e] = acc[e];
   __syncthreads();
-  int vt, vy, vx;
-  tile_extent(g, c, vt, vy, vx);
   const float cnt = static_cast<float>(vt * vy * vx);
   const int ld = means_ld(g.nT);
-  float* mz = means + (static_cast<size_t>(z) * g.B * g.H + bh) * D * ld;
+  float* mz = means + means_offset(gq, gk, z, bh);
   for (int col = threadIdx.x; col < D; col += kPoolThreads) {
     float sum = 0.f;
 #pragma unroll 8
@@ -267,7 +280,7 @@ constexpr int kWideMaxTiles = 768;
 constexpr int kNarrowMaxTiles = 256;   // below this the narrow kernel is used too (more, shorter CTAs)
 
 template <int D>
-__global__ void __launch_bounds__(kWideThreads) score_topk_kernel(Geom g, const float* __restrict__ means, int topk,
+__global__ void __launch_bounds__(kWideThreads) score_topk_kernel(Geom gq, Geom gk, const float* __restrict__ means, int topk,
                                                                   int32_t* __restrict__ idx) {
   constexpr int SPP = D / kWideSlice;      // stages per pass
   constexpr int SLICE = kWideSlice * kWideKeys;
@@ -278,22 +291,22 @@ __global__ void __launch_bounds__(kWideThreads) score_topk_kernel(Geom g, const 
   float* qT = reinterpret_cast<float*>(smem_raw);
   float* ring = qT + D * R;
   uint32_t* keys = reinterpret_cast<uint32_t*>(ring + kWideStages * SLICE);
-  const int nT = g.nT, ld = means_ld(nT);
+  const int nT = gk.nT;                     // key tiles (score columns, top-k candidates)
+  const int ldq = means_ld(gq.nT), ldk = means_ld(nT);
   const int bh = blockIdx.y;
   const int row0 = blockIdx.x * R;
-  const int nrows = min(R, nT - row0);
-  const size_t BH = static_cast<size_t>(g.B) * g.H;
-  const float* mq = means + static_cast<size_t>(bh) * D * ld;
-  const float* mk = means + (BH + bh) * D * ld;
+  const int nrows = min(R, gq.nT - row0);
+  const float* mq = means + means_offset(gq, gk, 0, bh);
+  const float* mk = means + means_offset(gq, gk, 1, bh);
   const int nstage = ceil_div(nT, kWideKeys) * SPP;
 
   // query means (joined to the first cp.async group); float4s past the row are zero
   for (int f = threadIdx.x; f < D * R / 4; f += kWideThreads) {
     const int c = f / (R / 4), r4 = f % (R / 4);
     const int row = row0 + 4 * r4;
-    const bool in = row < ld;
+    const bool in = row < ldq;
     cp_async16(smem_u32(qT + c * R + 4 * r4),
-               in ? static_cast<const void*>(mq + static_cast<size_t>(c) * ld + row) : static_cast<const void*>(mq),
+               in ? static_cast<const void*>(mq + static_cast<size_t>(c) * ldq + row) : static_cast<const void*>(mq),
                in ? 16u : 0u);
   }
   // stage st = (pass st / SPP, channel slice st % SPP) -> ring slot st % 3; one group per call
@@ -305,9 +318,9 @@ __global__ void __launch_bounds__(kWideThreads) score_topk_kernel(Geom g, const 
       for (int f = threadIdx.x; f < SLICE / 4; f += kWideThreads) {
         const int c = f / (kWideKeys / 4), k4 = f % (kWideKeys / 4);
         const int key = kc0 + 4 * k4;
-        const bool in = key < ld;
+        const bool in = key < ldk;
         cp_async16(smem_u32(dst + c * kWideKeys + 4 * k4),
-                   in ? static_cast<const void*>(mk + static_cast<size_t>(c0 + c) * ld + key)
+                   in ? static_cast<const void*>(mk + static_cast<size_t>(c0 + c) * ldk + key)
                       : static_cast<const void*>(mk),
                    in ? 16u : 0u);
       }
@@ -363,13 +376,13 @@ __global__ void __launch_bounds__(kWideThreads) score_topk_kernel(Geom g, const 
   }
   cp_async_wait<0>();
   __syncthreads();
-  topk_rows(keys, nT, nT, nrows, topk, idx + (static_cast<size_t>(bh) * nT + row0) * topk, kWideThreads / 32);
+  topk_rows(keys, nT, nT, nrows, topk, idx + (static_cast<size_t>(bh) * gq.nT + row0) * topk, kWideThreads / 32);
 }
 
 template <int D>
-inline size_t score_smem_bytes(const Geom& g) {
+inline size_t score_smem_bytes(const Geom& gk) {
   return sizeof(float) * (static_cast<size_t>(D) * kWideRows + kWideStages * kWideSlice * kWideKeys) +
-         sizeof(uint32_t) * static_cast<size_t>(kWideRows) * g.nT;
+         sizeof(uint32_t) * static_cast<size_t>(kWideRows) * gk.nT;
 }
 
 // Narrow kernel (heads of at most kNarrowMaxTiles tiles, and of more than
@@ -387,7 +400,7 @@ constexpr int kNarrowStages = 4;
 constexpr int kNarrowThreads = 256;
 
 template <int D>
-__global__ void __launch_bounds__(kNarrowThreads) score_topk_narrow_kernel(Geom g, const float* __restrict__ means,
+__global__ void __launch_bounds__(kNarrowThreads) score_topk_narrow_kernel(Geom gq, Geom gk, const float* __restrict__ means,
                                                                            int topk, int32_t* __restrict__ idx) {
   constexpr int SPP = D / kNarrowSlice;
   constexpr int SLICE = kNarrowSlice * kNarrowKeys;
@@ -397,21 +410,21 @@ __global__ void __launch_bounds__(kNarrowThreads) score_topk_narrow_kernel(Geom 
   float* qT = reinterpret_cast<float*>(smem_raw);
   float* ring = qT + D * R;
   uint32_t* keys = reinterpret_cast<uint32_t*>(ring + kNarrowStages * SLICE);
-  const int nT = g.nT, ld = means_ld(nT);
+  const int nT = gk.nT;                     // key tiles (score columns, top-k candidates)
+  const int ldq = means_ld(gq.nT), ldk = means_ld(nT);
   const int bh = blockIdx.y;
   const int row0 = blockIdx.x * R;
-  const int nrows = min(R, nT - row0);
-  const size_t BH = static_cast<size_t>(g.B) * g.H;
-  const float* mq = means + static_cast<size_t>(bh) * D * ld;
-  const float* mk = means + (BH + bh) * D * ld;
+  const int nrows = min(R, gq.nT - row0);
+  const float* mq = means + means_offset(gq, gk, 0, bh);
+  const float* mk = means + means_offset(gq, gk, 1, bh);
   const int nstage = ceil_div(nT, kNarrowKeys) * SPP;
 
   for (int f = threadIdx.x; f < D * R / 4; f += kNarrowThreads) {
     const int c = f / (R / 4), r4 = f % (R / 4);
     const int row = row0 + 4 * r4;
-    const bool in = row < ld;
+    const bool in = row < ldq;
     cp_async16(smem_u32(qT + c * R + 4 * r4),
-               in ? static_cast<const void*>(mq + static_cast<size_t>(c) * ld + row) : static_cast<const void*>(mq),
+               in ? static_cast<const void*>(mq + static_cast<size_t>(c) * ldq + row) : static_cast<const void*>(mq),
                in ? 16u : 0u);
   }
   auto issue = [&](int st) {
@@ -421,9 +434,9 @@ __global__ void __launch_bounds__(kNarrowThreads) score_topk_narrow_kernel(Geom 
       for (int f = threadIdx.x; f < SLICE / 4; f += kNarrowThreads) {
         const int c = f / (kNarrowKeys / 4), k4 = f % (kNarrowKeys / 4);
         const int key = kc0 + 4 * k4;
-        const bool in = key < ld;
+        const bool in = key < ldk;
         cp_async16(smem_u32(dst + c * kNarrowKeys + 4 * k4),
-                   in ? static_cast<const void*>(mk + static_cast<size_t>(c0 + c) * ld + key)
+                   in ? static_cast<const void*>(mk + static_cast<size_t>(c0 + c) * ldk + key)
                       : static_cast<const void*>(mk),
                    in ? 16u : 0u);
       }
@@ -471,13 +484,13 @@ __global__ void __launch_bounds__(kNarrowThreads) score_topk_narrow_kernel(Geom 
   }
   cp_async_wait<0>();
   __syncthreads();
-  topk_rows(keys, nT, nT, nrows, topk, idx + (static_cast<size_t>(bh) * nT + row0) * topk, kNarrowThreads / 32);
+  topk_rows(keys, nT, nT, nrows, topk, idx + (static_cast<size_t>(bh) * gq.nT + row0) * topk, kNarrowThreads / 32);
 }
 
 template <int D>
-inline size_t score_narrow_smem_bytes(const Geom& g) {
+inline size_t score_narrow_smem_bytes(const Geom& gk) {
   return sizeof(float) * (static_cast<size_t>(D) * kNarrowRows + kNarrowStages * kNarrowSlice * kNarrowKeys) +
-         sizeof(uint32_t) * static_cast<size_t>(kNarrowRows) * g.nT;
+         sizeof(uint32_t) * static_cast<size_t>(kNarrowRows) * gk.nT;
 }
 
 }  // namespace vsa

@@ -22,7 +22,46 @@ struct Geom {
   int lg_tt, lg_th, lg_tw;  // log2 of the (power-of-two) tile extents
   int vol;                  // tt * th * tw
   int f16;                  // element type: 0 bfloat16, 1 float16
+  int layout;               // 0: [B, H, N, d]; 1: [B, N, H, d]
 };
+
+// A query-side and a key/value-side Geom share B, H, d, f16 and layout; each
+// has its own grid, tile and tile count.
+
+// TMA coordinates (after the channel coordinate) of the box whose first token
+// is (t, y, x) of head bh.  The [B, H, N, d] view is (d, W, Hh, T, B*H); the
+// [B, N, H, d] view is (d, H, W, Hh, B*T) -- batch and time fold into one
+// dimension because a batch's stride is T times a frame's.
+struct BoxCoord {
+  int c1, c2, c3, c4;
+};
+
+__host__ __device__ inline BoxCoord box_coord(const Geom& g, int bh, int t, int y, int x) {
+  BoxCoord c;
+  if (g.layout == 1) {
+    const int b = bh / g.H;
+    c.c1 = bh - b * g.H;
+    c.c2 = x;
+    c.c3 = y;
+    c.c4 = b * g.T + t;
+  } else {
+    c.c1 = x;
+    c.c2 = y;
+    c.c3 = t;
+    c.c4 = bh;
+  }
+  return c;
+}
+
+// Element offset of token n of head bh (N = T * Hh * W tokens per head).
+__host__ __device__ inline size_t token_offset(const Geom& g, int bh, size_t n) {
+  const size_t N = static_cast<size_t>(g.T) * g.Hh * g.W;
+  if (g.layout == 1) {
+    const int b = bh / g.H;
+    return ((static_cast<size_t>(b) * N + n) * g.H + (bh - b * g.H)) * g.d;
+  }
+  return (static_cast<size_t>(bh) * N + n) * g.d;
+}
 
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 

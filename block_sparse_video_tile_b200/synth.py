@@ -79,35 +79,38 @@ def _field_head(freq: np.ndarray, phase: np.ndarray, grid: tuple) -> np.ndarray:
 
 
 def make_qkv(B: int, H: int, grid: tuple, d: int, seed: int = 0,
-             kind: str = "normal", dtype: str = "bf16"):
-    """Return (q, k, v) as uint16 arrays of shape [B, H, N, d] holding bfloat16
-    bit patterns (dtype "bf16") or IEEE half-precision ones ("f16").
+             kind: str = "normal", dtype: str = "bf16", grid_k: tuple | None = None):
+    """Return (q, k, v) as uint16 arrays holding bfloat16 bit patterns (dtype
+    "bf16") or IEEE half-precision ones ("f16"): q [B, H, Nq, d] over ``grid``,
+    k and v [B, H, Nk, d] over ``grid_k`` (default: the same grid).
 
     Values are drawn head by head in (b, h) order within each tensor; a
     Generator fills consecutive draws from one stream, so this equals drawing
-    each whole tensor at once.
+    each whole tensor at once.  For structured inputs K's field is the same
+    function of the normalised coordinates (t/T, y/Hh, x/W), sampled on its
+    own grid.
     """
-    T, Hh, W = grid
-    N = T * Hh * W
+    grids = (grid, grid_k or grid, grid_k or grid)
+    Ns = [g[0] * g[1] * g[2] for g in grids]
     rng = np.random.Generator(np.random.PCG64(seed))
-    out = [np.empty((B, H, N, d), dtype=np.uint16) for _ in range(3)]
+    out = [np.empty((B, H, N, d), dtype=np.uint16) for N in Ns]
     to_bits = f32_to_f16_bits if dtype == "f16" else f32_to_bf16_bits
     if kind == "normal":
-        for x in out:
+        for x, N in zip(out, Ns):
             for b in range(B):
                 for h in range(H):
                     x[b, h] = to_bits(rng.standard_normal((N, d), dtype=np.float32))
         return tuple(out)
     if kind == "field":
         freq, phase = _field_params(rng, B, H, d)
-        for x in out[:2]:                  # the field is recomputed for K (same values)
+        for x, g, N in zip(out[:2], grids[:2], Ns[:2]):   # the field is recomputed for K
             for b in range(B):
                 for h in range(H):
-                    fld = _field_head(freq[b, h], phase[b, h], grid)
+                    fld = _field_head(freq[b, h], phase[b, h], g)
                     noise = rng.standard_normal((N, d), dtype=np.float32)
                     x[b, h] = to_bits(fld + np.float32(0.5) * noise)
         for b in range(B):
             for h in range(H):
-                out[2][b, h] = to_bits(rng.standard_normal((N, d), dtype=np.float32))
+                out[2][b, h] = to_bits(rng.standard_normal((Ns[2], d), dtype=np.float32))
         return tuple(out)
     raise ValueError(f"unknown input kind {kind!r}")

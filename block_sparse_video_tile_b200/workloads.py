@@ -34,11 +34,22 @@ class Workload:
     topk: int
     kind: str = "normal"
     dtype: str = "bf16"        # element type of Q, K, V, O: "bf16" or "f16"
+    layout: str = "bhnd"       # "bhnd" = [B, H, N, d] or "bnhd" = [B, N, H, d]
+    grid_k: tuple | None = None   # key/value grid (None: the query grid)
+    tile_k: tuple | None = None   # key/value tile (None: the query tile)
 
     @property
     def N(self) -> int:
         T, Hh, W = self.grid
         return T * Hh * W
+
+    @property
+    def kv_grid(self) -> tuple:
+        return self.grid if self.grid_k is None else self.grid_k
+
+    @property
+    def kv_tile(self) -> tuple:
+        return self.tile if self.tile_k is None else self.tile_k
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)

@@ -13,25 +13,39 @@
  *
  * Conventions shared by every call
  * --------------------------------
- * Tensors are dense, row-major, on the current CUDA device:
- *   Q, K, V, O : bfloat16 or float16 (vsa_shape.dtype) [B, H, N, d],
- *                N = T*Hh*W, token n = (t*Hh + y)*W + x
- *                (raster order over the grid; no permutation to tile order is
- *                 needed -- the kernels evaluate the tile index map themselves,
- *                 as the fastbsa page's "How it works" describes)
- *   idx        : int32 [B, H, nT, topk], kept key tiles of each query tile,
- *                strictly ascending, each in [0, nT)
- *   LSE        : float32 [B, H, N], natural log of the softmax denominator
- * Tiles: nT = ceil(T/tt) * ceil(Hh/th) * ceil(W/tw) (the user guide's routing
- * log: grid (31,22,40), tile (4,8,8) -> 120 tiles); edge tiles are partial and
- * their missing tokens are left out of pooling and of the softmax.  Tile
- * j = (bt * ceil(Hh/th) + by) * ceil(W/tw) + bx (raster over tile coordinates).
+ * Tensors are dense, row-major, on the current CUDA device, in one of two
+ * layouts (vsa_shape.layout):
+ *   VSA_LAYOUT_BHND  Q : [B, H, Nq, d]   K, V : [B, H, Nk, d]   O like Q
+ *   VSA_LAYOUT_BNHD  Q : [B, Nq, H, d]   K, V : [B, Nk, H, d]   O like Q
+ *                (the token-major layout a DiT's projections produce)
+ *   element type bfloat16 or float16 (vsa_shape.dtype); Nq = T*Hh*W over the
+ *   query grid, Nk = Tk*Hk*Wk over the key/value grid; token n = (t*Hh + y)*W
+ *   + x (raster order over its grid; no permutation to tile order is needed
+ *   -- the kernels evaluate the tile index map themselves, as the fastbsa
+ *   page's "How it works" describes)
+ *   idx        : int32 [B, H, nTq, topk], kept key/value tiles of each query
+ *                tile, strictly ascending, each in [0, nTk)
+ *   LSE        : float32 [B, H, Nq] in both layouts, natural log of the
+ *                softmax denominator
+ *
+ * Query and key/value grids (fastbsa page, "Use": separate latent and chunk
+ * shapes for q and k): by default both sides use the query grid and tile
+ * (self-attention with equal lengths, the Wan route of the FastVideo guide).
+ * Setting Tk, Hk, Wk and/or tk, hk, wk gives the key/value side its own grid
+ * and tile; the two tiles must hold the same number of tokens.
+ *
+ * Tiles: nT = ceil(T/tt) * ceil(Hh/th) * ceil(W/tw) per side (the user
+ * guide's routing log: grid (31,22,40), tile (4,8,8) -> 120 tiles); edge tiles
+ * are partial and their missing tokens are left out of pooling and of the
+ * softmax.  Tile j = (bt * ceil(Hh/th) + by) * ceil(W/tw) + bx (raster over
+ * tile coordinates).
  *
  * Supported: bf16 or fp16 inputs (O has the input type; pooling, scores,
- * softmax and accumulation are float32); d in {64, 128}; tt, th, tw powers of two with tt*th*tw in
- * {64, 128, 256} (the guide's 4x4x4 = 64 and 4x8x8 = 256 blocks), and tt >= 2
- * when tt*th*tw = 256; H_q = H_kv; non-causal self-attention, no mask.
- * Inputs must be finite (NaN/Inf give unspecified results, never a fault).
+ * softmax and accumulation are float32); d in {64, 128}; tile extents powers
+ * of two with tt*th*tw in {64, 128, 256} (the guide's 4x4x4 = 64 and 4x8x8 =
+ * 256 blocks), the same on both sides, and tt >= 2 when it is 256; H_q =
+ * H_kv; non-causal attention, no mask.  Inputs must be finite (NaN/Inf give
+ * unspecified results, never a fault).
  *
  * Ownership: the caller allocates every buffer (including the select
  * workspace); no call allocates device memory.  (The one piece of device
@@ -55,11 +69,14 @@ extern "C" {
 
 typedef struct vsa_shape {
   int32_t B, H;          /* batch, heads (query heads == key/value heads)     */
-  int32_t T, Hh, W;      /* post-patch latent grid                            */
+  int32_t T, Hh, W;      /* query post-patch latent grid                      */
   int32_t d;             /* head dimension: 64 or 128                         */
-  int32_t tt, th, tw;    /* tile extents along T, Hh, W                        */
+  int32_t tt, th, tw;    /* query tile extents along T, Hh, W                  */
   int32_t dtype;         /* element type of Q, K, V, O: VSA_DTYPE_BF16 (0, the
                             default of a zeroed struct) or VSA_DTYPE_F16      */
+  int32_t layout;        /* VSA_LAYOUT_BHND (0, default) or VSA_LAYOUT_BNHD   */
+  int32_t Tk, Hk, Wk;    /* key/value grid; all 0 (default): the query grid   */
+  int32_t tk, hk, wk;    /* key/value tile; all 0 (default): the query tile   */
 } vsa_shape;
 
 /* Element types (FastVideo VSA guide, "Verify routing and fallback": the
@@ -67,37 +84,53 @@ typedef struct vsa_shape {
 #define VSA_DTYPE_BF16 0
 #define VSA_DTYPE_F16 1
 
+/* Memory layouts of Q, K, V and O (see the conventions above). */
+#define VSA_LAYOUT_BHND 0
+#define VSA_LAYOUT_BNHD 1
+
 typedef enum vsa_status {
   VSA_OK = 0,
   VSA_ERR_INVALID_ARG = 1,  /* NULL pointer, non-positive extent, bad scale    */
-  VSA_ERR_TOPK_RANGE = 2,   /* topk <= 0 or topk > nT (guide: topk must be
-                               positive; topk > num_blocks is invalid)         */
-  VSA_ERR_UNSUPPORTED = 3,  /* d, dtype or tile shape outside the supported set */
+  VSA_ERR_TOPK_RANGE = 2,   /* topk <= 0 or topk > nTk (guide: topk must be
+                               positive; topk > num_blocks is invalid), or a
+                               sparsity outside [0, 1)                          */
+  VSA_ERR_UNSUPPORTED = 3,  /* d, dtype, layout or tile shape outside the
+                               supported set (incl. unequal tile volumes)       */
   VSA_ERR_ALIGNMENT = 4,    /* a tensor pointer not 16-byte aligned            */
   VSA_ERR_WORKSPACE = 5,    /* workspace NULL or smaller than required         */
   VSA_ERR_ARCH = 6,         /* current device is not sm_100                    */
   VSA_ERR_CUDA = 7,         /* a CUDA runtime/driver call failed               */
-  VSA_ERR_TOO_LARGE = 8     /* more than 1536 tiles per head, B*H > 65535, or
+  VSA_ERR_TOO_LARGE = 8     /* more than 1536 tiles per head on a side, B*H > 65535, or
                                (64-token tiles) topk too large for shared memory */
 } vsa_status;
 
-/* Tile count of a shape (FastVideo VSA guide, "Wan top-k behavior": num_blocks).
- * num_tiles: out, nT.  tiles_per_axis: out [3] (ceil per axis) or NULL.
- * Host only; touches no device. */
+/* Query tile count of a shape (FastVideo VSA guide, "Wan top-k behavior":
+ * num_blocks).  num_tiles: out, nTq.  tiles_per_axis: out [3] (ceil per
+ * axis) or NULL.  Host only; touches no device. */
 int vsa_tile_count(const vsa_shape* shape, int32_t* num_tiles, int32_t* tiles_per_axis);
 
-/* Bytes of device workspace vsa_select needs for `shape`: the pooled Q and K
- * tile means, float32 [2, B, H, d, ldT] with ldT = nT rounded up to a
- * multiple of 4 (channel-major, so the score kernel reads contiguous tile
- * rows).  Returns 0 for an invalid shape. */
+/* Key/value tile count nTk (equal to nTq unless the shape gives the key/value
+ * side its own grid or tile).  Same arguments as vsa_tile_count. */
+int vsa_kv_tile_count(const vsa_shape* shape, int32_t* num_tiles, int32_t* tiles_per_axis);
+
+/* Kept tiles per query tile for a sparsity (fastbsa page, "Use": sparsity =
+ * the fraction of key/value tiles left out, 0.9375 keeping 45 of 720):
+ * topk = round((1 - sparsity) * nTk) (halves round up), clamped to [1, nTk].
+ * sparsity must lie in [0, 1).  Host only. */
+int vsa_topk_from_sparsity(const vsa_shape* shape, float sparsity, int32_t* topk);
+
+/* Bytes of device workspace vsa_select needs for `shape`: the pooled tile
+ * means, float32, channel-major so the score kernel reads contiguous tile
+ * rows: Q means [B*H, d, ldq] then K means [B*H, d, ldk], ldq and ldk = nTq
+ * and nTk rounded up to a multiple of 4.  Returns 0 for an invalid shape. */
 size_t vsa_select_workspace_bytes(const vsa_shape* shape);
 
 /* Tile selection (FastVideo VSA guide intro and "Wan top-k behavior"; fastbsa
  * page "How it works": selection kept on chip, no score matrix in HBM).
- *   q, k      : device [B, H, N, d] of shape->dtype, 16-byte aligned
- *   topk      : kept key tiles per query tile, 1 <= topk <= nT
- *               (topk == nT keeps every tile: the dense case)
- *   idx_out   : device int32 [B, H, nT, topk]; row i gets the topk tiles j with
+ *   q, k      : device Q and K in shape->layout and shape->dtype, 16-byte aligned
+ *   topk      : kept key tiles per query tile, 1 <= topk <= nTk
+ *               (topk == nTk keeps every tile: the dense case)
+ *   idx_out   : device int32 [B, H, nTq, topk]; row i gets the topk tiles j with
  *               the largest s_ij = mean_i(Q) . mean_j(K) (float32 means over the
  *               tile's valid tokens, float32 dot), ties to the lower j, written
  *               in ascending j order
@@ -136,13 +169,14 @@ int vsa_select_noalloc(const vsa_shape* shape, const void* q, const void* k, int
 /* Block-sparse attention forward (FastVideo VSA guide intro: attention only
  * against the selected top-k blocks; "Verify routing and fallback": scale
  * head_size ** -0.5 by default, non-causal, no mask).
- *   q, k, v       : device [B, H, N, d] of shape->dtype, 16-byte aligned
- *   idx           : device int32 [B, H, nT, topk], ascending distinct tiles
- *                   (as vsa_select writes them); an entry outside [0, nT)
+ *   q, k, v       : device Q, K, V in shape->layout and shape->dtype, 16-byte
+ *                   aligned
+ *   idx           : device int32 [B, H, nTq, topk], ascending distinct tiles
+ *                   (as vsa_select writes them); an entry outside [0, nTk)
  *                   raises a device error and is read as tile 0 instead
  *   softmax_scale : > 0 and finite; pass d ** -0.5 for the standard scale
- *   o             : device [B, H, N, d] out, same type as q, 16-byte aligned
- *   lse           : device float32 [B, H, N] out, natural log
+ *   o             : device O out, layout and type of q, 16-byte aligned
+ *   lse           : device float32 [B, H, Nq] out, natural log
  * For every token n of query tile i: O[n] = softmax_m(scale * Q[n].K[m]) V[m]
  * over the valid tokens m of the tiles idx[i, :]; LSE[n] = log of the
  * denominator.  One kernel launch on `stream`. */
@@ -157,7 +191,7 @@ int vsa_device_error(uint32_t* code, int32_t reset);
 
 #define VSA_DEVERR_NONE 0u
 #define VSA_DEVERR_WAIT_TIMEOUT 1u   /* an mbarrier wait ran past its bound     */
-#define VSA_DEVERR_BAD_INDEX 2u      /* idx entry outside [0, nT)              */
+#define VSA_DEVERR_BAD_INDEX 2u      /* idx entry outside [0, nTk)             */
 
 /* Human-readable name of a vsa_status value.  Never NULL. */
 const char* vsa_status_string(int32_t status);

@@ -32,6 +32,14 @@ What it computes, and where the pages fix each step:
 5. Dense reference (fastbsa page, "How it works": outputs are validated
    against dense attention): plain softmax attention over all N tokens, with no
    tiles at all.  With topk == num_blocks (all blocks kept) step 4 equals it.
+6. Separate key/value grid (fastbsa page, "Use": latent_shape_q /
+   latent_shape_k and chunk_3d_shape_q / chunk_3d_shape_k): the query tokens
+   are tiled with the query grid and chunk, the key/value tokens with their
+   own; steps 2-4 then run with query tiles on one side and key/value tiles on
+   the other (scores nTq x nTk, top-k over nTk).
+7. Sparsity (fastbsa page, "Use": sparsity=0.9375): the fraction of key/value
+   blocks left out.  Reading: topk = round((1 - sparsity) * nTk), halves
+   rounding up, clamped to [1, nTk] (0.9375 of 720 blocks keeps 45).
 """
 from __future__ import annotations
 
@@ -125,29 +133,46 @@ def tie_gap(s_row: np.ndarray, topk: int):
     return abs(a - b) / denom, NEAR_TIE_REL * denom
 
 
-def select_head(Q: np.ndarray, K: np.ndarray, grid, tile, topk: int):
-    """One head: (idx [nT, topk] int32 ascending, scores [nT, nT], near_tie [nT] bool)."""
-    nT = num_tiles(grid, tile)
-    if not 0 < topk <= nT:
-        raise ValueError(f"topk must be in [1, {nT}], got {topk}")
-    s = tile_scores(pool(Q, grid, tile), pool(K, grid, tile))
-    idx = np.stack([topk_row(s[i], topk) for i in range(nT)]).astype(np.int32)
-    near = np.array([tie_gap(s[i], topk)[0] < NEAR_TIE_REL for i in range(nT)])
+def select_head(Q: np.ndarray, K: np.ndarray, grid, tile, topk: int, grid_k=None, tile_k=None):
+    """One head: (idx [nTq, topk] int32 ascending, scores [nTq, nTk], near_tie [nTq] bool).
+
+    K is tiled with grid_k / tile_k (default: the query grid / tile).
+    """
+    grid_k = grid if grid_k is None else grid_k
+    tile_k = tile if tile_k is None else tile_k
+    nTq, nTk = num_tiles(grid, tile), num_tiles(grid_k, tile_k)
+    if not 0 < topk <= nTk:
+        raise ValueError(f"topk must be in [1, {nTk}], got {topk}")
+    s = tile_scores(pool(Q, grid, tile), pool(K, grid_k, tile_k))
+    idx = np.stack([topk_row(s[i], topk) for i in range(nTq)]).astype(np.int32)
+    near = np.array([tie_gap(s[i], topk)[0] < NEAR_TIE_REL for i in range(nTq)])
     return idx, s, near
 
 
-def select(q_bits, k_bits, grid, tile, topk: int, dtype: str = "bf16"):
-    """All (b, h): idx [B, H, nT, topk], scores [B, H, nT, nT], near_tie [B, H, nT]."""
+def select(q_bits, k_bits, grid, tile, topk: int, dtype: str = "bf16", grid_k=None, tile_k=None):
+    """All (b, h): idx [B, H, nTq, topk], scores [B, H, nTq, nTk], near_tie [B, H, nTq].
+
+    q_bits [B, H, Nq, d] and k_bits [B, H, Nk, d] hold 16-bit patterns.
+    """
     B, H = q_bits.shape[:2]
-    nT = num_tiles(grid, tile)
-    idx = np.empty((B, H, nT, topk), np.int32)
-    sc = np.empty((B, H, nT, nT), np.float64)
-    near = np.empty((B, H, nT), bool)
+    nTq = num_tiles(grid, tile)
+    nTk = num_tiles(grid if grid_k is None else grid_k, tile if tile_k is None else tile_k)
+    idx = np.empty((B, H, nTq, topk), np.int32)
+    sc = np.empty((B, H, nTq, nTk), np.float64)
+    near = np.empty((B, H, nTq), bool)
     for b in range(B):
         for h in range(H):
             idx[b, h], sc[b, h], near[b, h] = select_head(
-                widen(q_bits[b, h], dtype), widen(k_bits[b, h], dtype), grid, tile, topk)
+                widen(q_bits[b, h], dtype), widen(k_bits[b, h], dtype), grid, tile, topk, grid_k, tile_k)
     return idx, sc, near
+
+
+def topk_from_sparsity(n_kv_tiles: int, sparsity: float) -> int:
+    """Kept blocks per query block for a sparsity in [0, 1): round((1 - s) * n), halves up, in [1, n]."""
+    if not 0.0 <= sparsity < 1.0:
+        raise ValueError(f"sparsity must be in [0, 1), got {sparsity}")
+    k = math.floor((1.0 - sparsity) * n_kv_tiles + 0.5)
+    return int(min(max(k, 1), n_kv_tiles))
 
 
 def selection_is_valid(gpu_row: np.ndarray, s_row: np.ndarray, topk: int) -> bool:
@@ -174,21 +199,23 @@ def selection_is_valid(gpu_row: np.ndarray, s_row: np.ndarray, topk: int) -> boo
 
 
 # ------------------------------------------------------------------ attention
-def attend_head(Q, K, V, grid, tile, idx, scale: float, query_tiles=None):
+def attend_head(Q, K, V, grid, tile, idx, scale: float, query_tiles=None, grid_k=None, tile_k=None):
     """Block-sparse exact attention for one head.
 
-    Q, K, V: [N, d] float64.  idx: [nT, topk] kept blocks per query block.
-    Returns O [N, d] and LSE [N]; rows of query blocks not in ``query_tiles``
-    (default: all) are NaN.
+    Q: [Nq, d], K, V: [Nk, d] float64 (K and V tiled with grid_k / tile_k,
+    default the query's).  idx: [nTq, topk] kept key/value blocks per query
+    block.  Returns O [Nq, d] and LSE [Nq]; rows of query blocks not in
+    ``query_tiles`` (default: all) are NaN.
     """
     toks = tile_tokens(grid, tile)
+    ktoks = tile_tokens(grid if grid_k is None else grid_k, tile if tile_k is None else tile_k)
     N, d = Q.shape
     O = np.full((N, V.shape[1]), np.nan)
     L = np.full(N, np.nan)
     tiles = range(len(toks)) if query_tiles is None else query_tiles
     for i in tiles:
         rows = toks[i]
-        keys = np.concatenate([toks[j] for j in idx[i]])
+        keys = np.concatenate([ktoks[j] for j in idx[i]])
         z = scale * (Q[rows] @ K[keys].T)
         m = z.max(axis=1, keepdims=True)
         e = np.exp(z - m)

@@ -29,27 +29,41 @@ _CACHE = {}
 
 
 def inputs(w, seed=0):
-    """((q, k, v) host bf16 bits, (q, k, v) device bf16); the last two input
-    sets are kept so that tests on the same workload do not redraw them."""
-    key = (w.B, w.H, w.grid, w.d, w.kind, seed, w.dtype)
+    """((q, k, v) host 16-bit patterns [B, H, N, d], (q, k, v) device tensors
+    in the workload's layout); the last two input sets are kept so that tests
+    on the same workload do not redraw them."""
+    key = (w.B, w.H, w.grid, w.grid_k, w.d, w.kind, seed, w.dtype)
     if key not in _CACHE:
         if len(_CACHE) >= 2:
             _CACHE.pop(next(iter(_CACHE)))
-        _CACHE[key] = synth.make_qkv(w.B, w.H, w.grid, w.d, seed=seed, kind=w.kind, dtype=w.dtype)
+        _CACHE[key] = synth.make_qkv(w.B, w.H, w.grid, w.d, seed=seed, kind=w.kind, dtype=w.dtype,
+                                     grid_k=w.grid_k)
     q, k, v = _CACHE[key]
-    return (q, k, v), tuple(to_dev(x, w.dtype) for x in (q, k, v))
+    dev = [to_dev(x, w.dtype) for x in (q, k, v)]
+    if w.layout == "bnhd":
+        dev = [x.permute(0, 2, 1, 3).contiguous() for x in dev]
+    return (q, k, v), tuple(dev)
+
+
+def geo(w) -> dict:
+    """Keyword arguments of api.select / attn_fwd for the workload's key/value grid and layout."""
+    return dict(grid_k=w.grid_k, tile_k=w.tile_k, layout=w.layout)
+
+
+def to_bhnd(x: torch.Tensor, w) -> torch.Tensor:
+    """A device output in the workload's layout, as [B, H, N, ...]."""
+    return x.permute(0, 2, 1, 3) if w.layout == "bnhd" else x
 
 
 def oracle_scores(q, k, w):
-    """float64 tile scores [B, H, nT, nT] straight from the oracle's steps."""
+    """float64 tile scores [B, H, nTq, nTk] straight from the oracle's steps."""
     B, H = q.shape[:2]
     out = []
     for b in range(B):
         for h in range(H):
             Q, K = vo.widen(q[b, h], w.dtype), vo.widen(k[b, h], w.dtype)
-            out.append(vo.tile_scores(vo.pool(Q, w.grid, w.tile), vo.pool(K, w.grid, w.tile)))
-    nT = out[0].shape[0]
-    return np.stack(out).reshape(B, H, nT, nT)
+            out.append(vo.tile_scores(vo.pool(Q, w.grid, w.tile), vo.pool(K, w.kv_grid, w.kv_tile)))
+    return np.stack(out).reshape(B, H, *out[0].shape)
 
 
 def check_selection(gidx: np.ndarray, scores: np.ndarray, topk: int):
@@ -74,7 +88,7 @@ def check_attention(o_gpu, lse_gpu, q, k, v, w, idx, scale, tiles=None):
     (all of them when ``tiles`` is None).  Returns (max_abs, mean_abs, lse_abs)."""
     B, H = q.shape[:2]
     toks = vo.tile_tokens(w.grid, w.tile)
-    o_gpu = o_gpu.float().cpu().numpy()
+    o_gpu = to_bhnd(o_gpu, w).float().cpu().numpy()
     lse_gpu = lse_gpu.cpu().numpy()
     errs, lerrs = [], []
     by_head = {}
@@ -84,7 +98,8 @@ def check_attention(o_gpu, lse_gpu, q, k, v, w, idx, scale, tiles=None):
         by_head.setdefault((b, h), []).append(i)
     for (b, h), ts in by_head.items():
         Q, K, V = (vo.widen(x[b, h], w.dtype) for x in (q, k, v))
-        O, L = vo.attend_head(Q, K, V, w.grid, w.tile, idx[b, h], scale, query_tiles=ts)
+        O, L = vo.attend_head(Q, K, V, w.grid, w.tile, idx[b, h], scale, query_tiles=ts,
+                              grid_k=w.kv_grid, tile_k=w.kv_tile)
         rows = np.concatenate([toks[i] for i in ts])
         errs.append(np.abs(o_gpu[b, h][rows] - O[rows]))
         lerrs.append(np.abs(lse_gpu[b, h][rows] - L[rows]))

@@ -56,7 +56,10 @@ def test_tile_count_matches_oracle(name):
 @pytest.mark.parametrize("kw,status", [
     (dict(d=96), 3), (dict(d=0), 1), (dict(tile=(3, 8, 8)), 3), (dict(tile=(1, 16, 16)), 3),
     (dict(tile=(4, 8, 16)), 3), (dict(grid=(0, 22, 40)), 1), (dict(tile=(8, 8, 8)), 3),
-    (dict(dtype=torch.float32), 3),
+    (dict(dtype=torch.float32), 3), (dict(layout="bhdn"), 3),
+    # key/value side: its own tile must hold as many tokens; a partial grid is invalid
+    (dict(tile_k=(4, 4, 4)), 3), (dict(tile_k=(2, 8, 8)), 3), (dict(grid_k=(31, 0, 40)), 1),
+    (dict(grid_k=(31, 22, 40), tile_k=(1, 16, 16)), 3),
 ])
 def test_unsupported_shapes(kw, status):
     args = dict(B=1, H=1, grid=(31, 22, 40), d=128, tile=(4, 8, 8))
@@ -129,3 +132,43 @@ def test_f16_shape_accepted():
     assert shp.dtype == _native.DTYPE_F16
     n = ctypes.c_int32()
     assert _native.lib().vsa_tile_count(ctypes.byref(shp), ctypes.byref(n), None) == 0 and n.value == 120
+
+
+def test_kv_tile_count_and_workspace():
+    # query: (31, 22, 40) / 4x8x8 -> 120 tiles; keys: (12, 48, 80) / 2x8x16 -> 6 * 6 * 5 = 180
+    shp = api.make_shape(2, 3, (31, 22, 40), 64, (4, 8, 8), grid_k=(12, 48, 80), tile_k=(2, 8, 16))
+    n, per = ctypes.c_int32(), (ctypes.c_int32 * 3)()
+    assert _native.lib().vsa_tile_count(ctypes.byref(shp), ctypes.byref(n), per) == 0 and n.value == 120
+    assert _native.lib().vsa_kv_tile_count(ctypes.byref(shp), ctypes.byref(n), per) == 0
+    assert (n.value, tuple(per)) == (vo.num_tiles((12, 48, 80), (2, 8, 16)), (6, 6, 5))
+    assert api.kv_tile_count((31, 22, 40), (4, 8, 8), (12, 48, 80), (2, 8, 16))[0] == 180
+    # means: Q [B*H, d, 120] and K [B*H, d, 180] in float32
+    assert api.select_workspace_bytes(2, 3, (31, 22, 40), 64, (4, 8, 8), (12, 48, 80), (2, 8, 16)) == \
+        4 * 6 * 64 * (120 + 180)
+    # without a key/value grid both sides are the query's
+    shp0 = api.make_shape(1, 1, (12, 48, 80), 128, (4, 4, 4))
+    assert _native.lib().vsa_kv_tile_count(ctypes.byref(shp0), ctypes.byref(n), None) == 0 and n.value == 720
+
+
+@pytest.mark.parametrize("sparsity", [0.0, 0.5, 0.85, 0.9, 0.9375, 0.99, 0.999])
+def test_topk_from_sparsity_matches_oracle(sparsity):
+    for grid, tile, grid_k, tile_k in (((12, 48, 80), (4, 4, 4), None, None),
+                                      ((31, 22, 40), (4, 8, 8), None, None),
+                                      ((8, 16, 16), (4, 4, 4), (10, 20, 30), (2, 4, 8))):
+        n = vo.num_tiles(grid_k or grid, tile_k or tile)
+        assert api.topk_from_sparsity(grid, tile, sparsity, grid_k, tile_k) == vo.topk_from_sparsity(n, sparsity)
+
+
+def test_topk_from_sparsity_range():
+    for bad in (1.0, -0.01, float("nan")):
+        with pytest.raises(_native.VsaError):
+            api.topk_from_sparsity((12, 48, 80), (4, 4, 4), bad)
+
+
+def test_bnhd_layout_and_kv_grid_accepted_on_host():
+    shp = api.make_shape(2, 4, (9, 20, 20), 128, (4, 8, 8), torch.float16, layout="bnhd",
+                         grid_k=(13, 16, 24), tile_k=(2, 8, 16))
+    n = ctypes.c_int32()
+    assert _native.lib().vsa_tile_count(ctypes.byref(shp), ctypes.byref(n), None) == 0 and n.value == 27
+    assert _native.lib().vsa_kv_tile_count(ctypes.byref(shp), ctypes.byref(n), None) == 0
+    assert n.value == vo.num_tiles((13, 16, 24), (2, 8, 16))

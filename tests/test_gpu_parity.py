@@ -41,7 +41,21 @@ SMALL = [
     Workload("f16_shared", 1, 2, (9, 20, 20), 128, (4, 8, 8), 5, dtype="f16"),
     Workload("f16_tile_d64", 2, 1, (6, 12, 20), 64, (2, 8, 8), 4, dtype="f16"),
     Workload("f16_pair", 1, 2, (6, 10, 14), 128, (4, 4, 4), 5, "field", dtype="f16"),
+    # [B, N, H, d] layout with B = 2 and a partial last t-tile, whose boxes read
+    # the next batch's first frames (masked), in each kernel mode
+    Workload("bnhd_shared", 2, 2, (9, 20, 20), 128, (4, 8, 8), 5, layout="bnhd"),
+    Workload("bnhd_tile", 2, 3, (6, 12, 20), 64, (4, 4, 8), 4, layout="bnhd"),
+    Workload("bnhd_pair", 2, 2, (6, 10, 14), 128, (4, 4, 4), 5, "field", layout="bnhd"),
+    # keys and values on their own grid (fastbsa page, "Use": latent_shape_k,
+    # chunk_3d_shape_k), with the same or another tile of equal volume
+    Workload("kv_grid_shared", 1, 2, (9, 20, 20), 128, (4, 8, 8), 6, grid_k=(13, 16, 24)),
+    Workload("kv_tile_shared", 1, 2, (9, 20, 20), 128, (4, 8, 8), 6, "field", grid_k=(10, 18, 30),
+             tile_k=(2, 8, 16)),
+    Workload("kv_pair", 1, 2, (6, 10, 14), 128, (4, 4, 4), 5, "field", grid_k=(7, 12, 9), tile_k=(2, 4, 8)),
+    Workload("kv_tile_bnhd", 2, 1, (6, 12, 20), 64, (2, 8, 8), 4, grid_k=(5, 9, 26), tile_k=(4, 4, 8),
+             layout="bnhd"),
 ]
+BY_NAME = {w.name: w for w in SMALL}
 
 
 def _seed(w):
@@ -52,43 +66,45 @@ def _seed(w):
 def test_small_full_compare(w):
     (q, k, v), (qd, kd, vd) = gu.inputs(w, seed=_seed(w))
     scale = w.d ** -0.5
-    idx = api.select(qd, kd, w.grid, w.tile, w.topk)
+    idx = api.select(qd, kd, w.grid, w.tile, w.topk, **gu.geo(w))
     torch.cuda.synchronize()
     gu.assert_no_device_error()
     scores = gu.oracle_scores(q, k, w)
     rows, ties = gu.check_selection(idx.cpu().numpy(), scores, w.topk)
     # attention on the GPU's own selection (so a tie row is still checked)
-    o, lse = api.attn_fwd(qd, kd, vd, idx, w.grid, w.tile, scale=scale)
+    o, lse = api.attn_fwd(qd, kd, vd, idx, w.grid, w.tile, scale=scale, **gu.geo(w))
     gu.assert_no_device_error()
     gu.check_attention(o, lse, q, k, v, w, idx.cpu().numpy(), scale)
 
 
-@pytest.mark.parametrize("w", [SMALL[2], SMALL[5], SMALL[7]], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [BY_NAME[n] for n in ("ragged256", "ragged64", "vol128", "kv_tile_shared",
+                                                     "kv_pair", "bnhd_tile")], ids=lambda w: w.name)
 def test_oracle_indices_attention(w):
-    """Attention alone, fed the oracle's selection and an arbitrary one."""
+    """Attention alone, fed an arbitrary selection."""
     (q, k, v), (qd, kd, vd) = gu.inputs(w, seed=3)
-    nT = vo.num_tiles(w.grid, w.tile)
+    nT, nTk = vo.num_tiles(w.grid, w.tile), vo.num_tiles(w.kv_grid, w.kv_tile)
     rng = np.random.default_rng(5)
-    idx = np.sort(np.stack([[rng.choice(nT, w.topk, replace=False) for _ in range(nT)]
+    idx = np.sort(np.stack([[rng.choice(nTk, w.topk, replace=False) for _ in range(nT)]
                             for _ in range(w.B * w.H)]), axis=-1).reshape(w.B, w.H, nT, w.topk)
     idx = idx.astype(np.int32)
-    o, lse = api.attn_fwd(qd, kd, vd, torch.from_numpy(idx).cuda(), w.grid, w.tile, scale=0.3)
+    o, lse = api.attn_fwd(qd, kd, vd, torch.from_numpy(idx).cuda(), w.grid, w.tile, scale=0.3, **gu.geo(w))
     gu.assert_no_device_error()
     gu.check_attention(o, lse, q, k, v, w, idx, 0.3)
 
 
-@pytest.mark.parametrize("w", [SMALL[2], SMALL[5], SMALL[3]], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [BY_NAME[n] for n in ("ragged256", "ragged64", "ragged256_d64", "kv_grid_shared",
+                                                     "kv_pair", "bnhd_shared")], ids=lambda w: w.name)
 def test_all_tiles_equal_dense(w):
     """topk == num_blocks keeps every tile: the result is dense attention
-    (FastVideo VSA user guide, "Wan top-k behavior")."""
+    (FastVideo VSA user guide, "Wan top-k behavior"), over all Nk keys."""
     (q, k, v), (qd, kd, vd) = gu.inputs(w, seed=4)
-    nT = vo.num_tiles(w.grid, w.tile)
-    idx = api.select(qd, kd, w.grid, w.tile, nT)
-    assert (idx.cpu().numpy() == np.arange(nT)).all()
+    nTk = vo.num_tiles(w.kv_grid, w.kv_tile)
+    idx = api.select(qd, kd, w.grid, w.tile, nTk, **gu.geo(w))
+    assert (idx.cpu().numpy() == np.arange(nTk)).all()
     scale = w.d ** -0.5
-    o, lse = api.attn_fwd(qd, kd, vd, idx, w.grid, w.tile, scale=scale)
+    o, lse = api.attn_fwd(qd, kd, vd, idx, w.grid, w.tile, scale=scale, **gu.geo(w))
     gu.assert_no_device_error()
-    og, lg = o.float().cpu().numpy(), lse.cpu().numpy()
+    og, lg = gu.to_bhnd(o, w).float().cpu().numpy(), lse.cpu().numpy()
     for b in range(w.B):
         for h in range(w.H):
             Od, Ld = vo.dense_bruteforce(*(vo.widen(x[b, h], w.dtype) for x in (q, k, v)), scale)
@@ -153,10 +169,10 @@ def _full_case(w, seed=0, topks=None):
     rng = np.random.default_rng(11)
     report = {}
     for topk in (topks or [w.topk]):
-        idx = api.select(qd, kd, w.grid, w.tile, topk)
+        idx = api.select(qd, kd, w.grid, w.tile, topk, **gu.geo(w))
         gi = idx.cpu().numpy()
         rows, ties = gu.check_selection(gi, scores, topk)
-        o, lse = api.attn_fwd(qd, kd, vd, idx, w.grid, w.tile)
+        o, lse = api.attn_fwd(qd, kd, vd, idx, w.grid, w.tile, **gu.geo(w))
         gu.assert_no_device_error()
         errs = gu.check_attention(o, lse, q, k, v, w, gi, w.d ** -0.5, tiles=_sample_tiles(w, rng))
         report[topk] = (rows, ties, errs)
@@ -167,6 +183,31 @@ def _full_case(w, seed=0, topks=None):
 def test_full_size(w):
     rep = _full_case(w)
     print(w.name, rep)
+
+
+# A LongCat-style call (fastbsa page, "Use"): [B, N, H, d] tensors, keys and
+# values over 4 more latent frames than the queries, 4x4x4 chunks on both
+# sides, sparsity 0.9375 (960 key tiles -> 60 kept); 8 of the 32 heads.
+LONGCAT_KV = LONGCAT.with_(name="longcat_kv_bnhd", H=8, layout="bnhd", grid_k=(16, 48, 80), topk=60)
+
+
+def test_longcat_style_call():
+    w = LONGCAT_KV
+    assert api.topk_from_sparsity(w.grid, w.tile, 0.9375, w.grid_k) == w.topk
+    rep = _full_case(w)
+    print(w.name, rep)
+
+
+def test_forward_with_sparsity():
+    w = BY_NAME["kv_pair"]
+    (q, k, v), (qd, kd, vd) = gu.inputs(w, seed=2)
+    nTk = vo.num_tiles(w.kv_grid, w.kv_tile)
+    topk = vo.topk_from_sparsity(nTk, 0.8)
+    o, lse, idx = api.forward(qd, kd, vd, w.grid, w.tile, sparsity=0.8, **gu.geo(w))
+    assert idx.shape[-1] == topk
+    o2, lse2, idx2 = api.forward(qd, kd, vd, w.grid, w.tile, topk, **gu.geo(w))
+    assert torch.equal(idx, idx2) and torch.equal(o, o2) and torch.equal(lse, lse2)
+    gu.check_selection(idx.cpu().numpy(), gu.oracle_scores(q, k, w), topk)
 
 
 # Heads of up to 768 tiles take the wide score kernel (768: its largest head),

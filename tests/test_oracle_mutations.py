@@ -52,6 +52,17 @@ def _floor_tiles(grid, tile):
     return [t for t in _orig_tokens(grid, tile) if t.size == tile[0] * tile[1] * tile[2]]
 
 
+_orig_select_head = vo.select_head
+
+
+def _select_kv_with_query_tile(Q, K, grid, tile, topk, grid_k=None, tile_k=None):
+    return _orig_select_head(Q, K, grid, tile, topk, grid_k, tile)
+
+
+def _attend_kv_with_query_tiles(Q, K, V, grid, tile, idx, scale, query_tiles=None, grid_k=None, tile_k=None):
+    return _orig_attend(Q, K, V, grid, tile, idx, scale, query_tiles)
+
+
 CASES = [
     ("pool", _zero_padded_pool, lambda: pins.test_pool_constant_per_block_partial_edges()),
     ("tile_scores", _transposed_scores, lambda: pins.test_scores_hand_example()),
@@ -62,6 +73,9 @@ CASES = [
     ("attend_head", _attend_log2_lse, lambda: pins.test_lse_normalises_weights()),
     ("tile_tokens", _floor_tiles, lambda: pins.test_block_token_counts(
         pins.WAN5B, {256: 70, 192: 45, 144: 5})),
+    ("select_head", _select_kv_with_query_tile, lambda: pins.test_kv_pool_uses_kv_tiles()),
+    ("attend_head", _attend_kv_with_query_tiles,
+     lambda: pins.test_kv_grid_all_blocks_equals_dense(*pins.KV_CASES[0])),
 ]
 
 

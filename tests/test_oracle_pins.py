@@ -308,3 +308,60 @@ def test_f16_widening_textbook_values():
     # 1 + 2^-11 lies halfway between 1 and 1 + 2^-10: ties round to the even one (1.0)
     assert synth.f32_to_f16_bits(np.array([1 + 2 ** -11], np.float32))[0] == 0x3C00
     assert synth.f32_to_f16_bits(np.array([1 + 3 * 2 ** -11], np.float32))[0] == 0x3C02
+
+
+# ------------------------------------- separate key/value grid, sparsity (fastbsa page, "Use")
+KV_CASES = [
+    # (query grid, query tile, key/value grid, key/value tile); partial edge tiles on both sides
+    ((3, 5, 6), (2, 2, 2), (5, 4, 7), (2, 2, 2)),
+    ((4, 4, 4), (2, 2, 2), (6, 3, 5), (4, 2, 1)),
+]
+
+
+@pytest.mark.parametrize("grid_q,tile_q,grid_k,tile_k", KV_CASES)
+def test_kv_grid_all_blocks_equals_dense(grid_q, tile_q, grid_k, tile_k):
+    # keeping every key/value block is dense attention of the Nq queries over
+    # all Nk keys, whatever the two tilings (closed form, no tiles in the reference)
+    Nq, Nk, d = math.prod(grid_q), math.prod(grid_k), 8
+    Q, K, V = _rand((Nq, d), 21), _rand((Nk, d), 22), _rand((Nk, d), 23)
+    nTq, nTk = vo.num_tiles(grid_q, tile_q), vo.num_tiles(grid_k, tile_k)
+    idx, s, _ = vo.select_head(Q, K, grid_q, tile_q, nTk, grid_k, tile_k)
+    assert s.shape == (nTq, nTk)
+    assert (idx == np.arange(nTk)).all()
+    O, L = vo.attend_head(Q, K, V, grid_q, tile_q, idx, 0.3, grid_k=grid_k, tile_k=tile_k)
+    Od, Ld = vo.dense_bruteforce(Q, K, V, 0.3)
+    np.testing.assert_allclose(O, Od, atol=1e-12)
+    np.testing.assert_allclose(L, Ld, atol=1e-12)
+
+
+def test_kv_pool_uses_kv_tiles():
+    # K constant on each of its own (partial-edged) tiles: its means are those constants
+    grid_q, tile_q, grid_k, tile_k = KV_CASES[1]
+    d = 6
+    rng = np.random.default_rng(5)
+    toks = vo.tile_tokens(grid_k, tile_k)
+    vals = rng.standard_normal((len(toks), d))
+    K = np.zeros((math.prod(grid_k), d))
+    for j, t in enumerate(toks):
+        K[t] = vals[j]
+    Q = _rand((math.prod(grid_q), d), 24)
+    _, s, _ = vo.select_head(Q, K, grid_q, tile_q, 1, grid_k, tile_k)
+    assert s.shape == (vo.num_tiles(grid_q, tile_q), len(toks))
+    np.testing.assert_allclose(s, vo.pool(Q, grid_q, tile_q) @ vals.T, atol=1e-12)
+
+
+def test_topk_from_sparsity():
+    # fastbsa page, "Use": sparsity=0.9375 keeps one block in 16
+    assert vo.topk_from_sparsity(720, 0.9375) == 45
+    assert vo.topk_from_sparsity(16, 0.9375) == 1
+    # exact keep fractions need no rounding
+    for n, k in ((120, 64), (300, 30), (720, 45), (8, 2), (1536, 1536)):
+        assert vo.topk_from_sparsity(n, 1.0 - k / n) == k
+    for n in (1, 7, 120):
+        assert vo.topk_from_sparsity(n, 0.0) == n
+    # reading: halves round up, and at least one block is kept
+    assert vo.topk_from_sparsity(10, 0.85) == 2
+    assert vo.topk_from_sparsity(10, 0.99) == 1
+    for bad in (1.0, -0.1, 1.5):
+        with pytest.raises(ValueError):
+            vo.topk_from_sparsity(10, bad)
