@@ -43,7 +43,7 @@ namespace vsa {
 
 constexpr int kAttnThreads = 384;        // 3 warpgroups
 constexpr int kSoftmaxRegs = 208;        // per thread, warpgroups 0-1 (after setmaxnreg)
-constexpr int kProducerRegs = 80;        // per thread, warpgroup 2 (TMA + MMA warps)
+constexpr int kProducerRegs = 88;        // per thread, warpgroup 2 (TMA + MMA warps)
 constexpr int kSlotRows = 128;          // MMA M
 constexpr int kSubRows = 128;           // K/V rows per sub-block (S: N, PV: K)
 constexpr float kRescaleLog2 = 8.0f;
@@ -111,10 +111,23 @@ struct Slot {
   int tb0, yb0, xb0;     // MODE_PAIR: origin of tile B
 };
 
+// The key/value side's geometry and box t-extent.  SAME: the key/value side
+// uses the query grid and tile, known at compile time, so the kernel reads
+// one set of parameters (fewer live registers in the softmax warps).
+template <bool SAME>
+__device__ __forceinline__ const Geom& kv_geom(const AttnArgs& a) {
+  return SAME ? a.gq : a.gk;
+}
+template <bool SAME>
+__device__ __forceinline__ int kv_box_t(const AttnArgs& a) {
+  return SAME ? a.box_tq : a.box_tk;
+}
+
+template <bool SAME>
 __device__ __forceinline__ int load_tile_index(const AttnArgs& a, const int32_t* row, int e,
                                                bool report) {
   int j = __ldg(row + e);
-  if (j < 0 || j >= a.gk.nT) {
+  if (j < 0 || j >= kv_geom<SAME>(a).nT) {
     if (report) atomicCAS(a.err, 0u, kErrBadIndex);
     j = 0;
   }
@@ -146,7 +159,7 @@ struct Piece {
 //   MODE_PAIR:   the ascending union of tile A's and tile B's kept lists (built
 //                in shared memory at kernel start), two tiles per sub-block (a
 //                short last sub-block is padded).
-template <int MODE>
+template <int MODE, bool SAME>
 struct KvSeq {
   const int32_t* row;     // kept list of the slot's (first) query tile
   const uint32_t* uni;    // MODE_PAIR: the slot's union list in shared memory
@@ -164,24 +177,24 @@ struct KvSeq {
     half = 0;
   }
   __device__ bool second_half(const AttnArgs& a, int j) const {
-    return static_cast<int>(tab[j].x) * a.gk.tt + a.box_tk < a.gk.T;
+    return static_cast<int>(tab[j].x) * kv_geom<SAME>(a).tt + kv_box_t<SAME>(a) < kv_geom<SAME>(a).T;
   }
   __device__ int count(const AttnArgs& a) const {
     if (MODE == MODE_TILE) return a.topk;
     if (MODE == MODE_PAIR) return (ulen + 1) / 2;
     int n = 0;
-    for (int e = 0; e < a.topk; ++e) n += 1 + (second_half(a, load_tile_index(a, row, e, false)) ? 1 : 0);
+    for (int e = 0; e < a.topk; ++e) n += 1 + (second_half(a, load_tile_index<SAME>(a, row, e, false)) ? 1 : 0);
     return n;
   }
   // Piece p (0 or 1) of the current sub-block.
   __device__ Piece piece(const AttnArgs& a, int p, bool report) const {
     Piece pc;
     if (MODE == MODE_SHARED) {
-      pc.j = load_tile_index(a, row, pos, report);
-      pc.toff = half * a.box_tk;
+      pc.j = load_tile_index<SAME>(a, row, pos, report);
+      pc.toff = half * kv_box_t<SAME>(a);
       pc.real = pc.in_a = pc.in_b = true;
     } else if (MODE == MODE_TILE) {
-      pc.j = load_tile_index(a, row, pos, report);
+      pc.j = load_tile_index<SAME>(a, row, pos, report);
       pc.toff = 0;
       pc.real = pc.in_a = pc.in_b = true;
     } else {
@@ -198,7 +211,7 @@ struct KvSeq {
   }
   __device__ void advance(const AttnArgs& a) {
     if (MODE == MODE_SHARED) {
-      if (half == 0 && second_half(a, load_tile_index(a, row, pos, false))) {
+      if (half == 0 && second_half(a, load_tile_index<SAME>(a, row, pos, false))) {
         half = 1;
       } else {
         half = 0;
@@ -214,20 +227,21 @@ struct KvSeq {
 // kept lists, then the set tiles in ascending order with per-list flags
 // (prefix counts across the warp give each tile its position).  Returns the
 // union length (valid in every lane).
+template <bool SAME>
 __device__ __forceinline__ int build_union(const AttnArgs& a, const int32_t* row_a, bool has_b, uint32_t* bm_a,
                                            uint32_t* bm_b, uint32_t* out) {
   const int lane = threadIdx.x % 32;
-  const int nw = (a.gk.nT + 31) / 32;
+  const int nw = (kv_geom<SAME>(a).nT + 31) / 32;
   for (int w = lane; w < nw; w += 32) {
     bm_a[w] = 0u;
     bm_b[w] = 0u;
   }
   __syncwarp();
   for (int e = lane; e < a.topk; e += 32) {
-    const int ja = load_tile_index(a, row_a, e, true);
+    const int ja = load_tile_index<SAME>(a, row_a, e, true);
     atomicOr(bm_a + (ja >> 5), 1u << (ja & 31));
     if (has_b) {
-      const int jb = load_tile_index(a, row_a + a.topk, e, true);
+      const int jb = load_tile_index<SAME>(a, row_a + a.topk, e, true);
       atomicOr(bm_b + (jb >> 5), 1u << (jb & 31));
     }
   }
@@ -256,7 +270,7 @@ __device__ __forceinline__ int build_union(const AttnArgs& a, const int32_t* row
   return base;
 }
 
-template <int D, int MODE, bool F16>
+template <int D, int MODE, bool F16, bool SAME, bool BNHD>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
@@ -273,12 +287,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sp + L::kMisc + 4);
   uint2* tile_tab = reinterpret_cast<uint2*>(sp + L::kTiles);
   int* union_len = reinterpret_cast<int*>(sp + L::kMisc + 8);          // [2]
-  uint32_t* bitmaps = reinterpret_cast<uint32_t*>(sp + L::bitmap_off(a.gk.nT));
-  uint32_t* unions = reinterpret_cast<uint32_t*>(sp + L::union_off(a.gk.nT));
+  uint32_t* bitmaps = reinterpret_cast<uint32_t*>(sp + L::bitmap_off(kv_geom<SAME>(a).nT));
+  uint32_t* unions = reinterpret_cast<uint32_t*>(sp + L::union_off(kv_geom<SAME>(a).nT));
   auto bar = [&](int id) -> uint32_t { return sBar + 8u * static_cast<uint32_t>(id); };
 
   const Geom& g = a.gq;                                     // query side
-  const Geom& gk = a.gk;                                    // key/value side
+  const Geom& gk = kv_geom<SAME>(a);                        // key/value side
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int box_rows = SHARED ? kSubRows : g.vol;          // rows per TMA box (equal volumes)
   const uint32_t box_bytes = static_cast<uint32_t>(box_rows) * 128u;
@@ -347,7 +361,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (sl.active) {
       const int32_t* row_a = a.idx + (static_cast<size_t>(sl.bh) * g.nT + sl.tile) * a.topk;
       const int nw = L::bitmap_words(gk.nT);
-      len = build_union(a, row_a, sl.has_b, bitmaps + 2 * h * nw, bitmaps + (2 * h + 1) * nw,
+      len = build_union<SAME>(a, row_a, sl.has_b, bitmaps + 2 * h * nw, bitmaps + (2 * h + 1) * nw,
                         unions + h * 2 * a.topk);
     }
     if (lane == 0) union_len[h] = len;
@@ -388,8 +402,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!slot[h].active) continue;
         const int nbox = (PAIR && slot[h].has_b) ? 2 : 1;
         mbar_arrive_expect_tx(bar(BAR_Q_FULL + h), static_cast<uint32_t>(nbox * L::kSlabs) * box_bytes);
-        const BoxCoord ca = box_coord(g, slot[h].bh, slot[h].t0, slot[h].y0, slot[h].x0);
-        const BoxCoord cb = box_coord(g, slot[h].bh, slot[h].tb0, slot[h].yb0, slot[h].xb0);
+        const BoxCoord ca = box_coord_l<BNHD>(g, slot[h].bh, slot[h].t0, slot[h].y0, slot[h].x0);
+        const BoxCoord cb = box_coord_l<BNHD>(g, slot[h].bh, slot[h].tb0, slot[h].yb0, slot[h].xb0);
         for (int sl = 0; sl < L::kSlabs; ++sl) {
           tma_load_5d(sQ + h * L::kBufBytes + sl * L::kSlabBytes, &tmQ, bar(BAR_Q_FULL + h), sl * 64, ca.c1,
                       ca.c2, ca.c3, ca.c4);
@@ -398,7 +412,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         sl * 64, cb.c1, cb.c2, cb.c3, cb.c4);
         }
       }
-      KvSeq<MODE> sq[2];
+      KvSeq<MODE, SAME> sq[2];
       int n[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -428,7 +442,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             for (int p = 0; p < P; ++p) {
               const Piece pc = sq[h].piece(a, p, kv == 0);
               const TileCoord c = table_coord(tile_tab, pc.j);
-              const BoxCoord bc = box_coord(gk, slot[h].bh, c.bt * gk.tt + pc.toff, c.by * gk.th, c.bx * gk.tw);
+              const BoxCoord bc =
+                  box_coord_l<BNHD>(gk, slot[h].bh, c.bt * gk.tt + pc.toff, c.by * gk.th, c.bx * gk.tw);
               for (int sl = 0; sl < L::kSlabs; ++sl)
                 tma_load_5d(buf0 + st * L::kBufBytes + sl * L::kSlabBytes + p * box_bytes, tm,
                             bar(full + st), sl * 64, bc.c1, bc.c2, bc.c3, bc.c4);
@@ -454,7 +469,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int n[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        KvSeq<MODE> sq;
+        KvSeq<MODE, SAME> sq;
         sq.init(a, tile_tab, slot[h].bh, slot[h].tile, unions + h * 2 * a.topk, union_len[h]);
         n[h] = slot[h].active ? sq.count(a) : 0;
       }
@@ -552,7 +567,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     lt < (SHARED ? a.box_tq : g.tt) && (!in_b || me.has_b);
       }
 
-      KvSeq<MODE> sq;
+      KvSeq<MODE, SAME> sq;
       sq.init(a, tile_tab, me.bh, me.tile, unions + h * 2 * a.topk, union_len[h]);
       const int n = sq.count(a);
       float m = -INFINITY, l = 0.f;
@@ -573,9 +588,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const TileCoord c = table_coord(tile_tab, pc.j);
             int et, ey, ex;
             tile_extent(gk, c, et, ey, ex);
-            const int vt = SHARED ? min(a.box_tk, et - pc.toff) : et;
+            const int vt = SHARED ? min(kv_box_t<SAME>(a), et - pc.toff) : et;
             const bool use = pc.real && (in_b ? pc.in_b : pc.in_a);
-            const bool gfull = vt == (SHARED ? a.box_tk : gk.tt) && ey == gk.th && ex == gk.tw;
+            const bool gfull = vt == (SHARED ? kv_box_t<SAME>(a) : gk.tt) && ey == gk.th && ex == gk.tw;
             geo_full = geo_full && (!use || gfull);
             if (p == 0) { vt0 = vt; vy0 = ey; vx0 = ex; use0 = use; }
             else        { vt1 = vt; vy1 = ey; vx1 = ex; use1 = use; }

@@ -53,6 +53,26 @@ __host__ __device__ inline BoxCoord box_coord(const Geom& g, int bh, int t, int 
   return c;
 }
 
+// The same with the layout fixed at compile time (kernels instantiated per
+// layout: no division or branch in their box-issuing loops).
+template <bool BNHD>
+__host__ __device__ inline BoxCoord box_coord_l(const Geom& g, int bh, int t, int y, int x) {
+  BoxCoord c;
+  if (BNHD) {
+    const int b = bh / g.H;
+    c.c1 = bh - b * g.H;
+    c.c2 = x;
+    c.c3 = y;
+    c.c4 = b * g.T + t;
+  } else {
+    c.c1 = x;
+    c.c2 = y;
+    c.c3 = t;
+    c.c4 = bh;
+  }
+  return c;
+}
+
 // Element offset of token n of head bh (N = T * Hh * W tokens per head).
 __host__ __device__ inline size_t token_offset(const Geom& g, int bh, size_t n) {
   const size_t N = static_cast<size_t>(g.T) * g.Hh * g.W;
