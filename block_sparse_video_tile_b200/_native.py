@@ -31,7 +31,7 @@ LAYOUT_BHND, LAYOUT_BNHD = 0, 1
 class VsaShape(ctypes.Structure):
     """vsa_shape: zero key/value fields mean "the query grid / tile"."""
     _fields_ = [(n, ctypes.c_int32) for n in ("B", "H", "T", "Hh", "W", "d", "tt", "th", "tw", "dtype", "layout",
-                                              "Tk", "Hk", "Wk", "tk", "hk", "wk")]
+                                              "Tk", "Hk", "Wk", "tk", "hk", "wk", "prefix_tiles")]
 
 
 class VsaError(RuntimeError):

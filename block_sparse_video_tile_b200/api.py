@@ -25,13 +25,13 @@ _LAYOUTS = {"bhnd": LAYOUT_BHND, "bnhd": LAYOUT_BNHD}
 
 
 def make_shape(B: int, H: int, grid, d: int, tile, dtype=torch.bfloat16, *, layout: str = "bhnd",
-               grid_k=None, tile_k=None) -> VsaShape:
+               grid_k=None, tile_k=None, prefix_tiles: int = 0) -> VsaShape:
     T, Hh, W = grid
     tt, th, tw = tile
     Tk, Hk, Wk = grid_k if grid_k is not None else (0, 0, 0)
     tk, hk, wk = tile_k if tile_k is not None else (0, 0, 0)
     return VsaShape(B, H, T, Hh, W, d, tt, th, tw, _DTYPES.get(dtype, -1), _LAYOUTS.get(layout, -1),
-                    Tk, Hk, Wk, tk, hk, wk)
+                    Tk, Hk, Wk, tk, hk, wk, prefix_tiles)
 
 
 def _count(fn, shp):
@@ -51,9 +51,11 @@ def kv_tile_count(grid, tile, grid_k=None, tile_k=None, d: int = 128, B: int = 1
     return _count("vsa_kv_tile_count", make_shape(B, H, grid, d, tile, grid_k=grid_k, tile_k=tile_k))
 
 
-def topk_from_sparsity(grid, tile, sparsity: float, grid_k=None, tile_k=None, d: int = 128) -> int:
-    """Kept key/value tiles per query tile for a sparsity: round((1 - sparsity) * nTk), in [1, nTk]."""
-    shp = make_shape(1, 1, grid, d, tile, grid_k=grid_k, tile_k=tile_k)
+def topk_from_sparsity(grid, tile, sparsity: float, grid_k=None, tile_k=None, d: int = 128,
+                       prefix_tiles: int = 0) -> int:
+    """Kept key/value tiles per query tile for a sparsity: round((1 - sparsity) * nTk), in
+    [max(1, prefix_tiles), nTk]."""
+    shp = make_shape(1, 1, grid, d, tile, grid_k=grid_k, tile_k=tile_k, prefix_tiles=prefix_tiles)
     k = ctypes.c_int32()
     check("vsa_topk_from_sparsity", lib().vsa_topk_from_sparsity(ctypes.byref(shp), float(sparsity),
                                                                   ctypes.byref(k)))
@@ -97,13 +99,15 @@ def _stream(stream) -> int:
 
 
 def select(q: torch.Tensor, k: torch.Tensor, grid, tile, topk: int, *, grid_k=None, tile_k=None,
-           layout: str = "bhnd", out=None, workspace=None, stream=None) -> torch.Tensor:
-    """Top-k key tiles per query tile: int32 [B, H, nTq, topk], ascending."""
+           layout: str = "bhnd", prefix_tiles: int = 0, out=None, workspace=None, stream=None) -> torch.Tensor:
+    """Top-k key tiles per query tile: int32 [B, H, nTq, topk], ascending; key/value
+    tiles 0 .. prefix_tiles-1 are in every row (and count toward topk)."""
     B, H, Nq, d = _dims(q, layout)
     Nk = _grid_tokens(grid_k if grid_k is not None else grid)
     _check_qkv("q", q, (B, H, _grid_tokens(grid), d), layout)
     _check_qkv("k", k, (B, H, Nk, d), layout, q.dtype)
-    shp = make_shape(B, H, grid, d, tile, q.dtype, layout=layout, grid_k=grid_k, tile_k=tile_k)
+    shp = make_shape(B, H, grid, d, tile, q.dtype, layout=layout, grid_k=grid_k, tile_k=tile_k,
+                     prefix_tiles=prefix_tiles)
     nT, _ = tile_count(grid, tile, d, B, H)
     if out is None:
         out = torch.empty((B, H, nT, topk), dtype=torch.int32, device=q.device)
@@ -143,15 +147,15 @@ def attn_fwd(q, k, v, idx, grid, tile, *, grid_k=None, tile_k=None, layout: str 
 
 
 def forward(q, k, v, grid, tile, topk: int | None = None, *, sparsity: float | None = None, grid_k=None,
-            tile_k=None, layout: str = "bhnd", scale=None, stream=None):
+            tile_k=None, layout: str = "bhnd", prefix_tiles: int = 0, scale=None, stream=None):
     """select + attn_fwd: (O, LSE, idx).  Give topk, or sparsity (the fraction
     of key/value tiles left out, as in the fastbsa page's "Use" example)."""
     if (topk is None) == (sparsity is None):
         raise ValueError("give exactly one of topk and sparsity")
     if topk is None:
-        topk = topk_from_sparsity(grid, tile, sparsity, grid_k, tile_k, _dims(q, layout)[3])
+        topk = topk_from_sparsity(grid, tile, sparsity, grid_k, tile_k, _dims(q, layout)[3], prefix_tiles)
     kw = dict(grid_k=grid_k, tile_k=tile_k, layout=layout, stream=stream)
-    idx = select(q, k, grid, tile, topk, **kw)
+    idx = select(q, k, grid, tile, topk, prefix_tiles=prefix_tiles, **kw)
     o, lse = attn_fwd(q, k, v, idx, grid, tile, scale=scale, **kw)
     return o, lse, idx
 

@@ -40,6 +40,7 @@ static int side_geom(const vsa_shape* s, int T, int Hh, int W, int tt, int th, i
   g->vol = vol;
   g->f16 = s->dtype == VSA_DTYPE_F16 ? 1 : 0;
   g->layout = s->layout;
+  g->prefix = 0;
   g->nTt = ceil_div(T, tt);
   g->nTy = ceil_div(Hh, th);
   g->nTx = ceil_div(W, tw);
@@ -70,6 +71,8 @@ static int make_geoms(const vsa_shape* s, Geom* gq, Geom* gk) {
                  ktile ? s->hk : s->th, ktile ? s->wk : s->tw, gk);
   if (rc != VSA_OK) return rc;
   if (gq->vol != gk->vol) return VSA_ERR_UNSUPPORTED;
+  if (s->prefix_tiles < 0 || s->prefix_tiles > gk->nT) return VSA_ERR_INVALID_ARG;
+  gk->prefix = s->prefix_tiles;
   return VSA_OK;
 }
 
@@ -262,6 +265,7 @@ int vsa_topk_from_sparsity(const vsa_shape* shape, float sparsity, int32_t* topk
   const double keep = (1.0 - static_cast<double>(sparsity)) * gk.nT;
   long long k = static_cast<long long>(std::floor(keep + 0.5));
   if (k < 1) k = 1;
+  if (k < gk.prefix) k = gk.prefix;
   if (k > gk.nT) k = gk.nT;
   *topk = static_cast<int32_t>(k);
   return VSA_OK;
@@ -279,7 +283,7 @@ int vsa_select(const vsa_shape* shape, const void* q, const void* k, int32_t top
   int rc = make_geoms(shape, &gq, &gk);
   if (rc != VSA_OK) return rc;
   if (q == nullptr || k == nullptr || idx_out == nullptr) return VSA_ERR_INVALID_ARG;
-  if (topk <= 0 || topk > gk.nT) return VSA_ERR_TOPK_RANGE;
+  if (topk <= 0 || topk > gk.nT || topk < gk.prefix) return VSA_ERR_TOPK_RANGE;
   if (!aligned16(q) || !aligned16(k) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(idx_out) & 3u))
     return VSA_ERR_ALIGNMENT;
   if (workspace == nullptr || workspace_bytes < select_workspace_bytes(gq, gk)) return VSA_ERR_WORKSPACE;
@@ -294,7 +298,7 @@ int vsa_select_noalloc(const vsa_shape* shape, const void* q, const void* k, int
   int rc = make_geoms(shape, &gq, &gk);
   if (rc != VSA_OK) return rc;
   if (q == nullptr || k == nullptr || idx_out == nullptr) return VSA_ERR_INVALID_ARG;
-  if (topk <= 0 || topk > gk.nT) return VSA_ERR_TOPK_RANGE;
+  if (topk <= 0 || topk > gk.nT || topk < gk.prefix) return VSA_ERR_TOPK_RANGE;
   if (!aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(idx_out) & 3u)) return VSA_ERR_ALIGNMENT;
   if (select_workspace_bytes(gq, gk) > VSA_SELECT_NOALLOC_SCRATCH_BYTES) return VSA_ERR_WORKSPACE;
   if ((rc = check_arch()) != VSA_OK) return rc;

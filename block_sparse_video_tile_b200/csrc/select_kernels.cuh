@@ -52,6 +52,9 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
+// Order key of an always-kept (prefix) tile: above every finite score's key.
+constexpr uint32_t kKeepKey = 0xffffffffu;
+
 // Exact top-k of NR rows of order keys by one warp, keys held in registers
 // (lane l holds tiles l, l + 32, ...).  The topk-th largest key T of a row is
 // found bit by bit from the top: T keeps a bit when at least topk keys are
@@ -368,7 +371,7 @@ __global__ void __launch_bounds__(kWideThreads) score_topk_kernel(Geom gq, Geom 
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int key = kw0 + (j < 4 ? 0 : 32) + 4 * kg + (j & 3);
-          if (row < nrows && key < nT) keys[row * nT + key] = order_key(acc[i][j] + 0.f);
+          if (row < nrows && key < nT) keys[row * nT + key] = key < gk.prefix ? kKeepKey : order_key(acc[i][j] + 0.f);
           acc[i][j] = 0.f;
         }
       }
@@ -477,7 +480,8 @@ __global__ void __launch_bounds__(kNarrowThreads) score_topk_narrow_kernel(Geom 
       for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          if (4 * qg + i < nrows && kc0 + j < nT) keys[(4 * qg + i) * nT + kc0 + j] = order_key(acc[i][j] + 0.f);
+          if (4 * qg + i < nrows && kc0 + j < nT)
+            keys[(4 * qg + i) * nT + kc0 + j] = kc0 + j < gk.prefix ? kKeepKey : order_key(acc[i][j] + 0.f);
           acc[i][j] = 0.f;
         }
     }

@@ -23,6 +23,7 @@ struct Geom {
   int vol;                  // tt * th * tw
   int f16;                  // element type: 0 bfloat16, 1 float16
   int layout;               // 0: [B, H, N, d]; 1: [B, N, H, d]
+  int prefix;               // key/value side: tiles 0 .. prefix-1 are always kept (0 on the query side)
 };
 
 // A query-side and a key/value-side Geom share B, H, d, f16 and layout; each

@@ -37,6 +37,7 @@ class Workload:
     layout: str = "bhnd"       # "bhnd" = [B, H, N, d] or "bnhd" = [B, N, H, d]
     grid_k: tuple | None = None   # key/value grid (None: the query grid)
     tile_k: tuple | None = None   # key/value tile (None: the query tile)
+    prefix_tiles: int = 0         # key/value tiles kept for every query tile
 
     @property
     def N(self) -> int:

@@ -28,6 +28,13 @@
  *   LSE        : float32 [B, H, Nq] in both layouts, natural log of the
  *                softmax denominator
  *
+ * Always-kept prefix tiles (FastVideo guide, "Choose top-k": the H3 route
+ * uses 64-token blocks and keeps all prefix blocks): with prefix_tiles = P,
+ * key/value tiles 0 .. P-1 (the first in raster order -- e.g. the tiles of
+ * leading conditioning frames) are in every query tile's kept list whatever
+ * their scores, and the other topk - P are the best-scoring of the rest;
+ * P <= topk.
+ *
  * Query and key/value grids (fastbsa page, "Use": separate latent and chunk
  * shapes for q and k): by default both sides use the query grid and tile
  * (self-attention with equal lengths, the Wan route of the FastVideo guide).
@@ -77,6 +84,8 @@ typedef struct vsa_shape {
   int32_t layout;        /* VSA_LAYOUT_BHND (0, default) or VSA_LAYOUT_BNHD   */
   int32_t Tk, Hk, Wk;    /* key/value grid; all 0 (default): the query grid   */
   int32_t tk, hk, wk;    /* key/value tile; all 0 (default): the query tile   */
+  int32_t prefix_tiles;  /* key/value tiles 0 .. prefix_tiles-1 are kept for
+                            every query tile (counted in topk); 0: none        */
 } vsa_shape;
 
 /* Element types (FastVideo VSA guide, "Verify routing and fallback": the
@@ -91,9 +100,10 @@ typedef struct vsa_shape {
 typedef enum vsa_status {
   VSA_OK = 0,
   VSA_ERR_INVALID_ARG = 1,  /* NULL pointer, non-positive extent, bad scale    */
-  VSA_ERR_TOPK_RANGE = 2,   /* topk <= 0 or topk > nTk (guide: topk must be
-                               positive; topk > num_blocks is invalid), or a
-                               sparsity outside [0, 1)                          */
+  VSA_ERR_TOPK_RANGE = 2,   /* topk <= 0, topk > nTk or topk < prefix_tiles
+                               (guide: topk must be positive; topk >
+                               num_blocks is invalid), or a sparsity outside
+                               [0, 1)                                           */
   VSA_ERR_UNSUPPORTED = 3,  /* d, dtype, layout or tile shape outside the
                                supported set (incl. unequal tile volumes)       */
   VSA_ERR_ALIGNMENT = 4,    /* a tensor pointer not 16-byte aligned            */
@@ -115,7 +125,8 @@ int vsa_kv_tile_count(const vsa_shape* shape, int32_t* num_tiles, int32_t* tiles
 
 /* Kept tiles per query tile for a sparsity (fastbsa page, "Use": sparsity =
  * the fraction of key/value tiles left out, 0.9375 keeping 45 of 720):
- * topk = round((1 - sparsity) * nTk) (halves round up), clamped to [1, nTk].
+ * topk = round((1 - sparsity) * nTk) (halves round up), clamped to
+ * [max(1, prefix_tiles), nTk].
  * sparsity must lie in [0, 1).  Host only. */
 int vsa_topk_from_sparsity(const vsa_shape* shape, float sparsity, int32_t* topk);
 
@@ -128,7 +139,7 @@ size_t vsa_select_workspace_bytes(const vsa_shape* shape);
 /* Tile selection (FastVideo VSA guide intro and "Wan top-k behavior"; fastbsa
  * page "How it works": selection kept on chip, no score matrix in HBM).
  *   q, k      : device Q and K in shape->layout and shape->dtype, 16-byte aligned
- *   topk      : kept key tiles per query tile, 1 <= topk <= nTk
+ *   topk      : kept key tiles per query tile, max(1, prefix_tiles) <= topk <= nTk
  *               (topk == nTk keeps every tile: the dense case)
  *   idx_out   : device int32 [B, H, nTq, topk]; row i gets the topk tiles j with
  *               the largest s_ij = mean_i(Q) . mean_j(K) (float32 means over the

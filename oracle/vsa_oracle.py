@@ -39,7 +39,12 @@ What it computes, and where the pages fix each step:
    the other (scores nTq x nTk, top-k over nTk).
 7. Sparsity (fastbsa page, "Use": sparsity=0.9375): the fraction of key/value
    blocks left out.  Reading: topk = round((1 - sparsity) * nTk), halves
-   rounding up, clamped to [1, nTk] (0.9375 of 720 blocks keeps 45).
+   rounding up, clamped to [max(1, P), nTk] (0.9375 of 720 blocks keeps 45).
+8. Always-kept prefix blocks (user guide, "Choose top-k": H3 "keeps all prefix
+   blocks").  Reading: the first P key/value blocks in raster order are in
+   every query block's kept list whatever their scores (their scores count
+   as +inf for the selection) and count toward topk; the other topk - P are
+   the best-scoring of the rest.
 """
 from __future__ import annotations
 
@@ -120,36 +125,50 @@ def topk_row(s_row: np.ndarray, topk: int) -> np.ndarray:
 def tie_gap(s_row: np.ndarray, topk: int):
     """(relative gap, absolute band delta) between the k-th and (k+1)-th scores.
 
-    Returns (inf, 0) when topk == number of blocks (nothing is left out).
+    Returns (inf, 0) when topk == number of blocks (nothing is left out) or
+    when the cut falls next to an always-kept (+inf) block.
     """
     nT = s_row.shape[0]
     if topk >= nT:
         return math.inf, 0.0
     srt = np.sort(s_row)[::-1]
     a, b = srt[topk - 1], srt[topk]
-    denom = max(abs(a), abs(b), EPS_ROW_REL * float(np.max(np.abs(s_row))))
+    if not (np.isfinite(a) and np.isfinite(b)):
+        return math.inf, 0.0
+    finite = np.abs(s_row[np.isfinite(s_row)])
+    denom = max(abs(a), abs(b), EPS_ROW_REL * float(finite.max()))
     if denom == 0.0:
         return 0.0, 0.0
     return abs(a - b) / denom, NEAR_TIE_REL * denom
 
 
-def select_head(Q: np.ndarray, K: np.ndarray, grid, tile, topk: int, grid_k=None, tile_k=None):
+def keep_prefix(scores: np.ndarray, prefix: int) -> np.ndarray:
+    """Scores as the selection sees them: the first ``prefix`` key/value blocks at +inf."""
+    s = np.array(scores, dtype=np.float64, copy=True)
+    s[..., :prefix] = math.inf
+    return s
+
+
+def select_head(Q: np.ndarray, K: np.ndarray, grid, tile, topk: int, grid_k=None, tile_k=None, prefix: int = 0):
     """One head: (idx [nTq, topk] int32 ascending, scores [nTq, nTk], near_tie [nTq] bool).
 
-    K is tiled with grid_k / tile_k (default: the query grid / tile).
+    K is tiled with grid_k / tile_k (default: the query grid / tile).  The
+    scores returned are the selection's: the first ``prefix`` blocks at +inf.
     """
     grid_k = grid if grid_k is None else grid_k
     tile_k = tile if tile_k is None else tile_k
     nTq, nTk = num_tiles(grid, tile), num_tiles(grid_k, tile_k)
-    if not 0 < topk <= nTk:
-        raise ValueError(f"topk must be in [1, {nTk}], got {topk}")
-    s = tile_scores(pool(Q, grid, tile), pool(K, grid_k, tile_k))
+    if not 0 <= prefix <= nTk:
+        raise ValueError(f"prefix must be in [0, {nTk}], got {prefix}")
+    if not max(1, prefix) <= topk <= nTk:
+        raise ValueError(f"topk must be in [{max(1, prefix)}, {nTk}], got {topk}")
+    s = keep_prefix(tile_scores(pool(Q, grid, tile), pool(K, grid_k, tile_k)), prefix)
     idx = np.stack([topk_row(s[i], topk) for i in range(nTq)]).astype(np.int32)
     near = np.array([tie_gap(s[i], topk)[0] < NEAR_TIE_REL for i in range(nTq)])
     return idx, s, near
 
 
-def select(q_bits, k_bits, grid, tile, topk: int, dtype: str = "bf16", grid_k=None, tile_k=None):
+def select(q_bits, k_bits, grid, tile, topk: int, dtype: str = "bf16", grid_k=None, tile_k=None, prefix: int = 0):
     """All (b, h): idx [B, H, nTq, topk], scores [B, H, nTq, nTk], near_tie [B, H, nTq].
 
     q_bits [B, H, Nq, d] and k_bits [B, H, Nk, d] hold 16-bit patterns.
@@ -163,16 +182,17 @@ def select(q_bits, k_bits, grid, tile, topk: int, dtype: str = "bf16", grid_k=No
     for b in range(B):
         for h in range(H):
             idx[b, h], sc[b, h], near[b, h] = select_head(
-                widen(q_bits[b, h], dtype), widen(k_bits[b, h], dtype), grid, tile, topk, grid_k, tile_k)
+                widen(q_bits[b, h], dtype), widen(k_bits[b, h], dtype), grid, tile, topk, grid_k, tile_k, prefix)
     return idx, sc, near
 
 
-def topk_from_sparsity(n_kv_tiles: int, sparsity: float) -> int:
-    """Kept blocks per query block for a sparsity in [0, 1): round((1 - s) * n), halves up, in [1, n]."""
+def topk_from_sparsity(n_kv_tiles: int, sparsity: float, prefix: int = 0) -> int:
+    """Kept blocks per query block for a sparsity in [0, 1): round((1 - s) * n), halves up,
+    in [max(1, prefix), n]."""
     if not 0.0 <= sparsity < 1.0:
         raise ValueError(f"sparsity must be in [0, 1), got {sparsity}")
     k = math.floor((1.0 - sparsity) * n_kv_tiles + 0.5)
-    return int(min(max(k, 1), n_kv_tiles))
+    return int(min(max(k, 1, prefix), n_kv_tiles))
 
 
 def selection_is_valid(gpu_row: np.ndarray, s_row: np.ndarray, topk: int) -> bool:

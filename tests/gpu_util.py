@@ -46,8 +46,13 @@ def inputs(w, seed=0):
 
 
 def geo(w) -> dict:
-    """Keyword arguments of api.select / attn_fwd for the workload's key/value grid and layout."""
+    """Keyword arguments of api.attn_fwd for the workload's key/value grid and layout."""
     return dict(grid_k=w.grid_k, tile_k=w.tile_k, layout=w.layout)
+
+
+def sel(w) -> dict:
+    """Keyword arguments of api.select: geo(w) and the always-kept prefix tiles."""
+    return dict(geo(w), prefix_tiles=w.prefix_tiles)
 
 
 def to_bhnd(x: torch.Tensor, w) -> torch.Tensor:
@@ -56,13 +61,15 @@ def to_bhnd(x: torch.Tensor, w) -> torch.Tensor:
 
 
 def oracle_scores(q, k, w):
-    """float64 tile scores [B, H, nTq, nTk] straight from the oracle's steps."""
+    """float64 tile scores [B, H, nTq, nTk] straight from the oracle's steps (always-kept
+    prefix tiles at +inf, as the selection sees them)."""
     B, H = q.shape[:2]
     out = []
     for b in range(B):
         for h in range(H):
             Q, K = vo.widen(q[b, h], w.dtype), vo.widen(k[b, h], w.dtype)
-            out.append(vo.tile_scores(vo.pool(Q, w.grid, w.tile), vo.pool(K, w.kv_grid, w.kv_tile)))
+            out.append(vo.keep_prefix(vo.tile_scores(vo.pool(Q, w.grid, w.tile), vo.pool(K, w.kv_grid, w.kv_tile)),
+                                      w.prefix_tiles))
     return np.stack(out).reshape(B, H, *out[0].shape)
 
 

@@ -172,3 +172,14 @@ def test_bnhd_layout_and_kv_grid_accepted_on_host():
     assert _native.lib().vsa_tile_count(ctypes.byref(shp), ctypes.byref(n), None) == 0 and n.value == 27
     assert _native.lib().vsa_kv_tile_count(ctypes.byref(shp), ctypes.byref(n), None) == 0
     assert n.value == vo.num_tiles((13, 16, 24), (2, 8, 16))
+
+
+def test_prefix_tiles_checked_before_launch():
+    # 120 tiles; prefix beyond them is invalid, topk below the prefix is out of range
+    bad = api.make_shape(1, 2, (31, 22, 40), 128, (4, 8, 8), prefix_tiles=121)
+    n = ctypes.c_int32()
+    assert _native.lib().vsa_tile_count(ctypes.byref(bad), ctypes.byref(n), None) == 1
+    shp = api.make_shape(1, 2, (31, 22, 40), 128, (4, 8, 8), prefix_tiles=15)
+    assert _sel(shp, topk=14) == 2
+    assert _native.lib().vsa_tile_count(ctypes.byref(shp), ctypes.byref(n), None) == 0
+    assert api.topk_from_sparsity((31, 22, 40), (4, 8, 8), 0.99, prefix_tiles=15) == 15

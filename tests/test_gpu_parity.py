@@ -54,6 +54,14 @@ SMALL = [
     Workload("kv_pair", 1, 2, (6, 10, 14), 128, (4, 4, 4), 5, "field", grid_k=(7, 12, 9), tile_k=(2, 4, 8)),
     Workload("kv_tile_bnhd", 2, 1, (6, 12, 20), 64, (2, 8, 8), 4, grid_k=(5, 9, 26), tile_k=(4, 4, 8),
              layout="bnhd"),
+    # always-kept prefix tiles (user guide, "Choose top-k": H3 keeps all prefix
+    # blocks, 64-token blocks): the keys' first 4 frames (12 tiles) are kept by
+    # every query tile, plus 6 by score; and a self-attention case whose first
+    # temporal slice of tiles is the prefix, with topk == prefix_tiles on one
+    Workload("h3_prefix", 1, 2, (8, 12, 16), 128, (4, 4, 4), 18, "field", grid_k=(12, 12, 16), prefix_tiles=12),
+    Workload("h3_prefix_bnhd", 2, 2, (8, 12, 16), 64, (4, 4, 4), 12, grid_k=(12, 12, 16), prefix_tiles=12,
+             layout="bnhd"),
+    Workload("prefix_self", 1, 2, (9, 20, 20), 128, (4, 8, 8), 12, "field", prefix_tiles=9),
 ]
 BY_NAME = {w.name: w for w in SMALL}
 
@@ -66,7 +74,7 @@ def _seed(w):
 def test_small_full_compare(w):
     (q, k, v), (qd, kd, vd) = gu.inputs(w, seed=_seed(w))
     scale = w.d ** -0.5
-    idx = api.select(qd, kd, w.grid, w.tile, w.topk, **gu.geo(w))
+    idx = api.select(qd, kd, w.grid, w.tile, w.topk, **gu.sel(w))
     torch.cuda.synchronize()
     gu.assert_no_device_error()
     scores = gu.oracle_scores(q, k, w)
@@ -169,7 +177,7 @@ def _full_case(w, seed=0, topks=None):
     rng = np.random.default_rng(11)
     report = {}
     for topk in (topks or [w.topk]):
-        idx = api.select(qd, kd, w.grid, w.tile, topk, **gu.geo(w))
+        idx = api.select(qd, kd, w.grid, w.tile, topk, **gu.sel(w))
         gi = idx.cpu().numpy()
         rows, ties = gu.check_selection(gi, scores, topk)
         o, lse = api.attn_fwd(qd, kd, vd, idx, w.grid, w.tile, **gu.geo(w))

@@ -63,6 +63,12 @@ def _attend_kv_with_query_tiles(Q, K, V, grid, tile, idx, scale, query_tiles=Non
     return _orig_attend(Q, K, V, grid, tile, idx, scale, query_tiles)
 
 
+def _prefix_dropped(scores, prefix):
+    s = np.array(scores, dtype=np.float64, copy=True)
+    s[..., :prefix] = -np.inf
+    return s
+
+
 CASES = [
     ("pool", _zero_padded_pool, lambda: pins.test_pool_constant_per_block_partial_edges()),
     ("tile_scores", _transposed_scores, lambda: pins.test_scores_hand_example()),
@@ -76,6 +82,7 @@ CASES = [
     ("select_head", _select_kv_with_query_tile, lambda: pins.test_kv_pool_uses_kv_tiles()),
     ("attend_head", _attend_kv_with_query_tiles,
      lambda: pins.test_kv_grid_all_blocks_equals_dense(*pins.KV_CASES[0])),
+    ("keep_prefix", _prefix_dropped, lambda: pins.test_prefix_blocks_always_kept(3, 5)),
 ]
 
 

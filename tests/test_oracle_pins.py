@@ -365,3 +365,49 @@ def test_topk_from_sparsity():
     for bad in (1.0, -0.1, 1.5):
         with pytest.raises(ValueError):
             vo.topk_from_sparsity(10, bad)
+
+
+# ----------------------------- always-kept prefix blocks (user guide, "Choose top-k": H3)
+def _ranked(scores, k):
+    """The k best of (index, score) pairs, ties to the lower index, by a plain sort."""
+    return [j for _, j in sorted((-sc, j) for j, sc in scores)[:k]]
+
+
+@pytest.mark.parametrize("prefix,topk", [(0, 5), (3, 5), (3, 3), (6, 9)])
+def test_prefix_blocks_always_kept(prefix, topk):
+    # prefix blocks get the lowest means on purpose: plain top-k would drop them
+    grid, tile, d = (4, 6, 6), (2, 2, 2), 5                  # 2 x 3 x 3 = 18 blocks
+    rng = np.random.default_rng(9)
+    Q = _rand((math.prod(grid), d), 31)
+    K = _rand((math.prod(grid), d), 32)
+    toks = vo.tile_tokens(grid, tile)
+    qm = vo.pool(Q, grid, tile).mean(axis=0)
+    for j in range(prefix):
+        K[toks[j]] = -10.0 * qm / max(np.linalg.norm(qm), 1e-9) + 0.01 * rng.standard_normal((len(toks[j]), d))
+    idx, s, near = vo.select_head(Q, K, grid, tile, topk, prefix=prefix)
+    raw = vo.tile_scores(vo.pool(Q, grid, tile), vo.pool(K, grid, tile))
+    for i in range(len(toks)):
+        rest = _ranked([(j, raw[i, j]) for j in range(prefix, len(toks))], topk - prefix)
+        assert idx[i].tolist() == sorted(list(range(prefix)) + rest)
+    if prefix:
+        # the inputs are such that plain top-k would leave prefix blocks out
+        plain, _, _ = vo.select_head(Q, K, grid, tile, topk)
+        assert any(not set(range(prefix)) <= set(plain[i].tolist()) for i in range(len(toks)))
+    # the tie band only looks at the blocks that compete
+    for i in range(len(toks)):
+        rel, _ = vo.tie_gap(s[i], topk)
+        if topk == prefix:
+            assert rel == math.inf
+        else:
+            ref, _ = vo.tie_gap(raw[i, prefix:], topk - prefix)
+            assert rel == pytest.approx(ref, rel=1e-12, abs=1e-300) or (math.isinf(rel) and math.isinf(ref))
+
+
+def test_prefix_range_rejected():
+    grid, tile = (4, 4, 4), (2, 2, 2)
+    Q = _rand((64, 4), 33)
+    with pytest.raises(ValueError):
+        vo.select_head(Q, Q, grid, tile, 2, prefix=3)       # topk < prefix
+    with pytest.raises(ValueError):
+        vo.select_head(Q, Q, grid, tile, 8, prefix=9)       # prefix > nT
+    assert vo.topk_from_sparsity(8, 0.99, prefix=3) == 3
