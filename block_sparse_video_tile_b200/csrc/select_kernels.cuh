@@ -278,12 +278,13 @@ constexpr int kWideRows = 32;
 constexpr int kWideKeys = 512;
 constexpr int kWideSlice = 16;
 constexpr int kWideStages = 3;
-constexpr int kWideThreads = 256;
+constexpr int kWideMathWarps = 8;
+constexpr int kWideThreads = 512;     // warps 8-15 help only with copies and the top-k
 constexpr int kWideMaxTiles = 768;
 constexpr int kNarrowMaxTiles = 256;   // below this the narrow kernel is used too (more, shorter CTAs)
 
 template <int D>
-__global__ void __launch_bounds__(kWideThreads) score_topk_kernel(Geom gq, Geom gk, const float* __restrict__ means, int topk,
+__global__ void __launch_bounds__(kWideThreads, 1) score_topk_kernel(Geom gq, Geom gk, const float* __restrict__ means, int topk,
                                                                   int32_t* __restrict__ idx) {
   constexpr int SPP = D / kWideSlice;      // stages per pass
   constexpr int SLICE = kWideSlice * kWideKeys;
@@ -347,7 +348,7 @@ __global__ void __launch_bounds__(kWideThreads) score_topk_kernel(Geom gq, Geom 
     issue(st + kWideStages - 1);
     const int sl = st % SPP;
     const int kw0 = (st / SPP) * kWideKeys + 64 * warp;   // the warp's first key tile
-    if (kw0 < nT) {
+    if (warp < kWideMathWarps && kw0 < nT) {
       const float* kb = ring + (st % kWideStages) * SLICE + 64 * warp + 4 * kg;
       const float* qb = qT + sl * kWideSlice * R + 4 * qg;
 #pragma unroll
@@ -364,7 +365,7 @@ __global__ void __launch_bounds__(kWideThreads) score_topk_kernel(Geom gq, Geom 
           for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(qa[i], ka[j], acc[i][j]);
       }
     }
-    if (sl == SPP - 1) {             // end of a pass: scores -> order keys
+    if (sl == SPP - 1 && warp < kWideMathWarps) {   // end of a pass: scores -> order keys
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int row = (i < 4 ? 0 : 16) + 4 * qg + (i & 3);
@@ -400,7 +401,8 @@ constexpr int kNarrowRows = 16;
 constexpr int kNarrowKeys = 256;
 constexpr int kNarrowSlice = 16;
 constexpr int kNarrowStages = 4;
-constexpr int kNarrowThreads = 256;
+constexpr int kNarrowMathWarps = 8;
+constexpr int kNarrowThreads = 256;   // two CTAs per SM at small tile counts
 
 template <int D>
 __global__ void __launch_bounds__(kNarrowThreads) score_topk_narrow_kernel(Geom gq, Geom gk, const float* __restrict__ means,
@@ -461,20 +463,22 @@ __global__ void __launch_bounds__(kNarrowThreads) score_topk_narrow_kernel(Geom 
     __syncthreads();
     issue(st + kNarrowStages - 1);
     const int sl = st % SPP;
-    const float* kb = ring + (st % kNarrowStages) * SLICE + 32 * warp + 4 * kg;
+    const float* kb = ring + (st % kNarrowStages) * SLICE + 32 * (warp % kNarrowMathWarps) + 4 * kg;
     const float* qb = qT + sl * kNarrowSlice * R + 4 * qg;
+    if (warp < kNarrowMathWarps) {
 #pragma unroll
-    for (int c = 0; c < kNarrowSlice; ++c) {
-      const float4 qv = *reinterpret_cast<const float4*>(qb + c * R);
-      const float4 kv = *reinterpret_cast<const float4*>(kb + c * kNarrowKeys);
-      const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
-      const float ka[4] = {kv.x, kv.y, kv.z, kv.w};
+      for (int c = 0; c < kNarrowSlice; ++c) {
+        const float4 qv = *reinterpret_cast<const float4*>(qb + c * R);
+        const float4 kv = *reinterpret_cast<const float4*>(kb + c * kNarrowKeys);
+        const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
+        const float ka[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(qa[i], ka[j], acc[i][j]);
+          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(qa[i], ka[j], acc[i][j]);
+      }
     }
-    if (sl == SPP - 1) {
+    if (sl == SPP - 1 && warp < kNarrowMathWarps) {
       const int kc0 = (st / SPP) * kNarrowKeys + 32 * warp + 4 * kg;
 #pragma unroll
       for (int i = 0; i < 4; ++i)
