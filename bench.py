@@ -51,9 +51,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # ------------------------------------------------------------------ helpers
-def tile_counts(w) -> np.ndarray:
-    """Valid token count of every tile (raster tile order)."""
-    (T, Hh, W), (tt, th, tw) = w.grid, w.tile
+def tile_counts(w, kv: bool = False) -> np.ndarray:
+    """Valid token count of every query tile (key/value tile with kv=True), raster tile order."""
+    (T, Hh, W), (tt, th, tw) = (w.kv_grid, w.kv_tile) if kv else (w.grid, w.tile)
     ct = np.minimum(tt, T - np.arange(0, T, tt))
     cy = np.minimum(th, Hh - np.arange(0, Hh, th))
     cx = np.minimum(tw, W - np.arange(0, W, tw))
@@ -61,9 +61,9 @@ def tile_counts(w) -> np.ndarray:
 
 
 def exact_flops(idx: np.ndarray, w) -> float:
-    c = tile_counts(w)
-    kept = c[idx].sum(axis=-1)                      # [B, H, nT] kept key tokens per query tile
-    return float(4 * w.d * (kept * c[None, None, :]).sum())
+    cq, ck = tile_counts(w), tile_counts(w, kv=True)
+    kept = ck[idx].sum(axis=-1)                     # [B, H, nTq] kept key tokens per query tile
+    return float(4 * w.d * (kept * cq[None, None, :]).sum())
 
 
 def nominal_flops(w) -> float:
@@ -73,7 +73,8 @@ def nominal_flops(w) -> float:
 
 def select_bytes(w) -> float:
     nT = len(tile_counts(w))
-    return float(2 * w.B * w.H * w.N * w.d * 2 + w.B * w.H * nT * w.topk * 4)
+    Nk = math.prod(w.kv_grid)
+    return float(w.B * w.H * (w.N + Nk) * w.d * 2 + w.B * w.H * nT * w.topk * 4)
 
 
 def load_peaks():
@@ -169,28 +170,38 @@ def make_inputs(w, device, seed):
     generator): N(0,1), or for "field" workloads Q and K = a shared sum of 8
     random low-frequency sinusoids over (t, y, x) per (head, channel) + 0.5 N(0,1)
     noise each and V = N(0,1) -- the same families the parity tests draw on the
-    host (synth.py), not the same numbers."""
+    host (synth.py), not the same numbers.  Q covers the query grid, K and V
+    the key/value grid (K's field sampled on its own grid in normalised
+    coordinates); returned in the workload's layout."""
     g = torch.Generator(device=device)
     g.manual_seed(seed)
-    shape = (w.B, w.H, w.N, w.d)
+    Nk = math.prod(w.kv_grid)
+    qshape, kshape = (w.B, w.H, w.N, w.d), (w.B, w.H, Nk, w.d)
     if w.kind != "field":
-        return [torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
-                for _ in range(3)]
-    T, Hh, W = w.grid
-    n = torch.arange(w.N, device=device)
-    pos = torch.stack([(n // (Hh * W)) / T, ((n // W) % Hh) / Hh, (n % W) / W], dim=1).float()   # [N, 3]
-    q = torch.empty(shape, dtype=torch.bfloat16, device=device)
-    k = torch.empty_like(q)
-    for b in range(w.B):
-        for h in range(w.H):
-            freq = torch.rand((3, w.d * 8), generator=g, device=device) * 1.5
-            phase = torch.rand((w.d * 8,), generator=g, device=device) * (2 * math.pi)
-            ang = 2 * math.pi * (pos @ freq) + phase                                  # [N, d*8]
-            field = 0.5 * torch.sin(ang).view(w.N, w.d, 8).sum(-1)
-            q[b, h] = (field + 0.5 * torch.randn(field.shape, generator=g, device=device)).to(torch.bfloat16)
-            k[b, h] = (field + 0.5 * torch.randn(field.shape, generator=g, device=device)).to(torch.bfloat16)
-    v = torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
-    return [q, k, v]
+        out = [torch.randn(shp, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+               for shp in (qshape, kshape, kshape)]
+    else:
+        def positions(grid):
+            T, Hh, W = grid
+            n = torch.arange(T * Hh * W, device=device)
+            return torch.stack([(n // (Hh * W)) / T, ((n // W) % Hh) / Hh, (n % W) / W], dim=1).float()
+
+        pq, pk = positions(w.grid), positions(w.kv_grid)                  # [N, 3]
+        q = torch.empty(qshape, dtype=torch.bfloat16, device=device)
+        k = torch.empty(kshape, dtype=torch.bfloat16, device=device)
+        for b in range(w.B):
+            for h in range(w.H):
+                freq = torch.rand((3, w.d * 8), generator=g, device=device) * 1.5
+                phase = torch.rand((w.d * 8,), generator=g, device=device) * (2 * math.pi)
+                for x, pos in ((q, pq), (k, pk)):
+                    ang = 2 * math.pi * (pos @ freq) + phase                  # [N, d*8]
+                    field = 0.5 * torch.sin(ang).view(pos.shape[0], w.d, 8).sum(-1)
+                    x[b, h] = (field + 0.5 * torch.randn(field.shape, generator=g, device=device)).to(torch.bfloat16)
+        v = torch.randn(kshape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+        out = [q, k, v]
+    if w.layout == "bnhd":
+        out = [x.permute(0, 2, 1, 3).contiguous() for x in out]
+    return out
 
 
 # ---------------------------------------------------------------- oracle arm
@@ -200,16 +211,19 @@ def oracle_sample(q_bits, k_bits, v_bits, w, n_tiles):
     from oracle import vsa_oracle as vo
     t0 = time.perf_counter()
     Q, K, V = (vo.bf16_to_f64(x) for x in (q_bits, k_bits, v_bits))
-    idx, _, _ = vo.select_head(Q, K, w.grid, w.tile, w.topk)
-    vo.attend_head(Q, K, V, w.grid, w.tile, idx, w.d ** -0.5, query_tiles=range(n_tiles))
+    idx, _, _ = vo.select_head(Q, K, w.grid, w.tile, w.topk, w.kv_grid, w.kv_tile, w.prefix_tiles)
+    vo.attend_head(Q, K, V, w.grid, w.tile, idx, w.d ** -0.5, query_tiles=range(n_tiles),
+                   grid_k=w.kv_grid, tile_k=w.kv_tile)
     dt = time.perf_counter() - t0
-    c = tile_counts(w)
-    fl = float(4 * w.d * sum(c[i] * c[idx[i]].sum() for i in range(n_tiles)))
+    cq, ck = tile_counts(w), tile_counts(w, kv=True)
+    fl = float(4 * w.d * sum(cq[i] * ck[idx[i]].sum() for i in range(n_tiles)))
     return dt, fl
 
 
-def head_bits(x: torch.Tensor, b=0, h=0) -> np.ndarray:
-    return x[b, h].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+def head_bits(x: torch.Tensor, w, b=0, h=0) -> np.ndarray:
+    """One head's [N, d] 16-bit patterns from a tensor in the workload's layout."""
+    xh = x[b, :, h] if w.layout == "bnhd" else x[b, h]
+    return xh.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
 def run_reference(args, w, rank):
@@ -259,8 +273,15 @@ def aggregate_tflops(flops_per_rank_step: float, ms_max: float, steps: int, worl
 
 
 def describe(w) -> str:
+    extra = ""
+    if w.grid_k is not None or w.tile_k is not None:
+        extra += f" kv_grid={tuple(w.kv_grid)} kv_tile={tuple(w.kv_tile)}"
+    if w.prefix_tiles:
+        extra += f" prefix_tiles={w.prefix_tiles}"
+    if w.layout != "bhnd":
+        extra += f" layout={w.layout}"
     return (f"{w.name}: B={w.B} H={w.H} d={w.d} grid={tuple(w.grid)} tile={tuple(w.tile)} "
-            f"topk={w.topk} inputs={w.kind}")
+            f"topk={w.topk}{extra} inputs={w.kind}")
 
 
 # ------------------------------------------------------------------ our arm
@@ -269,8 +290,9 @@ def run_ours(args, w, rank, world, device):
     grid, tile = w.grid, w.tile
     nT = len(tile_counts(w))
     idx = torch.empty((w.B, w.H, nT, w.topk), dtype=torch.int32, device=device)
-    ws = torch.empty(api.select_workspace_bytes(w.B, w.H, grid, w.d, tile), dtype=torch.uint8,
-                     device=device)
+    geo = dict(grid_k=w.grid_k, tile_k=w.tile_k, layout=w.layout)
+    ws = torch.empty(api.select_workspace_bytes(w.B, w.H, grid, w.d, tile, w.grid_k, w.tile_k),
+                     dtype=torch.uint8, device=device)
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream()
@@ -278,10 +300,10 @@ def run_ours(args, w, rank, world, device):
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        api.select(q, k, grid, tile, w.topk, out=idx, workspace=ws)
+        api.select(q, k, grid, tile, w.topk, out=idx, workspace=ws, prefix_tiles=w.prefix_tiles, **geo)
         if ev is not None:
             ev[1].record(stream)
-        api.attn_fwd(q, k, v, idx, grid, tile, out=o, lse=lse)
+        api.attn_fwd(q, k, v, idx, grid, tile, out=o, lse=lse, **geo)
         if ev is not None:
             ev[2].record(stream)
 
@@ -313,27 +335,31 @@ def run_ours(args, w, rank, world, device):
 
     # end to end through the public host-to-host API (api.forward_host): the
     # timed region holds the uploads of Q, K, V from pinned host memory, the
-    # kernels and the downloads of O, LSE and idx, pipelined by chunks of heads
-    hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
-    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    hx = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
-    e2e_steps = max(3, min(args.steps, 10))
+    # kernels and the downloads of O, LSE and idx, pipelined by chunks of heads.
+    # forward_host covers [B, H, N, d] self-attention without prefix tiles.
+    host_path = w.grid_k is None and w.tile_k is None and w.layout == "bhnd" and not w.prefix_tiles
+    e2e_ms = float("nan")
+    if host_path:
+        hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        hx = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+        e2e_steps = max(3, min(args.steps, 10))
 
-    def e2e_step():
-        api.forward_host(hq, hk, hv, grid, tile, w.topk, out=ho, lse=hl, idx=hx, chunk_heads=4)
+        def e2e_step():
+            api.forward_host(hq, hk, hv, grid, tile, w.topk, out=ho, lse=hl, idx=hx, chunk_heads=4)
 
-    e2e_step()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    e0.record(stream)
-    for _ in range(e2e_steps):
         e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / e2e_steps
 
     ms_max, e2e_max = max_over_ranks([ms, e2e_ms], world, device)
     if rank != 0:
@@ -362,20 +388,22 @@ def run_ours(args, w, rank, world, device):
                      "peak": tensor_peak, "unit": "TFLOP/s", "frac": att_tflops / tensor_peak,
                      "peak_source": f"{src} {peak_kind}",
                      "traffic": recorded_traffic("attn_fwd_kernel", w.name)},
-        "select_roofline": {"kernels": "pool_kernel + " + ("score_topk_kernel" if 256 < nT <= 768 else "score_topk_narrow_kernel"), "bound": "hbm", "achieved": sel_gbs,
+        "select_roofline": {"kernels": "pool_kernel + " + ("score_topk_kernel" if 256 < len(tile_counts(w, kv=True)) <= 1024 else "score_topk_narrow_kernel"), "bound": "hbm", "achieved": sel_gbs,
                             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": sel_gbs / peaks["hbm_gbs"],
                             "peak_source": f"{src} hbm_gbs",
                             "traffic": recorded_traffic("pool_kernel", w.name)},
-        "e2e": {"value": aggregate_tflops(flops, e2e_max, 1, world), "unit": "TFLOP/s", "ms_per_step": e2e_max,
-                "h2d_bytes_per_step": int(3 * q.numel() * 2),
-                "d2h_bytes_per_step": int(o.numel() * 2 + lse.numel() * 4 + idx.numel() * 4),
-                "api": "forward_host (pinned host buffers, 4-head chunks on 3 streams)"},
+        "e2e": ({"value": aggregate_tflops(flops, e2e_max, 1, world), "unit": "TFLOP/s", "ms_per_step": e2e_max,
+                 "h2d_bytes_per_step": int((q.numel() + k.numel() + v.numel()) * 2),
+                 "d2h_bytes_per_step": int(o.numel() * 2 + lse.numel() * 4 + idx.numel() * 4),
+                 "api": "forward_host (pinned host buffers, 4-head chunks on 3 streams)"} if host_path else
+                {"value": None, "unit": "TFLOP/s",
+                 "why": "forward_host covers [B, H, N, d] self-attention without prefix tiles"}),
         "gpu_launches": 3 * args.steps,
         "clocks": clk.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:
         nt = nT                                   # one full head: ~10-30 s of CPU work
-        dt, fl = oracle_sample(head_bits(q), head_bits(k), head_bits(v), w, nt)
+        dt, fl = oracle_sample(head_bits(q, w), head_bits(k, w), head_bits(v, w), w, nt)
         out["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
                                "kind": "oracle",
                                "sample": f"one head: full tile selection + attention for {nt} of {nT} "

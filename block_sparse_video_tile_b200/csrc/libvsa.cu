@@ -102,32 +102,53 @@ static unsigned int* device_error_ptr() {
 // Score + top-k grid, launched as a programmatic dependent of the pooling
 // grid: its CTAs may start while pooling drains; griddepcontrol.wait holds
 // them until the pooled means are complete.  Heads of kNarrowMaxTiles + 1 ..
-// kWideMaxTiles tiles take the wide kernel (32 query tiles per CTA); smaller
-// heads (little score work, more CTAs) and larger ones (key rows that would
-// not fit beside the wide ring) take the narrow kernel (16).
+// kWideLongMaxTiles key tiles take the wide kernel (32 query tiles per CTA;
+// a 2-deep ring past kWideMaxTiles); smaller heads (little score work, more
+// CTAs) and larger ones (key rows that would not fit beside the wide ring)
+// take the narrow kernel (16).
+template <int D, int STAGES>
+static int launch_score_wide(const Geom& gq, const Geom& gk, int topk, int32_t* idx, const float* means,
+                             const cudaLaunchAttribute* attr, cudaStream_t st) {
+  const size_t smem = score_smem_bytes<D, STAGES>(gk);
+  if (cudaFuncSetAttribute(score_topk_kernel<D, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return VSA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ceil_div(gq.nT, kWideRows), gq.B * gq.H);
+  cfg.blockDim = dim3(kWideThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = const_cast<cudaLaunchAttribute*>(attr);
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, score_topk_kernel<D, STAGES>, gq, gk, means, topk, idx) == cudaSuccess
+             ? VSA_OK
+             : VSA_ERR_CUDA;
+}
+
 template <int D>
 static int launch_score(const Geom& gq, const Geom& gk, int topk, int32_t* idx, const float* means,
                         cudaStream_t st) {
-  const bool wide = gk.nT > kNarrowMaxTiles && gk.nT <= kWideMaxTiles;
-  const size_t smem = wide ? score_smem_bytes<D>(gk) : score_narrow_smem_bytes<D>(gk);
-  const void* fn = wide ? reinterpret_cast<const void*>(score_topk_kernel<D>)
-                        : reinterpret_cast<const void*>(score_topk_narrow_kernel<D>);
-  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
-    return VSA_ERR_CUDA;
-  const int rows = wide ? kWideRows : kNarrowRows;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(ceil_div(gq.nT, rows), gq.B * gq.H);
-  cfg.blockDim = dim3(wide ? kWideThreads : kNarrowThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  if (gk.nT > kNarrowMaxTiles && gk.nT <= kWideMaxTiles)
+    return launch_score_wide<D, kWideStages>(gq, gk, topk, idx, means, attr, st);
+  if (gk.nT > kWideMaxTiles && gk.nT <= kWideLongMaxTiles)
+    return launch_score_wide<D, kWideStagesLong>(gq, gk, topk, idx, means, attr, st);
+  const size_t smem = score_narrow_smem_bytes<D>(gk);
+  if (cudaFuncSetAttribute(score_topk_narrow_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return VSA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ceil_div(gq.nT, kNarrowRows), gq.B * gq.H);
+  cfg.blockDim = dim3(kNarrowThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = wide ? cudaLaunchKernelEx(&cfg, score_topk_kernel<D>, gq, gk, means, topk, idx)
-                             : cudaLaunchKernelEx(&cfg, score_topk_narrow_kernel<D>, gq, gk, means, topk, idx);
-  return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+  return cudaLaunchKernelEx(&cfg, score_topk_narrow_kernel<D>, gq, gk, means, topk, idx) == cudaSuccess
+             ? VSA_OK
+             : VSA_ERR_CUDA;
 }
 
 template <int D, bool F16>

@@ -262,28 +262,31 @@ __device__ __forceinline__ void topk_rows(const uint32_t* keys, int kst, int nT,
   }
 }
 
-// Wide kernel (heads of kNarrowMaxTiles + 1 .. kWideMaxTiles tiles): one CTA per (block of 32
+// Wide kernel (heads of kNarrowMaxTiles + 1 .. kWideLongMaxTiles tiles): one CTA per (block of 32
 // query tiles, head), 8 warps.  Per pass of 512 key tiles, warp w takes key
 // tiles 64w .. 64w + 63 of the pass against all 32 query tiles; lane
 // (qg = lane / 8, kg = lane % 8) holds the 8 x 8 block of query tiles
 // {4qg .. 4qg+3, 16+4qg .. 16+4qg+3} x key tiles {4kg .. 4kg+3, 32+4kg ..
 // 32+4kg+3} of the warp's 64, so each 16-byte load of a quarter-warp covers
 // 128 contiguous bytes (no bank conflicts).  Key means stream through shared
-// memory in slices of 16 channels x 512 key tiles on a 3-deep cp.async ring
+// memory in slices of 16 channels x 512 key tiles on a cp.async ring, 3 deep
+// (2 past kWideMaxTiles key tiles, where the key rows need the room)
 // (one barrier per slice).  Warps whose key tiles lie past nT skip the math.
 // Each score adds its channels in ascending order (deterministic); scores
 // become order keys in shared memory, never written to HBM.
-// Dynamic shared memory: qT [D][32] | ring [3][16][512] | keys [32][nT].
+// Dynamic shared memory: qT [D][32] | ring [STAGES][16][512] | keys [32][nT].
 constexpr int kWideRows = 32;
 constexpr int kWideKeys = 512;
 constexpr int kWideSlice = 16;
-constexpr int kWideStages = 3;
+constexpr int kWideStages = 3;        // ring depth up to kWideMaxTiles key tiles
+constexpr int kWideStagesLong = 2;    // ring depth up to kWideLongMaxTiles (room for the key rows)
 constexpr int kWideMathWarps = 8;
 constexpr int kWideThreads = 512;     // warps 8-15 help only with copies and the top-k
 constexpr int kWideMaxTiles = 768;
+constexpr int kWideLongMaxTiles = 1024;
 constexpr int kNarrowMaxTiles = 256;   // below this the narrow kernel is used too (more, shorter CTAs)
 
-template <int D>
+template <int D, int STAGES>
 __global__ void __launch_bounds__(kWideThreads, 1) score_topk_kernel(Geom gq, Geom gk, const float* __restrict__ means, int topk,
                                                                   int32_t* __restrict__ idx) {
   constexpr int SPP = D / kWideSlice;      // stages per pass
@@ -294,7 +297,7 @@ __global__ void __launch_bounds__(kWideThreads, 1) score_topk_kernel(Geom gq, Ge
   extern __shared__ __align__(16) unsigned char smem_raw[];
   float* qT = reinterpret_cast<float*>(smem_raw);
   float* ring = qT + D * R;
-  uint32_t* keys = reinterpret_cast<uint32_t*>(ring + kWideStages * SLICE);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(ring + STAGES * SLICE);
   const int nT = gk.nT;                     // key tiles (score columns, top-k candidates)
   const int ldq = means_ld(gq.nT), ldk = means_ld(nT);
   const int bh = blockIdx.y;
@@ -317,7 +320,7 @@ __global__ void __launch_bounds__(kWideThreads, 1) score_topk_kernel(Geom gq, Ge
   auto issue = [&](int st) {
     if (st < nstage) {
       const int kc0 = (st / SPP) * kWideKeys, c0 = (st % SPP) * kWideSlice;
-      float* dst = ring + (st % kWideStages) * SLICE;
+      float* dst = ring + (st % STAGES) * SLICE;
 #pragma unroll 4
       for (int f = threadIdx.x; f < SLICE / 4; f += kWideThreads) {
         const int c = f / (kWideKeys / 4), k4 = f % (kWideKeys / 4);
@@ -332,7 +335,7 @@ __global__ void __launch_bounds__(kWideThreads, 1) score_topk_kernel(Geom gq, Ge
     cp_async_commit();
   };
 #pragma unroll
-  for (int st = 0; st < kWideStages - 1; ++st) issue(st);
+  for (int st = 0; st < STAGES - 1; ++st) issue(st);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int qg = lane / 8, kg = lane % 8;
@@ -343,13 +346,13 @@ __global__ void __launch_bounds__(kWideThreads, 1) score_topk_kernel(Geom gq, Ge
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
 
   for (int st = 0; st < nstage; ++st) {
-    cp_async_wait<kWideStages - 2>();
+    cp_async_wait<STAGES - 2>();
     __syncthreads();                 // slice st visible; slot of slice st-1 free
-    issue(st + kWideStages - 1);
+    issue(st + STAGES - 1);
     const int sl = st % SPP;
     const int kw0 = (st / SPP) * kWideKeys + 64 * warp;   // the warp's first key tile
     if (warp < kWideMathWarps && kw0 < nT) {
-      const float* kb = ring + (st % kWideStages) * SLICE + 64 * warp + 4 * kg;
+      const float* kb = ring + (st % STAGES) * SLICE + 64 * warp + 4 * kg;
       const float* qb = qT + sl * kWideSlice * R + 4 * qg;
 #pragma unroll
       for (int c = 0; c < kWideSlice; ++c) {
@@ -383,14 +386,14 @@ __global__ void __launch_bounds__(kWideThreads, 1) score_topk_kernel(Geom gq, Ge
   topk_rows(keys, nT, nT, nrows, topk, idx + (static_cast<size_t>(bh) * gq.nT + row0) * topk, kWideThreads / 32);
 }
 
-template <int D>
+template <int D, int STAGES>
 inline size_t score_smem_bytes(const Geom& gk) {
-  return sizeof(float) * (static_cast<size_t>(D) * kWideRows + kWideStages * kWideSlice * kWideKeys) +
+  return sizeof(float) * (static_cast<size_t>(D) * kWideRows + STAGES * kWideSlice * kWideKeys) +
          sizeof(uint32_t) * static_cast<size_t>(kWideRows) * gk.nT;
 }
 
 // Narrow kernel (heads of at most kNarrowMaxTiles tiles, and of more than
-// kWideMaxTiles, whose 32 key rows would not fit beside the wide ring): one
+// kWideLongMaxTiles, whose 32 key rows would not fit beside the wide ring): one
 // CTA per (block of 16 query tiles,
 // head), 8 warps; lane (qg, kg) of warp w holds the 4 x 4 block of query
 // tiles 4qg .. 4qg+3 x key tiles 32w + 4kg .. 32w + 4kg + 3 of a pass of 256

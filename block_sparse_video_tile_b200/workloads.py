@@ -15,6 +15,9 @@ number of key/value tiles kept per query tile (topk).
 * ``longcat``  -- a LongCat-Video-like 720p grid (12, 48, 80), 4x4x4 chunks ->
   720 tiles, sparsity 0.9375 (topk 45) as in the fastbsa page's "Use" example;
   32 heads of 128; structured Q/K.
+* ``longcat_kv`` -- the LongCat-like grid called the fastbsa way: [B, N, H, d]
+  tensors, keys and values over 16 frames (4 conditioning frames more than the
+  queries' 12), sparsity 0.9375 -> 60 of 960 key tiles.
 * ``sweep``    -- the Wan-5B shape at topk 8, 16, 32, 64 and 120 (120 = all
   tiles, which must equal dense attention), N(0, 1) and structured inputs.
 """
@@ -60,8 +63,13 @@ TINY = Workload("tiny", 1, 2, (8, 8, 8), 64, (4, 4, 4), 2)
 WAN5B = Workload("wan5b", 1, 24, (31, 22, 40), 128, (4, 8, 8), 64)
 WAN14B = Workload("wan14b", 1, 40, (18, 48, 80), 128, (4, 8, 8), 30, "field")
 LONGCAT = Workload("longcat", 1, 32, (12, 48, 80), 128, (4, 4, 4), 45, "field")
+# The LongCat-style call of the fastbsa page ("Use"): [B, N, H, d] tensors, keys and
+# values over 4 more latent frames than the queries (conditioning frames), 4x4x4
+# chunks on both sides, sparsity 0.9375 -> 60 of 960 key/value tiles kept.
+LONGCAT_KV = Workload("longcat_kv", 1, 32, (12, 48, 80), 128, (4, 4, 4), 60, "field", layout="bnhd",
+                      grid_k=(16, 48, 80))
 SWEEP_TOPK = (8, 16, 32, 64, 120)
 SWEEP = tuple(WAN5B.with_(name=f"sweep_k{k}_{kind}", topk=k, kind=kind)
               for kind in ("normal", "field") for k in SWEEP_TOPK)
 
-ALL = {w.name: w for w in (TINY, WAN5B, WAN14B, LONGCAT) + SWEEP}
+ALL = {w.name: w for w in (TINY, WAN5B, WAN14B, LONGCAT, LONGCAT_KV) + SWEEP}
