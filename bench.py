@@ -85,9 +85,17 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def kernel_source_sha() -> str:
+KERNEL_SOURCES = {
+    "attn_fwd_kernel": ("attn_kernel.cuh", "vsa_ptx.cuh", "vsa_geometry.cuh"),
+    "pool_kernel": ("select_kernels.cuh", "vsa_ptx.cuh", "vsa_geometry.cuh"),
+}
+
+
+def kernel_source_sha(kernel: str) -> str:
+    """Hash of the sources one kernel is built from (a traffic record is valid
+    only for the sources it was captured on)."""
     h = hashlib.sha256()
-    for f in ("attn_kernel.cuh", "vsa_ptx.cuh", "vsa_geometry.cuh", "select_kernels.cuh"):
+    for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "block_sparse_video_tile_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -102,7 +110,7 @@ def recorded_traffic(kernel: str, workload: str):
     with open(p) as f:
         rec = json.load(f)
     e = rec.get(kernel, {}).get(workload)
-    if not e or e.get("source_sha") != kernel_source_sha():
+    if not e or e.get("source_sha") != kernel_source_sha(kernel):
         return None
     return e.get("bytes_per_launch")
 
