@@ -355,7 +355,7 @@ def run_ours(args, w, rank, world, device):
         e2e_steps = max(3, min(args.steps, 10))
 
         def e2e_step():
-            api.forward_host(hq, hk, hv, grid, tile, w.topk, out=ho, lse=hl, idx=hx, chunk_heads=4)
+            api.forward_host(hq, hk, hv, grid, tile, w.topk, out=ho, lse=hl, idx=hx, chunk_heads=2)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -403,7 +403,7 @@ def run_ours(args, w, rank, world, device):
         "e2e": ({"value": aggregate_tflops(flops, e2e_max, 1, world), "unit": "TFLOP/s", "ms_per_step": e2e_max,
                  "h2d_bytes_per_step": int((q.numel() + k.numel() + v.numel()) * 2),
                  "d2h_bytes_per_step": int(o.numel() * 2 + lse.numel() * 4 + idx.numel() * 4),
-                 "api": "forward_host (pinned host buffers, 4-head chunks on 3 streams)"} if host_path else
+                 "api": "forward_host (pinned host buffers, 2-head chunks on 3 streams)"} if host_path else
                 {"value": None, "unit": "TFLOP/s",
                  "why": "forward_host covers [B, H, N, d] self-attention without prefix tiles"}),
         "gpu_launches": 3 * args.steps,

@@ -178,7 +178,7 @@ class _HostPipeline:
 _PIPE = {}
 
 
-def forward_host(q, k, v, grid, tile, topk: int, *, scale=None, chunk_heads: int = 4,
+def forward_host(q, k, v, grid, tile, topk: int, *, scale=None, chunk_heads: int = 2,
                  out=None, lse=None, idx=None, device=None):
     """Host-to-host forward: select + attention for pinned CPU tensors.
 
