@@ -21,8 +21,9 @@
 //     work; at worst (disjoint lists) it is half, as with one padded tile.
 // Warp roles (384 threads): warps 0-3 softmax slot 0, warps 4-7 softmax slot 1
 // (thread = query row = TMEM lane), warp 8 TMA producer, warp 9 MMA issuer,
-// warps 10-11 idle.  The producer warpgroup gives registers to the softmax
-// warpgroups (setmaxnreg): 2*128*208 + 128*80 = 63488 <= 384*168, the launch budget.
+// warps 10-11 idle (in MODE_PAIR they build the union lists first).  The
+// producer warpgroup gives registers to the softmax warpgroups (setmaxnreg,
+// RegSplit: 208/88, or 200/96 in MODE_PAIR, within the launch's 384*168).
 // TMEM (512 columns): S_h at [128h, 128h+128), P_h (16-bit pairs) aliases the
 // first 64 columns of S_h, O_h at [256 + 128h, ...).  The MMA warp issues, per
 // K/V sub-block: PV_0(prev), S_0(cur), PV_1(prev), S_1(cur); tcgen05.mma ops
@@ -42,8 +43,16 @@
 namespace vsa {
 
 constexpr int kAttnThreads = 384;        // 3 warpgroups
-constexpr int kSoftmaxRegs = 208;        // per thread, warpgroups 0-1 (after setmaxnreg)
-constexpr int kProducerRegs = 88;        // per thread, warpgroup 2 (TMA + MMA warps)
+// Registers per thread after setmaxnreg: warpgroups 0-1 (softmax) and 2 (TMA
+// and MMA warps).  2*128*S + 128*P must stay within the launch's 384*168.
+// MODE_PAIR's producer walks two union lists and its softmax has less to
+// hold, so it moves 8 registers to the producer (fewer spills, measured).
+template <int MODE>
+struct RegSplit {
+  static constexpr int kSoftmax = MODE == 2 ? 200 : 208;
+  static constexpr int kProducer = MODE == 2 ? 96 : 88;
+  static_assert(2 * 128 * kSoftmax + 128 * kProducer <= 384 * 168, "register split over the launch budget");
+};
 constexpr int kSlotRows = 128;          // MMA M
 constexpr int kSubRows = 128;           // K/V rows per sub-block (S: N, PV: K)
 constexpr float kRescaleLog2 = 8.0f;
@@ -392,7 +401,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= 8) {
-    setmaxnreg_dec<kProducerRegs>();
+    setmaxnreg_dec<RegSplit<MODE>::kProducer>();
   }
   if (warp == 8) {
     // ====================================================== TMA producer
@@ -533,7 +542,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncwarp();
   } else if (warp < 8) {
     // ====================================================== softmax slot h
-    setmaxnreg_inc<kSoftmaxRegs>();
+    setmaxnreg_inc<RegSplit<MODE>::kSoftmax>();
     const int h = warp / 4;
     const int q = warp % 4;
     const int r = threadIdx.x % 128;                  // query row of the slot = TMEM lane
