@@ -55,95 +55,63 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 // Order key of an always-kept (prefix) tile: above every finite score's key.
 constexpr uint32_t kKeepKey = 0xffffffffu;
 
-// Exact top-k of NR rows of order keys by one warp, keys held in registers
-// (lane l holds tiles l, l + 32, ...).  The topk-th largest key T of a row is
-// found bit by bit from the top: T keeps a bit when at least topk keys are
-// >= T with that bit set (a warp-wide count per bit, no shared-memory
-// atomics).  Bits on which all keys of the row agree are decided without
-// counting, and the search stops once exactly topk keys are >= T.  The rows
-// advance together, so their warp reductions overlap.  Every key above T is
-// taken, then the keys equal to T in ascending tile order until topk are
-// taken (ties go to the lower tile index); indices are written in ascending
-// order.  Order keys of finite scores are never 0, so 0 marks padding slots.
-// Rows r < nrow are kr + r * kst, written to out + r * topk.
-template <int MAXE, int NR>
-__device__ __forceinline__ void bsearch_topk_rows(const uint32_t* kr, int kst, int nrow, int nT, int topk,
-                                                  int32_t* out) {
+// Exact top-k of one row of order keys by one warp, keys held in registers
+// (lane l holds tiles l, l + 32, ...).  The topk-th largest key T is found
+// bit by bit from the top: T keeps a bit when at least topk keys are >= T
+// with that bit set (a warp-wide count per bit, no shared-memory atomics).
+// Bits on which all keys agree are decided without counting, and the search
+// stops once exactly topk keys are >= T.  Every key above T is taken, then
+// the keys equal to T in ascending tile order until topk are taken (ties go
+// to the lower tile index); indices are written in ascending order.  Order
+// keys of finite scores are never 0, so 0 marks padding slots.
+template <int MAXE>
+__device__ __forceinline__ void bsearch_topk_row(const uint32_t* kr, int nT, int topk, int32_t* out) {
   const int lane = threadIdx.x % 32;
   const uint32_t lt_mask = (1u << lane) - 1u;
-  uint32_t key[NR][MAXE];
-  uint32_t T[NR];
-  int bit[NR];
+  uint32_t key[MAXE];
+  uint32_t kand = 0xffffffffu, kor = 0u;
 #pragma unroll
-  for (int r = 0; r < NR; ++r) {
-    uint32_t kand = 0xffffffffu, kor = 0u;
-#pragma unroll
-    for (int e = 0; e < MAXE; ++e) {
-      const int j = lane + 32 * e;
-      key[r][e] = (r < nrow && j < nT) ? kr[r * kst + j] : 0u;
-      if (j < nT) {
-        kand &= key[r][e];
-        kor |= key[r][e];
-      }
-    }
-    kand = __reduce_and_sync(0xffffffffu, kand);
-    kor = __reduce_or_sync(0xffffffffu, kor);
-    const int common = __clz(kand ^ kor);        // leading bits shared by all keys (32: all equal)
-    T[r] = common == 0 ? 0u : (kand & (0xffffffffu << (32 - common)));
-    bit[r] = r < nrow ? 31 - common : -1;        // next bit to decide; -1: done
-  }
-  for (;;) {
-    bool any = false;
-    uint32_t c[NR];
-#pragma unroll
-    for (int r = 0; r < NR; ++r) {
-      c[r] = 0;
-      if (bit[r] >= 0) {
-        any = true;
-        const uint32_t cand = T[r] | (1u << bit[r]);
-        uint32_t p[4] = {0u, 0u, 0u, 0u};   // four independent chains of adds
-#pragma unroll
-        for (int e = 0; e < MAXE; ++e) p[e & 3] += (key[r][e] >= cand) ? 1u : 0u;
-        c[r] = (p[0] + p[1]) + (p[2] + p[3]);
-      }
-    }
-    if (!any) break;
-#pragma unroll
-    for (int r = 0; r < NR; ++r) c[r] = __reduce_add_sync(0xffffffffu, c[r]);
-#pragma unroll
-    for (int r = 0; r < NR; ++r) {
-      if (bit[r] < 0) continue;
-      const uint32_t cand = T[r] | (1u << bit[r]);
-      --bit[r];
-      if (c[r] >= static_cast<uint32_t>(topk)) {
-        T[r] = cand;
-        // exactly topk keys are >= T: they are the answer whatever the lower bits
-        if (c[r] == static_cast<uint32_t>(topk)) bit[r] = -1;
-      }
+  for (int e = 0; e < MAXE; ++e) {
+    const int j = lane + 32 * e;
+    key[e] = (j < nT) ? kr[j] : 0u;
+    if (j < nT) {
+      kand &= key[e];
+      kor |= key[e];
     }
   }
+  kand = __reduce_and_sync(0xffffffffu, kand);
+  kor = __reduce_or_sync(0xffffffffu, kor);
+  const int common = __clz(kand ^ kor);          // leading bits shared by all keys (32: all equal)
+  uint32_t T = common == 0 ? 0u : (kand & (0xffffffffu << (32 - common)));
+  for (int b = 31 - common; b >= 0; --b) {
+    const uint32_t cand = T | (1u << b);
+    uint32_t p[4] = {0u, 0u, 0u, 0u};            // four independent chains of adds
 #pragma unroll
-  for (int r = 0; r < NR; ++r) {
-    if (r >= nrow) break;
-    uint32_t gt = 0;
-#pragma unroll
-    for (int e = 0; e < MAXE; ++e) gt += (key[r][e] > T[r]) ? 1u : 0u;
-    gt = __reduce_add_sync(0xffffffffu, gt);
-    const int want_eq = topk - static_cast<int>(gt);
-    int base = 0, eq_seen = 0;
-    int32_t* o = out + static_cast<size_t>(r) * topk;
-#pragma unroll
-    for (int e = 0; e < MAXE; ++e) {
-      if (32 * e >= nT) break;
-      const bool gtb = key[r][e] > T[r];
-      const bool eqb = key[r][e] == T[r];
-      const uint32_t eqm = __ballot_sync(0xffffffffu, eqb);
-      const bool take = gtb || (eqb && eq_seen + __popc(eqm & lt_mask) < want_eq);
-      const uint32_t tm = __ballot_sync(0xffffffffu, take);
-      if (take) o[base + __popc(tm & lt_mask)] = lane + 32 * e;
-      base += __popc(tm);
-      eq_seen += __popc(eqm);
+    for (int e = 0; e < MAXE; ++e) p[e & 3] += (key[e] >= cand) ? 1u : 0u;
+    const uint32_t c = __reduce_add_sync(0xffffffffu, (p[0] + p[1]) + (p[2] + p[3]));
+    if (c >= static_cast<uint32_t>(topk)) {
+      T = cand;
+      // exactly topk keys are >= T: they are the answer whatever the lower bits
+      if (c == static_cast<uint32_t>(topk)) break;
     }
+  }
+  uint32_t gt = 0;
+#pragma unroll
+  for (int e = 0; e < MAXE; ++e) gt += (key[e] > T) ? 1u : 0u;
+  gt = __reduce_add_sync(0xffffffffu, gt);
+  const int want_eq = topk - static_cast<int>(gt);
+  int base = 0, eq_seen = 0;
+#pragma unroll
+  for (int e = 0; e < MAXE; ++e) {
+    if (32 * e >= nT) break;
+    const bool gtb = key[e] > T;
+    const bool eqb = key[e] == T;
+    const uint32_t eqm = __ballot_sync(0xffffffffu, eqb);
+    const bool take = gtb || (eqb && eq_seen + __popc(eqm & lt_mask) < want_eq);
+    const uint32_t tm = __ballot_sync(0xffffffffu, take);
+    if (take) out[base + __popc(tm & lt_mask)] = lane + 32 * e;
+    base += __popc(tm);
+    eq_seen += __popc(eqm);
   }
 }
 
@@ -250,15 +218,15 @@ __device__ __forceinline__ void topk_rows(const uint32_t* keys, int kst, int nT,
     const uint32_t* kr = keys + r * kst;
     int32_t* out = out_rows + static_cast<size_t>(r) * topk;
     if (nT <= 32 * 8)
-      bsearch_topk_rows<8, 1>(kr, kst, 1, nT, topk, out);
+      bsearch_topk_row<8>(kr, nT, topk, out);
     else if (nT <= 32 * 12)
-      bsearch_topk_rows<12, 1>(kr, kst, 1, nT, topk, out);
+      bsearch_topk_row<12>(kr, nT, topk, out);
     else if (nT <= 32 * 16)
-      bsearch_topk_rows<16, 1>(kr, kst, 1, nT, topk, out);
+      bsearch_topk_row<16>(kr, nT, topk, out);
     else if (nT <= 32 * 24)
-      bsearch_topk_rows<24, 1>(kr, kst, 1, nT, topk, out);
+      bsearch_topk_row<24>(kr, nT, topk, out);
     else
-      bsearch_topk_rows<48, 1>(kr, kst, 1, nT, topk, out);
+      bsearch_topk_row<48>(kr, nT, topk, out);
   }
 }
 
