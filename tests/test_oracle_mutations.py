@@ -83,6 +83,7 @@ CASES = [
     ("attend_head", _attend_kv_with_query_tiles,
      lambda: pins.test_kv_grid_all_blocks_equals_dense(*pins.KV_CASES[0])),
     ("keep_prefix", _prefix_dropped, lambda: pins.test_prefix_blocks_always_kept(3, 5)),
+    ("bf16_to_f64", vo.f16_to_f64, lambda: pins.test_bf16_widening_textbook_values()),
 ]
 
 

@@ -299,6 +299,20 @@ def test_workload_table():
             assert vo.num_tiles(w.grid, w.tile) == 120 and w.topk in (8, 16, 32, 64, 120)
 
 
+def test_bf16_widening_textbook_values():
+    """bfloat16 encodings (the upper half of a float32): 1.0, -2.0, the largest
+    finite 0x7F7F = (2 - 2^-7) * 2^127, the smallest subnormal 2^-133, 1/3
+    rounded; and round-to-nearest-even when narrowing float32 to bfloat16."""
+    bits = np.array([0x3F80, 0xC000, 0x7F7F, 0x0001, 0x3EAB], dtype=np.uint16)
+    w = vo.bf16_to_f64(bits)
+    np.testing.assert_array_equal(w[:4], [1.0, -2.0, (2 - 2.0 ** -7) * 2.0 ** 127, 2.0 ** -133])
+    assert abs(w[4] - 1 / 3) < 2 ** -9
+    # 1 + 2^-8 lies halfway between 1 and 1 + 2^-7: ties round to the even one (1.0)
+    assert synth.f32_to_bf16_bits(np.array([1 + 2 ** -8], np.float32))[0] == 0x3F80
+    assert synth.f32_to_bf16_bits(np.array([1 + 3 * 2 ** -8], np.float32))[0] == 0x3F82
+    assert synth.f32_to_bf16_bits(np.array([-1.5], np.float32))[0] == 0xBFC0
+
+
 def test_f16_widening_textbook_values():
     """IEEE binary16 encodings: 1.0, -2.0, the largest finite 65504, the
     smallest subnormal 2^-24, and round-to-nearest-even at a tie."""
