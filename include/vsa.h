@@ -50,9 +50,11 @@
  * Supported: bf16 or fp16 inputs (O has the input type; pooling, scores,
  * softmax and accumulation are float32); d in {64, 128}; tile extents powers
  * of two with tt*th*tw in {64, 128, 256} (the guide's 4x4x4 = 64 and 4x8x8 =
- * 256 blocks), the same on both sides, and tt >= 2 when it is 256; H_q =
- * H_kv; non-causal attention, no mask.  Inputs must be finite (NaN/Inf give
- * unspecified results, never a fault).
+ * 256 blocks), the same volume on both sides, and tt >= 2 when it is 256;
+ * H_q = H_kv; non-causal attention, no mask.  Inputs must be finite (NaN/Inf
+ * give unspecified results, never a fault; in the [B, N, H, d] layout a box
+ * past the last frame reads the next batch's first frames and masks them,
+ * so those must be finite too).
  *
  * Ownership: the caller allocates every buffer (including the select
  * workspace); no call allocates device memory.  (The one piece of device
@@ -99,7 +101,9 @@ typedef struct vsa_shape {
 
 typedef enum vsa_status {
   VSA_OK = 0,
-  VSA_ERR_INVALID_ARG = 1,  /* NULL pointer, non-positive extent, bad scale    */
+  VSA_ERR_INVALID_ARG = 1,  /* NULL pointer, non-positive extent (incl. a key/
+                               value grid or tile given in part), bad scale,
+                               prefix_tiles outside [0, nTk]                    */
   VSA_ERR_TOPK_RANGE = 2,   /* topk <= 0, topk > nTk or topk < prefix_tiles
                                (guide: topk must be positive; topk >
                                num_blocks is invalid), or a sparsity outside
@@ -110,8 +114,9 @@ typedef enum vsa_status {
   VSA_ERR_WORKSPACE = 5,    /* workspace NULL or smaller than required         */
   VSA_ERR_ARCH = 6,         /* current device is not sm_100                    */
   VSA_ERR_CUDA = 7,         /* a CUDA runtime/driver call failed               */
-  VSA_ERR_TOO_LARGE = 8     /* more than 1536 tiles per head on a side, B*H > 65535, or
-                               (64-token tiles) topk too large for shared memory */
+  VSA_ERR_TOO_LARGE = 8     /* more than 1536 tiles per head on a side, B*H >
+                               65535, or (64-token tiles) topk too large for
+                               shared memory                                    */
 } vsa_status;
 
 /* Query tile count of a shape (FastVideo VSA guide, "Wan top-k behavior":
