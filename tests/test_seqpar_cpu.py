@@ -87,7 +87,7 @@ def _worker(rank, world, port, case, out):
 @pytest.mark.parametrize("case", sorted(CASES))
 def test_ulysses_equals_unsharded(case, world):
     B, H, grid, tile, topk, grid_k, d = CASES[case]
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_worker, args=(world, _free_port(), case, out), nprocs=world, join=True)
     q, k, v = _full(case)
