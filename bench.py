@@ -410,12 +410,18 @@ def run_ours(args, w, rank, world, device):
         "clocks": clk.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:
-        nt = nT                                   # one full head: ~10-30 s of CPU work
-        dt, fl = oracle_sample(head_bits(q, w), head_bits(k, w), head_bits(v, w), w, nt)
+        # whole heads (full selection + attention of every query tile) until
+        # about 10 s of CPU work, at most all heads of the workload
+        dt = fl = 0.0
+        heads = 0
+        while heads < w.B * w.H and (heads == 0 or dt < 10.0):
+            b, h = divmod(heads, w.H)
+            t, f = oracle_sample(head_bits(q, w, b, h), head_bits(k, w, b, h), head_bits(v, w, b, h), w, nT)
+            dt, fl, heads = dt + t, fl + f, heads + 1
         out["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
                                "kind": "oracle",
-                               "sample": f"one head: full tile selection + attention for {nt} of {nT} "
-                                         f"query tiles ({dt:.1f} s)"}
+                               "sample": f"{heads} of {w.B * w.H} heads, each a full tile selection + attention "
+                                         f"of all {nT} query tiles ({dt:.1f} s)"}
     return out
 
 
