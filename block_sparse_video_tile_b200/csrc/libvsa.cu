@@ -125,6 +125,26 @@ static int launch_score_wide(const Geom& gq, const Geom& gk, int topk, int32_t* 
              : VSA_ERR_CUDA;
 }
 
+template <int D, int KEYS, int STAGES>
+static int launch_score_narrow(const Geom& gq, const Geom& gk, int topk, int32_t* idx, const float* means,
+                               const cudaLaunchAttribute* attr, cudaStream_t st) {
+  const size_t smem = score_narrow_smem_bytes<D, KEYS, STAGES>(gk);
+  if (cudaFuncSetAttribute(score_topk_narrow_kernel<D, KEYS, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return VSA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ceil_div(gq.nT, kNarrowRows), gq.B * gq.H);
+  cfg.blockDim = dim3(kNarrowThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = const_cast<cudaLaunchAttribute*>(attr);
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, score_topk_narrow_kernel<D, KEYS, STAGES>, gq, gk, means, topk, idx) ==
+                 cudaSuccess
+             ? VSA_OK
+             : VSA_ERR_CUDA;
+}
+
 template <int D>
 static int launch_score(const Geom& gq, const Geom& gk, int topk, int32_t* idx, const float* means,
                         cudaStream_t st) {
@@ -135,20 +155,8 @@ static int launch_score(const Geom& gq, const Geom& gk, int topk, int32_t* idx, 
     return launch_score_wide<D, kWideStages>(gq, gk, topk, idx, means, attr, st);
   if (gk.nT > kWideMaxTiles && gk.nT <= kWideLongMaxTiles)
     return launch_score_wide<D, kWideStagesLong>(gq, gk, topk, idx, means, attr, st);
-  const size_t smem = score_narrow_smem_bytes<D>(gk);
-  if (cudaFuncSetAttribute(score_topk_narrow_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return VSA_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(ceil_div(gq.nT, kNarrowRows), gq.B * gq.H);
-  cfg.blockDim = dim3(kNarrowThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, score_topk_narrow_kernel<D>, gq, gk, means, topk, idx) == cudaSuccess
-             ? VSA_OK
-             : VSA_ERR_CUDA;
+  return gk.nT <= kShortKeys ? launch_score_narrow<D, kShortKeys, kShortStages>(gq, gk, topk, idx, means, attr, st)
+                             : launch_score_narrow<D, kNarrowKeys, kNarrowStages>(gq, gk, topk, idx, means, attr, st);
 }
 
 template <int D, bool F16>

@@ -362,30 +362,35 @@ inline size_t score_smem_bytes(const Geom& gk) {
 
 // Narrow kernel (heads of at most kNarrowMaxTiles tiles, and of more than
 // kWideLongMaxTiles, whose 32 key rows would not fit beside the wide ring): one
-// CTA per (block of 16 query tiles,
-// head), 8 warps; lane (qg, kg) of warp w holds the 4 x 4 block of query
-// tiles 4qg .. 4qg+3 x key tiles 32w + 4kg .. 32w + 4kg + 3 of a pass of 256
-// key tiles.  Key means stream in slices of 16 channels x 256 key tiles on a
-// 4-deep cp.async ring.  Same summation order and selection as the wide kernel.
-// Dynamic shared memory: qT [D][16] | ring [4][16][256] | keys [16][nT].
+// CTA per (block of 16 query tiles, head), 8 warps; lane (qg, kg) of warp w
+// holds the 4 x 4 block of query tiles 4qg .. 4qg+3 x key tiles 32w + 4kg ..
+// 32w + 4kg + 3 of a pass of KEYS key tiles (KEYS / 32 warps do the math).
+// Key means stream in slices of 16 channels x KEYS key tiles on a STAGES-deep
+// cp.async ring: 256-key passes on a 4-deep ring, or, for heads of at most
+// 128 tiles, 128-key passes on an 8-deep ring, so every slice of the single
+// pass is in flight at once (one L2 round trip instead of one per slice).
+// Same summation order and selection as the wide kernel.
+// Dynamic shared memory: qT [D][16] | ring [STAGES][16][KEYS] | keys [16][nT].
 constexpr int kNarrowRows = 16;
 constexpr int kNarrowKeys = 256;
 constexpr int kNarrowSlice = 16;
 constexpr int kNarrowStages = 4;
-constexpr int kNarrowMathWarps = 8;
+constexpr int kShortKeys = 128;       // heads of at most kShortKeys tiles
+constexpr int kShortStages = 8;
 constexpr int kNarrowThreads = 256;   // two CTAs per SM at small tile counts
 
-template <int D>
+template <int D, int KEYS, int STAGES>
 __global__ void __launch_bounds__(kNarrowThreads) score_topk_narrow_kernel(Geom gq, Geom gk, const float* __restrict__ means,
                                                                            int topk, int32_t* __restrict__ idx) {
   constexpr int SPP = D / kNarrowSlice;
-  constexpr int SLICE = kNarrowSlice * kNarrowKeys;
+  constexpr int SLICE = kNarrowSlice * KEYS;
+  constexpr int MW = KEYS / 32;             // math warps
   constexpr int R = kNarrowRows;
   asm volatile("griddepcontrol.wait;" ::: "memory");
   extern __shared__ __align__(16) unsigned char smem_raw[];
   float* qT = reinterpret_cast<float*>(smem_raw);
   float* ring = qT + D * R;
-  uint32_t* keys = reinterpret_cast<uint32_t*>(ring + kNarrowStages * SLICE);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(ring + STAGES * SLICE);
   const int nT = gk.nT;                     // key tiles (score columns, top-k candidates)
   const int ldq = means_ld(gq.nT), ldk = means_ld(nT);
   const int bh = blockIdx.y;
@@ -393,7 +398,7 @@ __global__ void __launch_bounds__(kNarrowThreads) score_topk_narrow_kernel(Geom 
   const int nrows = min(R, gq.nT - row0);
   const float* mq = means + means_offset(gq, gk, 0, bh);
   const float* mk = means + means_offset(gq, gk, 1, bh);
-  const int nstage = ceil_div(nT, kNarrowKeys) * SPP;
+  const int nstage = ceil_div(nT, KEYS) * SPP;
 
   for (int f = threadIdx.x; f < D * R / 4; f += kNarrowThreads) {
     const int c = f / (R / 4), r4 = f % (R / 4);
@@ -405,13 +410,13 @@ __global__ void __launch_bounds__(kNarrowThreads) score_topk_narrow_kernel(Geom 
   }
   auto issue = [&](int st) {
     if (st < nstage) {
-      const int kc0 = (st / SPP) * kNarrowKeys, c0 = (st % SPP) * kNarrowSlice;
-      float* dst = ring + (st % kNarrowStages) * SLICE;
+      const int kc0 = (st / SPP) * KEYS, c0 = (st % SPP) * kNarrowSlice;
+      float* dst = ring + (st % STAGES) * SLICE;
       for (int f = threadIdx.x; f < SLICE / 4; f += kNarrowThreads) {
-        const int c = f / (kNarrowKeys / 4), k4 = f % (kNarrowKeys / 4);
+        const int c = f / (KEYS / 4), k4 = f % (KEYS / 4);
         const int key = kc0 + 4 * k4;
         const bool in = key < ldk;
-        cp_async16(smem_u32(dst + c * kNarrowKeys + 4 * k4),
+        cp_async16(smem_u32(dst + c * KEYS + 4 * k4),
                    in ? static_cast<const void*>(mk + static_cast<size_t>(c0 + c) * ldk + key)
                       : static_cast<const void*>(mk),
                    in ? 16u : 0u);
@@ -420,7 +425,7 @@ __global__ void __launch_bounds__(kNarrowThreads) score_topk_narrow_kernel(Geom 
     cp_async_commit();
   };
 #pragma unroll
-  for (int st = 0; st < kNarrowStages - 1; ++st) issue(st);
+  for (int st = 0; st < STAGES - 1; ++st) issue(st);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int qg = lane / 8, kg = lane % 8;
@@ -430,17 +435,17 @@ __global__ void __launch_bounds__(kNarrowThreads) score_topk_narrow_kernel(Geom 
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
   for (int st = 0; st < nstage; ++st) {
-    cp_async_wait<kNarrowStages - 2>();
+    cp_async_wait<STAGES - 2>();
     __syncthreads();
-    issue(st + kNarrowStages - 1);
+    issue(st + STAGES - 1);
     const int sl = st % SPP;
-    const float* kb = ring + (st % kNarrowStages) * SLICE + 32 * (warp % kNarrowMathWarps) + 4 * kg;
+    const float* kb = ring + (st % STAGES) * SLICE + 32 * (warp % MW) + 4 * kg;
     const float* qb = qT + sl * kNarrowSlice * R + 4 * qg;
-    if (warp < kNarrowMathWarps) {
+    if (warp < MW) {
 #pragma unroll
       for (int c = 0; c < kNarrowSlice; ++c) {
         const float4 qv = *reinterpret_cast<const float4*>(qb + c * R);
-        const float4 kv = *reinterpret_cast<const float4*>(kb + c * kNarrowKeys);
+        const float4 kv = *reinterpret_cast<const float4*>(kb + c * KEYS);
         const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
         const float ka[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
@@ -449,8 +454,8 @@ __global__ void __launch_bounds__(kNarrowThreads) score_topk_narrow_kernel(Geom 
           for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(qa[i], ka[j], acc[i][j]);
       }
     }
-    if (sl == SPP - 1 && warp < kNarrowMathWarps) {
-      const int kc0 = (st / SPP) * kNarrowKeys + 32 * warp + 4 * kg;
+    if (sl == SPP - 1 && warp < MW) {
+      const int kc0 = (st / SPP) * KEYS + 32 * warp + 4 * kg;
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -466,9 +471,9 @@ __global__ void __launch_bounds__(kNarrowThreads) score_topk_narrow_kernel(Geom 
   topk_rows(keys, nT, nT, nrows, topk, idx + (static_cast<size_t>(bh) * gq.nT + row0) * topk, kNarrowThreads / 32);
 }
 
-template <int D>
+template <int D, int KEYS, int STAGES>
 inline size_t score_narrow_smem_bytes(const Geom& gk) {
-  return sizeof(float) * (static_cast<size_t>(D) * kNarrowRows + kNarrowStages * kNarrowSlice * kNarrowKeys) +
+  return sizeof(float) * (static_cast<size_t>(D) * kNarrowRows + STAGES * kNarrowSlice * KEYS) +
          sizeof(uint32_t) * static_cast<size_t>(kNarrowRows) * gk.nT;
 }
 

@@ -218,10 +218,13 @@ def test_forward_with_sparsity():
     gu.check_selection(idx.cpu().numpy(), gu.oracle_scores(q, k, w), topk)
 
 
-# Heads of 257..768 key tiles take the wide score kernel with a 3-deep ring,
-# 769..1024 with a 2-deep one, larger ones the narrow kernel, up to the
-# 1536-tile limit; ragged on every axis.
+# Score kernel per head size: up to 128 key tiles the narrow kernel with
+# 128-key passes (the small cases and Wan-5B), 129..256 with 256-key passes,
+# 257..768 the wide kernel with a 3-deep ring, 769..1024 with a 2-deep one,
+# larger ones the narrow kernel again, up to the 1536-tile limit; ragged on
+# every axis.
 MANY_TILES = [
+    Workload("tiles150", 1, 2, (10, 19, 40), 64, (4, 4, 4), 20, "field"),
     Workload("tiles768", 1, 1, (15, 47, 63), 64, (4, 4, 4), 48, "field"),
     Workload("tiles960", 1, 2, (19, 45, 62), 64, (4, 4, 4), 60, "field"),
     Workload("tiles1024", 1, 1, (15, 61, 62), 128, (4, 4, 4), 64, "field"),
