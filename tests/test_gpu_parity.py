@@ -62,6 +62,13 @@ SMALL = [
     Workload("h3_prefix_bnhd", 2, 2, (8, 12, 16), 64, (4, 4, 4), 12, grid_k=(12, 12, 16), prefix_tiles=12,
              layout="bnhd"),
     Workload("prefix_self", 1, 2, (9, 20, 20), 128, (4, 8, 8), 12, "field", prefix_tiles=9),
+    # options combined: fp16, [B, N, H, d], own key/value grid and tile, prefix tiles
+    Workload("combo_f16_shared", 2, 2, (9, 20, 20), 128, (4, 8, 8), 8, "field", dtype="f16", layout="bnhd",
+             grid_k=(10, 18, 30), tile_k=(2, 8, 16), prefix_tiles=4),
+    Workload("combo_f16_pair", 1, 3, (6, 10, 14), 64, (4, 4, 4), 9, "field", dtype="f16", layout="bnhd",
+             grid_k=(7, 12, 9), tile_k=(2, 4, 8), prefix_tiles=9),
+    Workload("combo_tile_d64", 2, 2, (6, 12, 20), 64, (2, 8, 8), 5, grid_k=(5, 9, 26), tile_k=(4, 4, 8),
+             prefix_tiles=2),
 ]
 BY_NAME = {w.name: w for w in SMALL}
 
