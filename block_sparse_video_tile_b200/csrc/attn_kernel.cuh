@@ -355,9 +355,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                              static_cast<uint32_t>(c.by) | (static_cast<uint32_t>(c.bx) << 16));
   }
   if (threadIdx.x == 0) {
+    // MODE_SHARED: each active slot's issuer releases every K/V stage and drains
+    const uint32_t n_issuers = SHARED ? static_cast<uint32_t>(last_active + 1) : 1u;
     for (int b = 0; b < L::kNumBars; ++b) {
       const bool p_bar = (b == BAR_P_FULL || b == BAR_P_FULL + 1);
-      mbar_init(bar(b), p_bar ? 128u : 1u);
+      const bool shared_bar = b == BAR_K_EMPTY || b == BAR_K_EMPTY + 1 || b == BAR_V_EMPTY ||
+                              b == BAR_V_EMPTY + 1 || b == BAR_DRAIN;
+      mbar_init(bar(b), p_bar ? 128u : (shared_bar ? n_issuers : 1u));
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -470,11 +474,100 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_wait(bar((kv == 0 ? BAR_K_FULL : BAR_V_FULL) + st), last_use[kv][st] & 1, nullptr, a.err);
     }
     __syncwarp();
-  } else if (warp == 9) {
-    // ====================================================== MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_f16kind_f32(kSlotRows, kSubRows, false, F16);
-      constexpr uint32_t idPV = idesc_f16kind_f32(kSlotRows, D, true, F16);
+  } else if (warp == 9 || (SHARED && warp == 10)) {
+    // ====================================================== MMA issuer(s)
+    constexpr uint32_t idS = idesc_f16kind_f32(kSlotRows, kSubRows, false, F16);
+    constexpr uint32_t idPV = idesc_f16kind_f32(kSlotRows, D, true, F16);
+    // Operand descriptors.  MODE_SHARED holds three and adds (byte offset >>
+    // 4): the address field keeps shared-memory addresses >> 4 in 14 bits,
+    // and every address here is 16-byte aligned and below 256 KB, so the sum
+    // never carries out of it (2 % faster there; the other modes have no
+    // registers to spare and build each descriptor in place).
+    const uint64_t dQ = smem_desc_sw128(sQ, 16, 1024);
+    const uint64_t dK = smem_desc_sw128(sK, 16, 1024);
+    const uint64_t dV = smem_desc_sw128(sV, L::kSlabBytes, 1024);
+    auto desc_qk = [&](uint64_t d0, uint32_t s0, int buf, int kk) -> uint64_t {
+      const int sl = kk / 4, koff = (kk % 4) * 32;        // 16 channels = 32 B within a 64-channel slab
+      const uint32_t off = static_cast<uint32_t>(buf * L::kBufBytes + sl * L::kSlabBytes + koff);
+      return SHARED ? d0 + (off >> 4) : smem_desc_sw128(s0 + off, 16, 1024);
+    };
+    auto issue_pv = [&](int h, int vst, bool acc) {
+      const uint32_t tS = tmem + 128u * h, tO = tmem + 256u + 128u * h;
+#pragma unroll
+      for (int kk = 0; kk < kSubRows / 16; ++kk) {        // 16 keys = 16 rows of 128 B
+        const uint32_t off = static_cast<uint32_t>(vst * L::kBufBytes + kk * 2048);
+        const uint64_t bd = SHARED ? dV + (off >> 4) : smem_desc_sw128(sV + off, L::kSlabBytes, 1024);
+        mma_ts(tO, tS + 8u * kk, bd, idPV, (acc || kk > 0) ? 1u : 0u);
+      }
+    };
+    auto issue_s = [&](int h, int kst) {
+      const uint32_t tS = tmem + 128u * h;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk)
+        mma_ss(tS, desc_qk(dQ, sQ, h, kk), desc_qk(dK, sK, kst, kk), idS, kk > 0 ? 1u : 0u);
+    };
+
+    if (SHARED) {
+      // One issuer warp per slot (warp 9 + h), whole warp in the loop (waits,
+      // counters and descriptors are warp-uniform), one elected lane issuing
+      // each group and its commits (a commit tracks the MMAs of the thread
+      // that issued them; the warp is converged at every election, so it is
+      // always the same lane).  After a thread queues MMAs, its own next
+      // shared-memory access -- a barrier test included -- waits until that
+      // queue has nearly drained, so a single issuer for both slots would see
+      // slot 1's P only when slot 0's S is almost done and leave the tensor
+      // pipe idle while it catches up.  Here each warp tests its own slot's
+      // barriers with an empty queue.  The two warps pass a token through
+      // named barriers 1 and 2 (which do not wait for the MMA queue), so the
+      // groups still enter the pipe in the order PV_0, S_0, PV_1, S_1: groups
+      // of two issuers left free to interleave finish later for both slots.
+      // Both warps take the same n + 1 token steps whatever happens (a failed
+      // wait only skips the MMAs), so neither can be left at a named barrier.
+      const int h = warp - 9;
+      if (slot[h].active) {
+        KvSeq<MODE, SAME> sq;
+        sq.init(a, tile_tab, slot[h].bh, slot[h].tile, unions + h * 2 * a.topk, union_len[h]);
+        const int n = sq.count(a);                     // the same for both slots: one query tile
+        const bool token = last_active == 1;           // two issuers
+        bool ok = __all_sync(0xffffffffu, mbar_wait(bar(BAR_Q_FULL + h), 0, abort_flag, a.err));
+        for (int it = 0; it <= n; ++it) {
+          if (token) {
+            if (h == 1) named_bar_sync(1, 64);
+            else if (it > 0) named_bar_sync(2, 64);
+          }
+          const int kst = it & 1, kpar = (it >> 1) & 1;
+          const int vst = (it - 1) & 1, vpar = ((it - 1) >> 1) & 1;
+          if (ok && it < n) ok = __all_sync(0xffffffffu, mbar_wait(bar(BAR_K_FULL + kst), kpar, abort_flag, a.err));
+          if (ok && it > 0)
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(BAR_P_FULL + h), (it - 1) & 1, abort_flag, a.err) &&
+                                             mbar_wait(bar(BAR_V_FULL + vst), vpar, abort_flag, a.err));
+          if (ok) {
+            tc_fence_after();
+            if (elect_one_sync()) {
+              if (it > 0) {
+                issue_pv(h, vst, it - 1 > 0);
+                mma_commit(bar(it == n ? BAR_O_FULL + h : BAR_V_EMPTY + vst));
+              }
+              if (it < n) {
+                issue_s(h, kst);
+                mma_commit(bar(BAR_S_FULL + h));
+                mma_commit(bar(BAR_K_EMPTY + kst));
+              }
+            }
+            __syncwarp();
+          }
+          if (token) named_bar_arrive(h == 0 ? 1 : 2, 64);
+        }
+        if (token && h == 0) named_bar_sync(2, 64);    // warp 10's last arrival
+        // Drain: every MMA of both issuers has finished before TMEM is freed.
+        if (elect_one_sync()) mma_commit(bar(BAR_DRAIN));
+        __syncwarp();
+        mbar_wait(bar(BAR_DRAIN), 0, nullptr, a.err);
+      }
+    } else if (lane == 0) {
+      // MODE_TILE and MODE_PAIR: one single-lane issuer for both slots (the
+      // whole-warp form measured 7-14 % slower in MODE_TILE and no faster in
+      // MODE_PAIR).
       int n[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -487,25 +580,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int h = 0; h < 2; ++h)
         if (ok && slot[h].active) ok = mbar_wait(bar(BAR_Q_FULL + h), 0, abort_flag, a.err);
 
-      auto issue_pv = [&](int h, int vst, bool acc) {
-        const uint32_t tS = tmem + 128u * h, tO = tmem + 256u + 128u * h;
-#pragma unroll
-        for (int kk = 0; kk < kSubRows / 16; ++kk) {
-          const uint64_t bd = smem_desc_sw128(sV + vst * L::kBufBytes + kk * 2048, L::kSlabBytes, 1024);
-          mma_ts(tO, tS + 8u * kk, bd, idPV, (acc || kk > 0) ? 1u : 0u);
-        }
-      };
-      auto issue_s = [&](int h, int kst) {
-        const uint32_t tS = tmem + 128u * h;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int sl = kk / 4, koff = (kk % 4) * 32;
-          const uint64_t ad = smem_desc_sw128(sQ + h * L::kBufBytes + sl * L::kSlabBytes + koff, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sK + kst * L::kBufBytes + sl * L::kSlabBytes + koff, 16, 1024);
-          mma_ss(tS, ad, bd, idS, kk > 0 ? 1u : 0u);
-        }
-      };
-
       // iteration it of slot h: PV_h(it-1) then S_h(it); one step past the
       // slot's last sub-block, only the final PV and the O_FULL commit.
       const int n_max = max(n[0], n[1]);
@@ -513,26 +587,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           if (!ok || !slot[h].active || it > n[h]) continue;
-          const int kst = SHARED ? (it & 1) : h;
-          const int kpar = SHARED ? ((it >> 1) & 1) : (it & 1);
-          if (it < n[h] && !mbar_wait(bar(BAR_K_FULL + kst), kpar, abort_flag, a.err)) { ok = false; continue; }
+          const int kst = h, kpar = it & 1;
+          if (it < n[h] && !mbar_wait(bar(BAR_K_FULL + kst), kpar, abort_flag, a.err)) {
+            ok = false;
+            continue;
+          }
           if (it > 0) {
-            const int vst = SHARED ? ((it - 1) & 1) : h;
-            const int vpar = SHARED ? (((it - 1) >> 1) & 1) : ((it - 1) & 1);
+            const int vst = h, vpar = (it - 1) & 1;
             if (!mbar_wait(bar(BAR_P_FULL + h), (it - 1) & 1, abort_flag, a.err) ||
-                !mbar_wait(bar(BAR_V_FULL + vst), vpar, abort_flag, a.err)) { ok = false; continue; }
+                !mbar_wait(bar(BAR_V_FULL + vst), vpar, abort_flag, a.err)) {
+              ok = false;
+              continue;
+            }
             tc_fence_after();
             issue_pv(h, vst, it - 1 > 0);
             if (it == n[h]) {
               mma_commit(bar(BAR_O_FULL + h));
               continue;
             }
-            if (!SHARED || h == last_active) mma_commit(bar(BAR_V_EMPTY + vst));
+            mma_commit(bar(BAR_V_EMPTY + vst));
           }
           tc_fence_after();
           issue_s(h, kst);
           mma_commit(bar(BAR_S_FULL + h));
-          if (!SHARED || h == last_active) mma_commit(bar(BAR_K_EMPTY + kst));
+          mma_commit(bar(BAR_K_EMPTY + kst));
         }
       }
       // Drain: every MMA issued above has finished before TMEM is freed.

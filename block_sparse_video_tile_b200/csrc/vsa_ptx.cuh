@@ -59,6 +59,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Named CTA barriers (ids 1..15; 0 is __syncthreads): `count` threads, a
+// multiple of 32, arrive in whole warps.  bar.sync waits, bar.arrive does not.
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void named_bar_arrive(int id, int count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Bounded wait for the phase with the given parity to complete.  `abort` is a
 // CTA-shared flag (or nullptr): once any role has given up, the others stop
 // waiting too.  Returns false on timeout or abort (and records the timeout in
@@ -146,6 +155,18 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// True in exactly one lane of a converged warp (the lowest active lane, so
+// the same lane at every call while all 32 lanes are active).
+__device__ __forceinline__ bool elect_one_sync() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
 }
 
 // Arrive once on `bar` when every tcgen05 operation this thread issued so far
