@@ -338,8 +338,11 @@ def run_ours(args, w, rank, world, device):
     ms = start.elapsed_time(end)
     if api.device_error() != 0:
         raise RuntimeError("device error during the timed region")
-    sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    att_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    # per-phase split: median over the timed steps (the first step's select
+    # also holds the host's launch latency while the device waits for it; the
+    # whole-step figure above counts everything)
+    sel_ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+    att_ms = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
 
     # end to end through the public host-to-host API (api.forward_host): the
     # timed region holds the uploads of Q, K, V from pinned host memory, the
