@@ -20,16 +20,19 @@
 //     video keep mostly the same tiles, so most of each 128-row MMA is useful
 //     work; at worst (disjoint lists) it is half, as with one padded tile.
 // Warp roles (384 threads): warps 0-3 softmax slot 0, warps 4-7 softmax slot 1
-// (thread = query row = TMEM lane), warp 8 TMA producer, warp 9 MMA issuer,
-// warps 10-11 idle (in MODE_PAIR they build the union lists first).  The
-// producer warpgroup gives registers to the softmax warpgroups (setmaxnreg,
-// RegSplit: 208/88, or 200/96 in MODE_PAIR, within the launch's 384*168).
+// (thread = query row = TMEM lane); warp 9 + h issues slot h's MMAs; warp 8
+// is the TMA producer (for both slots in MODE_SHARED, whose slots share one
+// K/V stream; for slot 0 otherwise, with warp 11 producing slot 1), and in
+// MODE_PAIR warps 10-11 first build the union lists.  The producer warpgroup
+// gives registers to the softmax warpgroups (setmaxnreg, RegSplit: 208/88, or
+// 200/96 in MODE_PAIR, within the launch's 384*168).
 // TMEM (512 columns): S_h at [128h, 128h+128), P_h (16-bit pairs) aliases the
-// first 64 columns of S_h, O_h at [256 + 128h, ...).  The MMA warp issues, per
-// K/V sub-block: PV_0(prev), S_0(cur), PV_1(prev), S_1(cur); tcgen05.mma ops
-// from one thread execute in issue order, so S_h(cur) overwrites P_h(prev)
-// only after PV_h(prev) has read it, and softmax h works while the tensor
-// pipe runs the other slot.  Online softmax in float32 with lazy rescaling (O
+// first 64 columns of S_h, O_h at [256 + 128h, ...).  Per K/V sub-block the
+// MMA groups enter the tensor pipe in the order PV_0(prev), S_0(cur),
+// PV_1(prev), S_1(cur) (the two issuers pass a token); one thread issues a
+// slot's MMAs, and tcgen05.mma ops from one thread execute in issue order, so
+// S_h(cur) overwrites P_h(prev) only after PV_h(prev) has read it, and
+// softmax h works while the tensor pipe runs the other slot.  Online softmax in float32 with lazy rescaling (O
 // and l are only rescaled when the running max grows by more than 2^8).
 #pragma once
 
@@ -356,12 +359,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   if (threadIdx.x == 0) {
     // MODE_SHARED: each active slot's issuer releases every K/V stage and drains
-    const uint32_t n_issuers = SHARED ? static_cast<uint32_t>(last_active + 1) : 1u;
+    const uint32_t n_issuers = static_cast<uint32_t>(last_active + 1);
     for (int b = 0; b < L::kNumBars; ++b) {
       const bool p_bar = (b == BAR_P_FULL || b == BAR_P_FULL + 1);
-      const bool shared_bar = b == BAR_K_EMPTY || b == BAR_K_EMPTY + 1 || b == BAR_V_EMPTY ||
-                              b == BAR_V_EMPTY + 1 || b == BAR_DRAIN;
-      mbar_init(bar(b), p_bar ? 128u : (shared_bar ? n_issuers : 1u));
+      const bool kv_bar = b == BAR_K_EMPTY || b == BAR_K_EMPTY + 1 || b == BAR_V_EMPTY || b == BAR_V_EMPTY + 1;
+      mbar_init(bar(b), p_bar ? 128u : ((b == BAR_DRAIN || (SHARED && kv_bar)) ? n_issuers : 1u));
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -407,12 +409,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (warp >= 8) {
     setmaxnreg_dec<RegSplit<MODE>::kProducer>();
   }
-  if (warp == 8) {
-    // ====================================================== TMA producer
+  if (warp == 8 || (!SHARED && warp == 11)) {
+    // ====================================================== TMA producer(s)
+    // MODE_SHARED streams one K/V sequence for both slots (warp 8).  In
+    // MODE_TILE and MODE_PAIR each slot owns one K and one V stage and warp 8
+    // serves slot 0, warp 11 slot 1: with one producer for both, a slot's next
+    // K waited behind the other slot's V release (LongCat-like: the MMA issuer
+    // waited ~1300 clk for K after P was ready).
+    const int h_only = SHARED ? -1 : (warp == 8 ? 0 : 1);
     if (lane == 0) {
       bool ok = true;
       for (int h = 0; h < 2; ++h) {
-        if (!slot[h].active) continue;
+        if (!slot[h].active || (h_only >= 0 && h != h_only)) continue;
         const int nbox = (PAIR && slot[h].has_b) ? 2 : 1;
         mbar_arrive_expect_tx(bar(BAR_Q_FULL + h), static_cast<uint32_t>(nbox * L::kSlabs) * box_bytes);
         const BoxCoord ca = box_coord_l<BNHD>(g, slot[h].bh, slot[h].t0, slot[h].y0, slot[h].x0);
@@ -442,7 +450,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const int empty = kv == 0 ? BAR_K_EMPTY : BAR_V_EMPTY;
 #pragma unroll
           for (int h = 0; h < (SHARED ? 1 : 2); ++h) {
-            if (!ok || it >= n[h]) continue;
+            if (!ok || it >= n[h] || (h_only >= 0 && h != h_only)) continue;
             const int st = SHARED ? (it & 1) : h;
             const int use = SHARED ? (it >> 1) : it;
             if (use > 0 && !mbar_wait(bar(empty + st), (use - 1) & 1, abort_flag, a.err)) {
@@ -474,7 +482,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_wait(bar((kv == 0 ? BAR_K_FULL : BAR_V_FULL) + st), last_use[kv][st] & 1, nullptr, a.err);
     }
     __syncwarp();
-  } else if (warp == 9 || (SHARED && warp == 10)) {
+  } else if (warp == 9 || warp == 10) {
     // ====================================================== MMA issuer(s)
     constexpr uint32_t idS = idesc_f16kind_f32(kSlotRows, kSubRows, false, F16);
     constexpr uint32_t idPV = idesc_f16kind_f32(kSlotRows, D, true, F16);
@@ -507,36 +515,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mma_ss(tS, desc_qk(dQ, sQ, h, kk), desc_qk(dK, sK, kst, kk), idS, kk > 0 ? 1u : 0u);
     };
 
-    if (SHARED) {
-      // One issuer warp per slot (warp 9 + h), whole warp in the loop (waits,
-      // counters and descriptors are warp-uniform), one elected lane issuing
-      // each group and its commits (a commit tracks the MMAs of the thread
-      // that issued them; the warp is converged at every election, so it is
-      // always the same lane).  After a thread queues MMAs, its own next
-      // shared-memory access -- a barrier test included -- waits until that
-      // queue has nearly drained, so a single issuer for both slots would see
-      // slot 1's P only when slot 0's S is almost done and leave the tensor
-      // pipe idle while it catches up.  Here each warp tests its own slot's
-      // barriers with an empty queue.  The two warps pass a token through
-      // named barriers 1 and 2 (which do not wait for the MMA queue), so the
-      // groups still enter the pipe in the order PV_0, S_0, PV_1, S_1: groups
-      // of two issuers left free to interleave finish later for both slots.
-      // Both warps take the same n + 1 token steps whatever happens (a failed
-      // wait only skips the MMAs), so neither can be left at a named barrier.
+    // One issuer warp per slot (warp 9 + h), whole warp in the loop (waits,
+    // counters and descriptors are warp-uniform), one elected lane issuing
+    // each group and its commits (a commit tracks the MMAs of the thread that
+    // issued them; the warp is converged at every election, so it is always
+    // the same lane).  After a thread queues MMAs, its own next shared-memory
+    // access -- a barrier test included -- waits until that queue has nearly
+    // drained, so a single issuer for both slots would see slot 1's P only
+    // when slot 0's S is almost done and leave the tensor pipe idle while it
+    // catches up.  Here each warp tests its own slot's barriers with an empty
+    // queue.  The two warps pass a token through named barriers 1 and 2 (which
+    // do not wait for the MMA queue), so the groups still enter the pipe in
+    // the order PV_0, S_0, PV_1, S_1: groups of two issuers left free to
+    // interleave finish later for both slots.  Both warps take the same
+    // n_max + 1 token steps whatever happens (a failed wait, or a slot with
+    // fewer sub-blocks, only skips the MMAs), so neither can be left waiting
+    // at a named barrier.  In MODE_SHARED both issuers release each K/V stage
+    // (barrier count = active slots); otherwise a stage belongs to one slot.
+    {
       const int h = warp - 9;
+      int nn[2];
+#pragma unroll
+      for (int s2 = 0; s2 < 2; ++s2) {
+        KvSeq<MODE, SAME> sq2;
+        sq2.init(a, tile_tab, slot[s2].bh, slot[s2].tile, unions + s2 * 2 * a.topk, union_len[s2]);
+        nn[s2] = slot[s2].active ? sq2.count(a) : 0;
+      }
+      const int n = h ? nn[1] : nn[0];
+      const int n_max = max(nn[0], nn[1]);
       if (slot[h].active) {
-        KvSeq<MODE, SAME> sq;
-        sq.init(a, tile_tab, slot[h].bh, slot[h].tile, unions + h * 2 * a.topk, union_len[h]);
-        const int n = sq.count(a);                     // the same for both slots: one query tile
         const bool token = last_active == 1;           // two issuers
         bool ok = __all_sync(0xffffffffu, mbar_wait(bar(BAR_Q_FULL + h), 0, abort_flag, a.err));
-        for (int it = 0; it <= n; ++it) {
+        for (int it = 0; it <= n_max; ++it) {
           if (token) {
             if (h == 1) named_bar_sync(1, 64);
             else if (it > 0) named_bar_sync(2, 64);
           }
-          const int kst = it & 1, kpar = (it >> 1) & 1;
-          const int vst = (it - 1) & 1, vpar = ((it - 1) >> 1) & 1;
+          const int kst = SHARED ? (it & 1) : h, kpar = SHARED ? ((it >> 1) & 1) : (it & 1);
+          const int vst = SHARED ? ((it - 1) & 1) : h, vpar = SHARED ? (((it - 1) >> 1) & 1) : ((it - 1) & 1);
+          if (it > n) { if (token) named_bar_arrive(h == 0 ? 1 : 2, 64); continue; }
           if (ok && it < n) ok = __all_sync(0xffffffffu, mbar_wait(bar(BAR_K_FULL + kst), kpar, abort_flag, a.err));
           if (ok && it > 0)
             ok = __all_sync(0xffffffffu, mbar_wait(bar(BAR_P_FULL + h), (it - 1) & 1, abort_flag, a.err) &&
@@ -564,58 +581,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         __syncwarp();
         mbar_wait(bar(BAR_DRAIN), 0, nullptr, a.err);
       }
-    } else if (lane == 0) {
-      // MODE_TILE and MODE_PAIR: one single-lane issuer for both slots (the
-      // whole-warp form measured 7-14 % slower in MODE_TILE and no faster in
-      // MODE_PAIR).
-      int n[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        KvSeq<MODE, SAME> sq;
-        sq.init(a, tile_tab, slot[h].bh, slot[h].tile, unions + h * 2 * a.topk, union_len[h]);
-        n[h] = slot[h].active ? sq.count(a) : 0;
-      }
-      bool ok = true;
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-        if (ok && slot[h].active) ok = mbar_wait(bar(BAR_Q_FULL + h), 0, abort_flag, a.err);
-
-      // iteration it of slot h: PV_h(it-1) then S_h(it); one step past the
-      // slot's last sub-block, only the final PV and the O_FULL commit.
-      const int n_max = max(n[0], n[1]);
-      for (int it = 0; it <= n_max && ok; ++it) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (!ok || !slot[h].active || it > n[h]) continue;
-          const int kst = h, kpar = it & 1;
-          if (it < n[h] && !mbar_wait(bar(BAR_K_FULL + kst), kpar, abort_flag, a.err)) {
-            ok = false;
-            continue;
-          }
-          if (it > 0) {
-            const int vst = h, vpar = (it - 1) & 1;
-            if (!mbar_wait(bar(BAR_P_FULL + h), (it - 1) & 1, abort_flag, a.err) ||
-                !mbar_wait(bar(BAR_V_FULL + vst), vpar, abort_flag, a.err)) {
-              ok = false;
-              continue;
-            }
-            tc_fence_after();
-            issue_pv(h, vst, it - 1 > 0);
-            if (it == n[h]) {
-              mma_commit(bar(BAR_O_FULL + h));
-              continue;
-            }
-            mma_commit(bar(BAR_V_EMPTY + vst));
-          }
-          tc_fence_after();
-          issue_s(h, kst);
-          mma_commit(bar(BAR_S_FULL + h));
-          mma_commit(bar(BAR_K_EMPTY + kst));
-        }
-      }
-      // Drain: every MMA issued above has finished before TMEM is freed.
-      mma_commit(bar(BAR_DRAIN));
-      mbar_wait(bar(BAR_DRAIN), 0, nullptr, a.err);
     }
     __syncwarp();
   } else if (warp < 8) {
@@ -750,6 +715,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (!(hf ? use1 : use0)) {
 #pragma unroll
             for (int c = 32 * hf; c < 32 * hf + 32; ++c) s[c] = 0u;     // P = 0
+            tmem_st32(tS + 32u * hf, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * hf]));
             continue;
           }
 #pragma unroll
@@ -767,14 +733,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             ls2[c & 3] = f2_add(ls2[c & 3], f2_pack(p0, p1));
             s[c] = (kPackAlu && !F16) ? pack_bf16x2_alu(p0, p1) : pack_elem2<F16>(p0, p1);
           }
+          // store each half of P as soon as it is packed: the first store
+          // overlaps the second half's exponentials
+          tmem_st32(tS + 32u * hf, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * hf]));
         }
         {
           float a0, a1;
           f2_unpack(f2_add(f2_add(ls2[0], ls2[1]), f2_add(ls2[2], ls2[3])), a0, a1);
           l += a0 + a1;
         }
-        tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
         if (rescale) {
           // O_h is idle here: PV_h(it-1) completed before S_h(it) did, and
           // PV_h(it) waits for this slot's P_FULL arrival below.
