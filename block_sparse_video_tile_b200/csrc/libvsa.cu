@@ -106,11 +106,11 @@ static unsigned int* device_error_ptr() {
 // a 2-deep ring past kWideMaxTiles); smaller heads (little score work, more
 // CTAs) and larger ones (key rows that would not fit beside the wide ring)
 // take the narrow kernel (16).
-template <int D, int STAGES>
+template <int D, int STAGES, int KEYS>
 static int launch_score_wide(const Geom& gq, const Geom& gk, int topk, int32_t* idx, const float* means,
                              const cudaLaunchAttribute* attr, cudaStream_t st) {
-  const size_t smem = score_smem_bytes<D, STAGES>(gk);
-  if (cudaFuncSetAttribute(score_topk_kernel<D, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const size_t smem = score_smem_bytes<D, STAGES, KEYS>(gk);
+  if (cudaFuncSetAttribute(score_topk_kernel<D, STAGES, KEYS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return VSA_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
@@ -120,7 +120,7 @@ static int launch_score_wide(const Geom& gq, const Geom& gk, int topk, int32_t* 
   cfg.stream = st;
   cfg.attrs = const_cast<cudaLaunchAttribute*>(attr);
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, score_topk_kernel<D, STAGES>, gq, gk, means, topk, idx) == cudaSuccess
+  return cudaLaunchKernelEx(&cfg, score_topk_kernel<D, STAGES, KEYS>, gq, gk, means, topk, idx) == cudaSuccess
              ? VSA_OK
              : VSA_ERR_CUDA;
 }
@@ -151,10 +151,12 @@ static int launch_score(const Geom& gq, const Geom& gk, int topk, int32_t* idx, 
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
-  if (gk.nT > kNarrowMaxTiles && gk.nT <= kWideMaxTiles)
-    return launch_score_wide<D, kWideStages>(gq, gk, topk, idx, means, attr, st);
+  if (gk.nT > kNarrowMaxTiles && gk.nT <= kWideKeys)
+    return launch_score_wide<D, kWideStages, kWideKeys>(gq, gk, topk, idx, means, attr, st);
+  if (gk.nT > kWideKeys && gk.nT <= kWideMaxTiles)          // one pass, 12 math warps, 2-deep ring
+    return launch_score_wide<D, 2, kWideKeysOne>(gq, gk, topk, idx, means, attr, st);
   if (gk.nT > kWideMaxTiles && gk.nT <= kWideLongMaxTiles)
-    return launch_score_wide<D, kWideStagesLong>(gq, gk, topk, idx, means, attr, st);
+    return launch_score_wide<D, kWideStagesLong, kWideKeys>(gq, gk, topk, idx, means, attr, st);
   return gk.nT <= kShortKeys ? launch_score_narrow<D, kShortKeys, kShortStages>(gq, gk, topk, idx, means, attr, st)
                              : launch_score_narrow<D, kNarrowKeys, kNarrowStages>(gq, gk, topk, idx, means, attr, st);
 }

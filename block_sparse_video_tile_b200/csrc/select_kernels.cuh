@@ -244,21 +244,22 @@ __device__ __forceinline__ void topk_rows(const uint32_t* keys, int kst, int nT,
 // become order keys in shared memory, never written to HBM.
 // Dynamic shared memory: qT [D][32] | ring [STAGES][16][512] | keys [32][nT].
 constexpr int kWideRows = 32;
-constexpr int kWideKeys = 512;
+constexpr int kWideKeys = 512;        // key tiles per pass (8 math warps), heads of up to 512
+constexpr int kWideKeysOne = 768;     // one pass of 768 (12 math warps) for 513-768 key tiles
 constexpr int kWideSlice = 16;
 constexpr int kWideStages = 3;        // ring depth up to kWideMaxTiles key tiles
 constexpr int kWideStagesLong = 2;    // ring depth up to kWideLongMaxTiles (room for the key rows)
-constexpr int kWideMathWarps = 8;
-constexpr int kWideThreads = 512;     // warps 8-15 help only with copies and the top-k
+constexpr int kWideThreads = 512;     // warps past KEYS / 64 help only with copies and the top-k
 constexpr int kWideMaxTiles = 768;
 constexpr int kWideLongMaxTiles = 1024;
 constexpr int kNarrowMaxTiles = 256;   // below this the narrow kernel is used too (more, shorter CTAs)
 
-template <int D, int STAGES>
+template <int D, int STAGES, int KEYS>
 __global__ void __launch_bounds__(kWideThreads, 1) score_topk_kernel(Geom gq, Geom gk, const float* __restrict__ means, int topk,
                                                                   int32_t* __restrict__ idx) {
   constexpr int SPP = D / kWideSlice;      // stages per pass
-  constexpr int SLICE = kWideSlice * kWideKeys;
+  constexpr int SLICE = kWideSlice * KEYS;
+  constexpr int MW = KEYS / 64;            // math warps: 64 key tiles each
   constexpr int R = kWideRows;
   // the pooled means are written by the previous grid: wait for it
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -273,7 +274,7 @@ __global__ void __launch_bounds__(kWideThreads, 1) score_topk_kernel(Geom gq, Ge
   const int nrows = min(R, gq.nT - row0);
   const float* mq = means + means_offset(gq, gk, 0, bh);
   const float* mk = means + means_offset(gq, gk, 1, bh);
-  const int nstage = ceil_div(nT, kWideKeys) * SPP;
+  const int nstage = ceil_div(nT, KEYS) * SPP;
 
   // query means (joined to the first cp.async group); float4s past the row are zero
   for (int f = threadIdx.x; f < D * R / 4; f += kWideThreads) {
@@ -287,14 +288,14 @@ __global__ void __launch_bounds__(kWideThreads, 1) score_topk_kernel(Geom gq, Ge
   // stage st = (pass st / SPP, channel slice st % SPP) -> ring slot st % 3; one group per call
   auto issue = [&](int st) {
     if (st < nstage) {
-      const int kc0 = (st / SPP) * kWideKeys, c0 = (st % SPP) * kWideSlice;
+      const int kc0 = (st / SPP) * KEYS, c0 = (st % SPP) * kWideSlice;
       float* dst = ring + (st % STAGES) * SLICE;
 #pragma unroll 4
       for (int f = threadIdx.x; f < SLICE / 4; f += kWideThreads) {
-        const int c = f / (kWideKeys / 4), k4 = f % (kWideKeys / 4);
+        const int c = f / (KEYS / 4), k4 = f % (KEYS / 4);
         const int key = kc0 + 4 * k4;
         const bool in = key < ldk;
-        cp_async16(smem_u32(dst + c * kWideKeys + 4 * k4),
+        cp_async16(smem_u32(dst + c * KEYS + 4 * k4),
                    in ? static_cast<const void*>(mk + static_cast<size_t>(c0 + c) * ldk + key)
                       : static_cast<const void*>(mk),
                    in ? 16u : 0u);
@@ -318,16 +319,16 @@ __global__ void __launch_bounds__(kWideThreads, 1) score_topk_kernel(Geom gq, Ge
     __syncthreads();                 // slice st visible; slot of slice st-1 free
     issue(st + STAGES - 1);
     const int sl = st % SPP;
-    const int kw0 = (st / SPP) * kWideKeys + 64 * warp;   // the warp's first key tile
-    if (warp < kWideMathWarps && kw0 < nT) {
+    const int kw0 = (st / SPP) * KEYS + 64 * warp;   // the warp's first key tile
+    if (warp < MW && kw0 < nT) {
       const float* kb = ring + (st % STAGES) * SLICE + 64 * warp + 4 * kg;
       const float* qb = qT + sl * kWideSlice * R + 4 * qg;
 #pragma unroll
       for (int c = 0; c < kWideSlice; ++c) {
         const float4 q0 = *reinterpret_cast<const float4*>(qb + c * R);
         const float4 q1 = *reinterpret_cast<const float4*>(qb + c * R + 16);
-        const float4 k0 = *reinterpret_cast<const float4*>(kb + c * kWideKeys);
-        const float4 k1 = *reinterpret_cast<const float4*>(kb + c * kWideKeys + 32);
+        const float4 k0 = *reinterpret_cast<const float4*>(kb + c * KEYS);
+        const float4 k1 = *reinterpret_cast<const float4*>(kb + c * KEYS + 32);
         const float qa[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
         const float ka[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
 #pragma unroll
@@ -336,7 +337,7 @@ __global__ void __launch_bounds__(kWideThreads, 1) score_topk_kernel(Geom gq, Ge
           for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(qa[i], ka[j], acc[i][j]);
       }
     }
-    if (sl == SPP - 1 && warp < kWideMathWarps) {   // end of a pass: scores -> order keys
+    if (sl == SPP - 1 && warp < MW) {   // end of a pass: scores -> order keys
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int row = (i < 4 ? 0 : 16) + 4 * qg + (i & 3);
@@ -354,9 +355,9 @@ __global__ void __launch_bounds__(kWideThreads, 1) score_topk_kernel(Geom gq, Ge
   topk_rows(keys, nT, nT, nrows, topk, idx + (static_cast<size_t>(bh) * gq.nT + row0) * topk, kWideThreads / 32);
 }
 
-template <int D, int STAGES>
+template <int D, int STAGES, int KEYS>
 inline size_t score_smem_bytes(const Geom& gk) {
-  return sizeof(float) * (static_cast<size_t>(D) * kWideRows + STAGES * kWideSlice * kWideKeys) +
+  return sizeof(float) * (static_cast<size_t>(D) * kWideRows + STAGES * kWideSlice * KEYS) +
          sizeof(uint32_t) * static_cast<size_t>(kWideRows) * gk.nT;
 }
 

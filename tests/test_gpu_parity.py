@@ -29,6 +29,9 @@ SMALL = [
     Workload("ragged64", 1, 2, (6, 10, 14), 128, (4, 4, 4), 5),
     Workload("ragged64_d64", 1, 3, (5, 9, 11), 64, (4, 4, 4), 6),
     Workload("vol128", 2, 1, (6, 12, 20), 128, (2, 8, 8), 4),
+    # 128-token tiles, an odd count of (head, tile) units (3 heads x 9 tiles):
+    # the last CTA's second slot is empty and its MMA issuer runs alone
+    Workload("tile_odd", 1, 3, (6, 8, 24), 128, (2, 8, 8), 4),
     Workload("topk1", 1, 2, (9, 20, 20), 128, (4, 8, 8), 1),
     # 64-token tiles, odd tile count per head: the last pair has no tile B
     Workload("pair_odd", 1, 3, (4, 4, 20), 128, (4, 4, 4), 3),
