@@ -48,8 +48,9 @@ namespace vsa {
 constexpr int kAttnThreads = 384;        // 3 warpgroups
 // Registers per thread after setmaxnreg: warpgroups 0-1 (softmax) and 2 (TMA
 // and MMA warps).  2*128*S + 128*P must stay within the launch's 384*168.
-// MODE_PAIR's producer walks two union lists and its softmax has less to
-// hold, so it moves 8 registers to the producer (fewer spills, measured).
+// In MODE_PAIR the producer and issuer warps walk union lists (pieces with
+// membership flags) and the softmax has less to hold, so 8 registers move to
+// the producer warpgroup (fewer spills and faster, measured).
 template <int MODE>
 struct RegSplit {
   static constexpr int kSoftmax = MODE == 2 ? 200 : 208;
