@@ -106,3 +106,30 @@ def attend(Q, K, V, grid, tile, idx, scale):
             O[n] = [c / l for c in o]
             L[n] = m + math.log(l)
     return O, L
+
+
+def coarse(Q, K, V, grid, tile, scale):
+    """Tile-level attention: o_coarse per query block (list of lists)."""
+    bl = blocks(grid, tile)
+    qb = [mean_rows(Q, grid, toks) for toks in bl]
+    kb = [mean_rows(K, grid, toks) for toks in bl]
+    vb = [mean_rows(V, grid, toks) for toks in bl]
+    out = []
+    for i in range(len(bl)):
+        z = [scale * dot(qb[i], kb[j]) for j in range(len(bl))]
+        m = max(z)
+        w = [math.exp(v - m) for v in z]
+        l = sum(w)
+        out.append([sum(w[j] * vb[j][c] for j in range(len(bl))) / l for c in range(len(vb[0]))])
+    return out
+
+
+def gated(O, G, oc, grid, tile):
+    """O (dict or list by token) plus G[n] * oc[block of n], as a dict token -> list."""
+    T, Hh, W = grid
+    res = {}
+    for i, toks in enumerate(blocks(grid, tile)):
+        for t, y, x in toks:
+            n = (t * Hh + y) * W + x
+            res[n] = [O[n][c] + G[n][c] * oc[i][c] for c in range(len(oc[i]))]
+    return res

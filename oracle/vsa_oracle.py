@@ -45,6 +45,17 @@ What it computes, and where the pages fix each step:
    every query block's kept list whatever their scores (their scores count
    as +inf for the selection) and count toward topk; the other topk - P are
    the best-scoring of the rest.
+9. Pooled coarse branch (user guide, "Checkpoint behavior": checkpoints
+   that carry learned `to_gate_compress` weights add a gated compensation to
+   the sparse branch; without them the sparse branch runs alone).  The pages
+   name the branch but not its math -- parity unpinned by the pages.
+   Reading: attention at tile granularity.  Each query block's mean row
+   attends over every key/value block's mean row with the fine branch's
+   scale, softmax over all key/value blocks (each block one entry, whatever
+   its token count), values = the blocks' mean V rows; the result
+   o_coarse[i] is added to every token n of query block i through a gate
+   the caller supplies (the projection's output, same shape as O):
+   O[n] = O_sparse[n] + gate[n] * o_coarse[i].
 """
 from __future__ import annotations
 
@@ -252,3 +263,28 @@ def dense_bruteforce(Q, K, V, scale: float):
     e = np.exp(z - m)
     l = e.sum(axis=1, keepdims=True)
     return (e @ V) / l, (m + np.log(l))[:, 0]
+
+
+# ----------------------------------------------------------- coarse branch
+def coarse_head(Q, K, V, grid, tile, scale: float, grid_k=None, tile_k=None):
+    """Tile-level attention of one head (docstring step 9): o_coarse [nTq, d].
+
+    Q: [Nq, d], K, V: [Nk, d] float64; K and V pooled on grid_k / tile_k
+    (default the query's)."""
+    grid_k = grid if grid_k is None else grid_k
+    tile_k = tile if tile_k is None else tile_k
+    qbar, kbar, vbar = pool(Q, grid, tile), pool(K, grid_k, tile_k), pool(V, grid_k, tile_k)
+    z = scale * tile_scores(qbar, kbar)
+    m = z.max(axis=1, keepdims=True)
+    e = np.exp(z - m)
+    return (e @ vbar) / e.sum(axis=1, keepdims=True)
+
+
+def gated_output(O_sparse, gate, o_coarse, grid, tile):
+    """O_sparse + gate * o_coarse of each token's query block (docstring step 9).
+
+    O_sparse, gate: [Nq, d]; o_coarse: [nTq, d].  Returns a new [Nq, d] array."""
+    out = np.array(O_sparse, dtype=np.float64, copy=True)
+    for i, tok in enumerate(tile_tokens(grid, tile)):
+        out[tok] += gate[tok] * o_coarse[i]
+    return out

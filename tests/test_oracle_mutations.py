@@ -69,6 +69,35 @@ def _prefix_dropped(scores, prefix):
     return s
 
 
+def _coarse_unscaled(Q, K, V, grid, tile, scale, grid_k=None, tile_k=None):
+    return _orig_coarse(Q, K, V, grid, tile, 1.0, grid_k, tile_k)
+
+
+def _coarse_token_weighted(Q, K, V, grid, tile, scale, grid_k=None, tile_k=None):
+    """Softmax weights multiplied by each key block's token count."""
+    qbar, kbar, vbar = vo.pool(Q, grid, tile), vo.pool(K, grid, tile), vo.pool(V, grid, tile)
+    cnt = np.array([t.size for t in vo.tile_tokens(grid, tile)], dtype=np.float64)
+    z = scale * (qbar @ kbar.T)
+    e = np.exp(z - z.max(axis=1, keepdims=True)) * cnt[None, :]
+    return (e @ vbar) / e.sum(axis=1, keepdims=True)
+
+
+def _coarse_softmax_wrong_axis(Q, K, V, grid, tile, scale, grid_k=None, tile_k=None):
+    qbar, kbar, vbar = vo.pool(Q, grid, tile), vo.pool(K, grid, tile), vo.pool(V, grid, tile)
+    z = scale * (qbar @ kbar.T)
+    e = np.exp(z - z.max(axis=0, keepdims=True))
+    return (e @ vbar) / e.sum(axis=0, keepdims=True)
+
+
+_orig_coarse = vo.coarse_head
+
+
+def _gate_next_block(O, gate, oc, grid, tile):
+    return _orig_gated(O, gate, np.roll(oc, 1, axis=0), grid, tile)
+
+
+_orig_gated = vo.gated_output
+
 CASES = [
     ("pool", _zero_padded_pool, lambda: pins.test_pool_constant_per_block_partial_edges()),
     ("tile_scores", _transposed_scores, lambda: pins.test_scores_hand_example()),
@@ -84,6 +113,11 @@ CASES = [
      lambda: pins.test_kv_grid_all_blocks_equals_dense(*pins.KV_CASES[0])),
     ("keep_prefix", _prefix_dropped, lambda: pins.test_prefix_blocks_always_kept(3, 5)),
     ("bf16_to_f64", vo.f16_to_f64, lambda: pins.test_bf16_widening_textbook_values()),
+    ("coarse_head", _coarse_unscaled, lambda: pins.test_coarse_scale_matters()),
+    ("coarse_head", _coarse_token_weighted,
+     lambda: pins.test_coarse_uniform_keys_average_block_values(*pins.RAGGED_COARSE)),
+    ("coarse_head", _coarse_softmax_wrong_axis, lambda: pins.test_coarse_constant_values_pass_through()),
+    ("gated_output", _gate_next_block, lambda: pins.test_coarse_and_gate_vs_loops(*pins.RAGGED_COARSE)),
 ]
 
 

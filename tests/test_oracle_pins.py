@@ -425,3 +425,100 @@ def test_prefix_range_rejected():
     with pytest.raises(ValueError):
         vo.select_head(Q, Q, grid, tile, 8, prefix=9)       # prefix > nT
     assert vo.topk_from_sparsity(8, 0.99, prefix=3) == 3
+
+
+# ------------------------------------------------------------ coarse branch
+# The pooled coarse branch (FastVideo VSA user guide, "Checkpoint behavior":
+# a learned gate_compress compensation added to the sparse branch) has no
+# formula on the pages; the oracle's reading is tile-level attention over the
+# blocks' mean rows, added through a caller-given gate.  These pins fix that
+# reading by closed forms and by the pure-Python restatement.
+RAGGED_COARSE = ((5, 6, 7), (2, 4, 4))      # 3 x 2 x 2 blocks, partial on every axis
+
+
+def _block_means_loops(X, grid, tile):
+    """Mean rows of every block, from the pure-Python block lists."""
+    return np.array([loops.mean_rows(X.tolist(), grid, toks) for toks in loops.blocks(grid, tile)])
+
+
+@pytest.mark.parametrize("grid, tile", [(TINY.grid, TINY.tile), RAGGED_COARSE])
+def test_coarse_uniform_keys_average_block_values(grid, tile):
+    """All key blocks with the same mean (or a zero scale): every block gets
+    the same weight, so o_coarse is the plain average of the blocks' mean V
+    rows -- each partial block counting once, not by its token count."""
+    N = math.prod(grid)
+    Q, V = _rand((N, 8), 1), _rand((N, 8), 2)
+    K = np.tile(_rand((1, 8), 3), (N, 1))
+    expect = _block_means_loops(V, grid, tile).mean(axis=0)
+    oc = vo.coarse_head(Q, K, V, grid, tile, 0.7)
+    np.testing.assert_allclose(oc, np.broadcast_to(expect, oc.shape), rtol=0, atol=1e-12)
+    oc0 = vo.coarse_head(Q, _rand((N, 8), 4), V, grid, tile, 0.0)
+    np.testing.assert_allclose(oc0, np.broadcast_to(expect, oc0.shape), rtol=0, atol=1e-12)
+    if N % math.prod(tile):
+        # partial blocks: a zero-padded mean over the full block volume would differ
+        assert not np.allclose(expect, V.sum(axis=0) / (len(loops.blocks(grid, tile)) * math.prod(tile)))
+
+
+def test_coarse_dominant_block_selects_its_values():
+    """One key block whose mean points along every query mean, with a large
+    scale: its weight is 1 - O(nT e^-60), so o_coarse is that block's mean V."""
+    grid, tile = RAGGED_COARSE
+    N = math.prod(grid)
+    Q = np.zeros((N, 8))
+    Q[:, 0] = 1.0
+    K = np.zeros((N, 8))
+    star = 5
+    toks = loops.blocks(grid, tile)[star]
+    for t, y, x in toks:
+        K[(t * grid[1] + y) * grid[2] + x, 0] = 60.0
+    V = _rand((N, 8), 5)
+    oc = vo.coarse_head(Q, K, V, grid, tile, 1.0)
+    expect = _block_means_loops(V, grid, tile)[star]
+    np.testing.assert_allclose(oc, np.broadcast_to(expect, oc.shape), rtol=0, atol=1e-12)
+
+
+def test_coarse_constant_values_pass_through():
+    """V equal to one row c everywhere: the softmax weights sum to 1, so
+    o_coarse = c for every query block."""
+    grid, tile = RAGGED_COARSE
+    N = math.prod(grid)
+    c = _rand((1, 8), 6)
+    oc = vo.coarse_head(_rand((N, 8), 7), _rand((N, 8), 8), np.tile(c, (N, 1)), grid, tile, 0.9)
+    np.testing.assert_allclose(oc, np.broadcast_to(c, oc.shape), rtol=0, atol=1e-12)
+
+
+def test_coarse_scale_matters():
+    """The scale multiplies the tile scores before the softmax: a larger
+    scale sharpens the weights (an unscaled oracle would give equal outputs)."""
+    grid, tile = RAGGED_COARSE
+    N = math.prod(grid)
+    Q, K, V = _rand((N, 8), 9), _rand((N, 8), 10), _rand((N, 8), 11)
+    a = vo.coarse_head(Q, K, V, grid, tile, 0.1)
+    b = vo.coarse_head(Q, K, V, grid, tile, 10.0)
+    assert np.abs(a - b).max() > 1e-3
+
+
+@pytest.mark.parametrize("grid, tile", [(TINY.grid, TINY.tile), RAGGED_COARSE])
+def test_coarse_and_gate_vs_loops(grid, tile):
+    """NumPy coarse branch and gated output against the pure-Python
+    restatement (its own block lists, dot products and exp)."""
+    N = math.prod(grid)
+    d = 8
+    Q, K, V, G, O = (_rand((N, d), s) for s in (12, 13, 14, 15, 16))
+    oc = vo.coarse_head(Q, K, V, grid, tile, 0.35)
+    loc = loops.coarse(Q.tolist(), K.tolist(), V.tolist(), grid, tile, 0.35)
+    np.testing.assert_allclose(oc, np.array(loc), rtol=0, atol=1e-12)
+    out = vo.gated_output(O, G, oc, grid, tile)
+    lout = loops.gated(O.tolist(), G.tolist(), loc, grid, tile)
+    np.testing.assert_allclose(out, np.array([lout[n] for n in range(N)]), rtol=0, atol=1e-12)
+
+
+def test_gate_zero_is_identity_and_gate_is_linear():
+    grid, tile = RAGGED_COARSE
+    N = math.prod(grid)
+    O, G = _rand((N, 8), 17), _rand((N, 8), 18)
+    oc = _rand((len(loops.blocks(grid, tile)), 8), 19)
+    assert np.array_equal(vo.gated_output(O, np.zeros_like(G), oc, grid, tile), O)
+    one = vo.gated_output(O, G, oc, grid, tile) - O
+    two = vo.gated_output(O, 2 * G, oc, grid, tile) - O
+    np.testing.assert_allclose(two, 2 * one, rtol=0, atol=1e-12)
