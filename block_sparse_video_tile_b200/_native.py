@@ -17,7 +17,7 @@ STATUS = {
     4: "VSA_ERR_ALIGNMENT", 5: "VSA_ERR_WORKSPACE", 6: "VSA_ERR_ARCH", 7: "VSA_ERR_CUDA",
     8: "VSA_ERR_TOO_LARGE",
 }
-DEVERR = {0: "none", 1: "wait timeout", 2: "tile index out of range"}
+DEVERR = {0: "none", 1: "wait timeout", 2: "tile index out of range", 3: "kept list not strictly ascending"}
 
 EXPORTS = ("vsa_tile_count", "vsa_kv_tile_count", "vsa_topk_from_sparsity", "vsa_select_workspace_bytes",
            "vsa_select", "vsa_select_noalloc", "vsa_attn_fwd", "vsa_device_error", "vsa_status_string")

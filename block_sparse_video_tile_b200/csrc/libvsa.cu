@@ -93,10 +93,63 @@ static int check_arch() {
   return cached[dev] == 1 ? VSA_OK : VSA_ERR_ARCH;
 }
 
+// Device addresses of this library's __device__ arrays, looked up with
+// cudaGetSymbolAddress once per device and context and cached: a symbol's
+// address is fixed for the life of the context that loaded the module, and a
+// new context (after cudaDeviceReset, say) loads it again elsewhere, so the
+// cache is keyed by the context's process-unique id.  The driver calls are
+// reached through the runtime's entry-point query (no link against libcuda).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+static bool current_ctx_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (get_cur == nullptr || get_id == nullptr || get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+struct SymbolCache {
+  void* ptr[kMaxDevices] = {};
+  unsigned long long ctx[kMaxDevices] = {};
+  std::mutex mu;
+};
+
+// Address of `symbol` on the current device (its context is created by the
+// lookup if the runtime has not made one yet).
+static int symbol_address(const void* symbol, SymbolCache& c, void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VSA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return VSA_ERR_ARCH;
+  std::lock_guard<std::mutex> lock(c.mu);
+  unsigned long long id = 0;
+  if (c.ptr[dev] == nullptr || !current_ctx_id(&id) || id != c.ctx[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, symbol) != cudaSuccess || p == nullptr) return VSA_ERR_CUDA;
+    if (!current_ctx_id(&id)) return VSA_ERR_CUDA;
+    c.ptr[dev] = p;
+    c.ctx[dev] = id;
+  }
+  *out = c.ptr[dev];
+  return VSA_OK;
+}
+
 static unsigned int* device_error_ptr() {
+  static SymbolCache cache;
   void* p = nullptr;
-  if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-  return static_cast<unsigned int*>(p);
+  return symbol_address(&g_device_error, cache, &p) == VSA_OK ? static_cast<unsigned int*>(p) : nullptr;
 }
 
 // Score + top-k grid, launched as a programmatic dependent of the pooling
@@ -191,9 +244,9 @@ static int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     return VSA_ERR_CUDA;
   const long long BH = 1ll * a.gq.B * a.gq.H;
   long long grid;
-  if (MODE == MODE_SHARED) grid = BH * a.gq.nT;                            // one tile, two t-halves
-  else if (MODE == MODE_TILE) grid = (BH * a.gq.nT + 1) / 2;               // two tiles
-  else grid = (BH * ((a.gq.nT + 1) / 2) + 1) / 2;                          // two pairs of tiles
+  if (MODE == MODE_SHARED) grid = BH * a.gq.nT * 2;                        // a t-half of a tile
+  else if (MODE == MODE_TILE) grid = BH * a.gq.nT;                         // a tile
+  else grid = BH * ((a.gq.nT + 1) / 2);                                    // a pair of tiles
   attn_fwd_kernel<D, MODE, F16, SAME, BNHD><<<static_cast<unsigned>(grid), kAttnThreads, smem, st>>>(mq, mk, mv, a);
   return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
@@ -205,19 +258,11 @@ static int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
 static __device__ __align__(256) float g_select_scratch[VSA_SELECT_NOALLOC_SCRATCH_BYTES / sizeof(float)];
 
 static int select_scratch_ptr(float** out) {
-  static float* cached[kMaxDevices];
-  static std::mutex mu;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return VSA_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return VSA_ERR_ARCH;
-  std::lock_guard<std::mutex> lock(mu);
-  if (cached[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess || p == nullptr) return VSA_ERR_CUDA;
-    cached[dev] = static_cast<float*>(p);
-  }
-  *out = cached[dev];
-  return VSA_OK;
+  static SymbolCache cache;
+  void* p = nullptr;
+  const int rc = symbol_address(g_select_scratch, cache, &p);
+  *out = static_cast<float*>(p);
+  return rc;
 }
 
 // SAME: the key/value side has the query grid and tile (the kernel then

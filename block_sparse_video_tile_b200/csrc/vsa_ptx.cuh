@@ -106,14 +106,6 @@ __device__ __forceinline__ void tma_load_5d(uint32_t dst, const void* desc, uint
       : "memory");
 }
 
-// Contiguous global -> shared copy by the bulk-copy engine (addresses 16-byte
-// aligned, size a multiple of 16), completion counted on `bar` in bytes.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-               : "memory");
-}
-
 // ------------------------------------------------------------------ tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
@@ -313,17 +305,6 @@ __device__ __forceinline__ void setmaxnreg_inc() {
 template <int N>
 __device__ __forceinline__ void setmaxnreg_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-
-// Two non-negative finite float32 -> bf16x2 on the integer ALU: add half a
-// bf16 unit in the last place to the bits (a carry into the exponent rounds up
-// a binade) and keep the upper halves.  Equals round-to-nearest except at
-// exact ties, which round up.  Used for softmax probabilities, keeping the
-// conversion off the unit that evaluates the exponentials.
-__device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
-  const uint32_t a = __float_as_uint(lo) + 0x8000u;
-  const uint32_t b = __float_as_uint(hi) + 0x8000u;
-  return __byte_perm(a, b, 0x7632);
 }
 
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {

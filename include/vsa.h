@@ -59,12 +59,12 @@
  * Ownership: the caller allocates every buffer (including the select
  * workspace); no call allocates device memory.  (The one piece of device
  * memory the library owns is the fixed scratch array of vsa_select_noalloc,
- * reserved when the library is loaded.)  Calls are asynchronous
- * on `stream` (a cudaStream_t; NULL = legacy default stream).  Every call
- * checks its arguments before launching anything and returns a vsa_status;
- * nothing is launched on error.  Faults inside a kernel are reported through
- * vsa_device_error() (bounded waits in the kernels turn a stall into an error
- * code instead of a hang).
+ * reserved when the library's device code is first loaded on a GPU.)  Calls
+ * are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ * stream).  Every call checks its arguments before launching anything and
+ * returns a vsa_status; nothing is launched on error.  Faults inside a
+ * kernel are reported through vsa_device_error() (bounded waits in the
+ * kernels turn a stall into an error code instead of a hang).
  */
 #ifndef VSA_H_
 #define VSA_H_
@@ -161,22 +161,30 @@ int vsa_select(const vsa_shape* shape, const void* q, const void* k, int32_t top
  *
  * Same arguments and results as vsa_select, minus the workspace: the pooled
  * tile means live in a fixed scratch array inside the library
- * (VSA_SELECT_NOALLOC_SCRATCH_BYTES, allocated once per GPU when the library
- * loads and held until the process exits).  Meant for callers that must not
- * call cudaMalloc -- a host framework that owns all device memory through its
- * own pool, code running inside a region where allocation is forbidden, or a
- * plugin with no allocator handle.  This call itself allocates nothing (no
- * cudaMalloc, no cudaFree, no allocating library routine).
+ * (VSA_SELECT_NOALLOC_SCRATCH_BYTES per GPU, held until the process exits).
+ * Meant for callers that must not call cudaMalloc -- a host framework that
+ * owns all device memory through its own pool, code running inside a region
+ * where allocation is forbidden, or a plugin with no allocator handle.  This
+ * call itself allocates nothing (no cudaMalloc, no cudaFree, no allocating
+ * library routine).
+ *   - The scratch array is reserved when the library's device code is first
+ *     loaded on a GPU.  With CUDA's lazy module loading (the default) that
+ *     happens inside the first vsa_* call that touches the device, which may
+ *     be this one: make one call on each device early -- vsa_device_error
+ *     will do -- before a memory pool takes the device's memory and before
+ *     any CUDA stream capture.
  *   - The scratch needs vsa_select_workspace_bytes(shape) bytes (about
- *     2*B*H*nT*d*4); larger shapes are rejected with
- *     VSA_ERR_WORKSPACE before anything is launched.
+ *     2*B*H*nT*d*4); larger shapes are rejected with VSA_ERR_WORKSPACE before
+ *     anything is launched.
  *   - The first call on a device (with that device current) looks up the
- *     scratch array's device address; make that first call before any CUDA
- *     stream capture.
+ *     scratch array's device address (again after a cudaDeviceReset, which
+ *     makes a new context); make that first call before any stream capture.
  *   - Every call on a device shares the one scratch array: calls that can
  *     overlap on the GPU (different streams, no ordering) race and give
- *     wrong indices.  Nothing needs clearing between calls (each call
- *     overwrites every scratch element it reads).
+ *     wrong indices.  Nothing needs clearing between calls: every mean a
+ *     call uses is written by that call first (the score kernel also reads
+ *     the row padding past nT, left from earlier calls, but masks those
+ *     columns out).
  * Two kernel launches on `stream`. */
 #define VSA_SELECT_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 int vsa_select_noalloc(const vsa_shape* shape, const void* q, const void* k, int32_t topk,
@@ -187,9 +195,12 @@ int vsa_select_noalloc(const vsa_shape* shape, const void* q, const void* k, int
  * head_size ** -0.5 by default, non-causal, no mask).
  *   q, k, v       : device Q, K, V in shape->layout and shape->dtype, 16-byte
  *                   aligned
- *   idx           : device int32 [B, H, nTq, topk], ascending distinct tiles
+ *   idx           : device int32 [B, H, nTq, topk], strictly ascending tiles
  *                   (as vsa_select writes them); an entry outside [0, nTk)
- *                   raises a device error and is read as tile 0 instead
+ *                   sets VSA_DEVERR_BAD_INDEX and is read as tile 0 instead,
+ *                   a row that is not strictly ascending sets
+ *                   VSA_DEVERR_BAD_ORDER (the row is still attended, with an
+ *                   unspecified result); neither faults
  *   softmax_scale : > 0 and finite; pass d ** -0.5 for the standard scale
  *   o             : device O out, layout and type of q, 16-byte aligned
  *   lse           : device float32 [B, H, Nq] out, natural log
@@ -208,6 +219,8 @@ int vsa_device_error(uint32_t* code, int32_t reset);
 #define VSA_DEVERR_NONE 0u
 #define VSA_DEVERR_WAIT_TIMEOUT 1u   /* an mbarrier wait ran past its bound     */
 #define VSA_DEVERR_BAD_INDEX 2u      /* idx entry outside [0, nTk)             */
+#define VSA_DEVERR_BAD_ORDER 3u      /* idx row not strictly ascending (a
+                                        repeated or out-of-order tile)         */
 
 /* Human-readable name of a vsa_status value.  Never NULL. */
 const char* vsa_status_string(int32_t status);

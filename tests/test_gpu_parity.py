@@ -151,10 +151,32 @@ def test_out_of_range_index_reports_error():
     _, (qd, kd, vd) = gu.inputs(w, seed=2)
     idx = api.select(qd, kd, w.grid, w.tile, w.topk)
     gu.assert_no_device_error()
-    idx[0, 0, 3, 1] = 10_000
+    idx[0, 0, 3, -1] = 10_000                  # last entry: the list stays ascending
     o, lse = api.attn_fwd(qd, kd, vd, idx, w.grid, w.tile)
     assert api.device_error(reset=True) == 2
     assert torch.isfinite(lse).all()
+
+
+@pytest.mark.parametrize("name", ["ragged256", "vol128", "ragged64"])
+def test_unordered_index_reports_error(name):
+    """A kept list that is not strictly ascending (a repeated tile, or two
+    tiles swapped) is reported through the device error word in every kernel
+    mode (256-, 128- and 64-token tiles; in the last, row 3 is tile B of a
+    pair); the kernel completes and an untouched list gives no error."""
+    w = BY_NAME[name]
+    _, (qd, kd, vd) = gu.inputs(w, seed=2)
+    idx = api.select(qd, kd, w.grid, w.tile, w.topk)
+    api.attn_fwd(qd, kd, vd, idx, w.grid, w.tile)
+    gu.assert_no_device_error()
+    for edit in ("repeat", "swap"):
+        bad = idx.clone()
+        if edit == "repeat":
+            bad[0, 0, 3, 1] = bad[0, 0, 3, 0]
+        else:
+            bad[0, -1, 3, 0], bad[0, -1, 3, 1] = idx[0, -1, 3, 1], idx[0, -1, 3, 0]
+        o, lse = api.attn_fwd(qd, kd, vd, bad, w.grid, w.tile)
+        assert api.device_error(reset=True) == 3, edit
+        assert torch.isfinite(lse).all()
 
 
 def test_bad_topk_raises():

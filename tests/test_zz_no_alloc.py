@@ -53,8 +53,12 @@ def test_noalloc_matches_workspace_select(w):
         ref = torch.full((w.B, w.H, nT, w.topk), -1, dtype=torch.int32, device="cuda")
         got = torch.full_like(ref, -2)
         _select_with_workspace(shp, qd, kd, w.topk, ref)
+        torch.cuda.synchronize()
+        free_before = torch.cuda.mem_get_info()[0]
         _select_noalloc(shp, qd, kd, w.topk, got)
         torch.cuda.synchronize()
+        # the scratch belongs to the loaded library: this call takes no device memory
+        assert torch.cuda.mem_get_info()[0] == free_before, "vsa_select_noalloc allocated device memory"
         assert torch.equal(ref, got), f"seed {seed}: noalloc indices differ"
         assert int(ref.min()) >= 0
     gu.assert_no_device_error()
