@@ -20,7 +20,8 @@ STATUS = {
 DEVERR = {0: "none", 1: "wait timeout", 2: "tile index out of range", 3: "kept list not strictly ascending"}
 
 EXPORTS = ("vsa_tile_count", "vsa_kv_tile_count", "vsa_topk_from_sparsity", "vsa_select_workspace_bytes",
-           "vsa_select", "vsa_select_noalloc", "vsa_attn_fwd", "vsa_device_error", "vsa_status_string")
+           "vsa_select", "vsa_select_noalloc", "vsa_attn_fwd", "vsa_select_coarse_workspace_bytes",
+           "vsa_select_coarse", "vsa_attn_fwd_gated", "vsa_device_error", "vsa_status_string")
 SELECT_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
@@ -67,6 +68,12 @@ def lib() -> ctypes.CDLL:
         L.vsa_select_noalloc.restype = ctypes.c_int
         L.vsa_attn_fwd.argtypes = [S, P, P, P, P, I32, ctypes.c_float, P, P, P]
         L.vsa_attn_fwd.restype = ctypes.c_int
+        L.vsa_select_coarse_workspace_bytes.argtypes = [S]
+        L.vsa_select_coarse_workspace_bytes.restype = SZ
+        L.vsa_select_coarse.argtypes = [S, P, P, P, I32, ctypes.c_float, P, P, P, SZ, P]
+        L.vsa_select_coarse.restype = ctypes.c_int
+        L.vsa_attn_fwd_gated.argtypes = [S, P, P, P, P, I32, ctypes.c_float, P, P, P, P, P]
+        L.vsa_attn_fwd_gated.restype = ctypes.c_int
         L.vsa_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), I32]
         L.vsa_device_error.restype = ctypes.c_int
         L.vsa_status_string.argtypes = [I32]

@@ -16,8 +16,8 @@ import torch
 
 from ._native import DTYPE_BF16, DTYPE_F16, LAYOUT_BHND, LAYOUT_BNHD, VsaShape, check, lib
 
-__all__ = ["make_shape", "tile_count", "kv_tile_count", "topk_from_sparsity", "select", "attn_fwd", "forward",
-           "forward_host", "device_error", "select_workspace_bytes"]
+__all__ = ["make_shape", "tile_count", "kv_tile_count", "topk_from_sparsity", "select", "select_coarse", "attn_fwd",
+           "forward", "forward_host", "device_error", "select_workspace_bytes"]
 
 
 _DTYPES = {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_F16}
@@ -120,9 +120,38 @@ def select(q: torch.Tensor, k: torch.Tensor, grid, tile, topk: int, *, grid_k=No
     return out
 
 
+def select_coarse(q, k, v, grid, tile, topk: int, *, scale: float | None = None, grid_k=None, tile_k=None,
+                  layout: str = "bhnd", prefix_tiles: int = 0, out=None, coarse=None, workspace=None, stream=None):
+    """select() plus the pooled coarse branch: (idx, o_coarse f32 [B, H, nTq, d]),
+    o_coarse[i] = sum_j softmax_j(scale * mean_i(Q) . mean_j(K)) mean_j(V)."""
+    B, H, Nq, d = _dims(q, layout)
+    Nk = _grid_tokens(grid_k if grid_k is not None else grid)
+    _check_qkv("q", q, (B, H, _grid_tokens(grid), d), layout)
+    for name, x in (("k", k), ("v", v)):
+        _check_qkv(name, x, (B, H, Nk, d), layout, q.dtype)
+    shp = make_shape(B, H, grid, d, tile, q.dtype, layout=layout, grid_k=grid_k, tile_k=tile_k,
+                     prefix_tiles=prefix_tiles)
+    nT, _ = tile_count(grid, tile, d, B, H)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, H, nT, topk), dtype=torch.int32, device=q.device)
+    if coarse is None:
+        coarse = torch.empty((B, H, nT, d), dtype=torch.float32, device=q.device)
+    ws_bytes = int(lib().vsa_select_coarse_workspace_bytes(ctypes.byref(shp)))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    check("vsa_select_coarse", lib().vsa_select_coarse(
+        ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(), int(topk), float(scale), out.data_ptr(),
+        coarse.data_ptr(), workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out, coarse
+
+
 def attn_fwd(q, k, v, idx, grid, tile, *, grid_k=None, tile_k=None, layout: str = "bhnd",
-             scale: float | None = None, out=None, lse=None, stream=None):
-    """Block-sparse attention over the kept tiles: (O like q, LSE f32 [B, H, Nq])."""
+             scale: float | None = None, out=None, lse=None, coarse=None, gate=None, stream=None):
+    """Block-sparse attention over the kept tiles: (O like q, LSE f32 [B, H, Nq]).
+    With coarse (f32 [B, H, nTq, d], from select_coarse) and gate (like q), O
+    also carries the gated coarse branch: O += gate * coarse[query tile]."""
     B, H, Nq, d = _dims(q, layout)
     Nk = _grid_tokens(grid_k if grid_k is not None else grid)
     _check_qkv("q", q, (B, H, _grid_tokens(grid), d), layout)
@@ -140,23 +169,40 @@ def attn_fwd(q, k, v, idx, grid, tile, *, grid_k=None, tile_k=None, layout: str 
     shp = make_shape(B, H, grid, d, tile, q.dtype, layout=layout, grid_k=grid_k, tile_k=tile_k)
     if out.dtype != q.dtype:
         raise ValueError("out must have the dtype of q")
-    check("vsa_attn_fwd", lib().vsa_attn_fwd(
+    if (coarse is None) != (gate is None):
+        raise ValueError("give both coarse and gate, or neither")
+    if gate is None:
+        check("vsa_attn_fwd", lib().vsa_attn_fwd(
+            ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(), int(topk),
+            float(scale), out.data_ptr(), lse.data_ptr(), _stream(stream)))
+        return out, lse
+    _check_qkv("gate", gate, (B, H, Nq, d), layout, q.dtype)
+    nT = idx.shape[2]
+    if not (coarse.is_cuda and coarse.dtype == torch.float32 and coarse.is_contiguous()
+            and tuple(coarse.shape) == (B, H, nT, d)):
+        raise ValueError(f"coarse must be a contiguous CUDA float32 tensor of shape {(B, H, nT, d)}")
+    check("vsa_attn_fwd_gated", lib().vsa_attn_fwd_gated(
         ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(), int(topk),
-        float(scale), out.data_ptr(), lse.data_ptr(), _stream(stream)))
+        float(scale), coarse.data_ptr(), gate.data_ptr(), out.data_ptr(), lse.data_ptr(), _stream(stream)))
     return out, lse
 
 
 def forward(q, k, v, grid, tile, topk: int | None = None, *, sparsity: float | None = None, grid_k=None,
-            tile_k=None, layout: str = "bhnd", prefix_tiles: int = 0, scale=None, stream=None):
+            tile_k=None, layout: str = "bhnd", prefix_tiles: int = 0, scale=None, gate=None, stream=None):
     """select + attn_fwd: (O, LSE, idx).  Give topk, or sparsity (the fraction
-    of key/value tiles left out, as in the fastbsa page's "Use" example)."""
+    of key/value tiles left out, as in the fastbsa page's "Use" example).
+    With gate (like q), O also carries the gated pooled coarse branch."""
     if (topk is None) == (sparsity is None):
         raise ValueError("give exactly one of topk and sparsity")
     if topk is None:
         topk = topk_from_sparsity(grid, tile, sparsity, grid_k, tile_k, _dims(q, layout)[3], prefix_tiles)
     kw = dict(grid_k=grid_k, tile_k=tile_k, layout=layout, stream=stream)
-    idx = select(q, k, grid, tile, topk, prefix_tiles=prefix_tiles, **kw)
-    o, lse = attn_fwd(q, k, v, idx, grid, tile, scale=scale, **kw)
+    if gate is None:
+        idx = select(q, k, grid, tile, topk, prefix_tiles=prefix_tiles, **kw)
+        o, lse = attn_fwd(q, k, v, idx, grid, tile, scale=scale, **kw)
+    else:
+        idx, coarse = select_coarse(q, k, v, grid, tile, topk, scale=scale, prefix_tiles=prefix_tiles, **kw)
+        o, lse = attn_fwd(q, k, v, idx, grid, tile, scale=scale, coarse=coarse, gate=gate, **kw)
     return o, lse, idx
 
 

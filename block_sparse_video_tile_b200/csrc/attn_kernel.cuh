@@ -94,6 +94,9 @@ struct AttnArgs {
   float* lse;                // [B*H, Nq]
   unsigned int* err;         // device error word
   int box_tq, box_tk;        // t-extent of one TMA box per side (tt/2 in MODE_SHARED, else tt)
+  // pooled coarse branch (both or neither): O += gate * coarse[query tile]
+  const uint16_t* gate;      // Q's layout and type, or nullptr
+  const float* coarse;       // [B*H, nTq, d] float32
 };
 
 template <int D>
@@ -863,10 +866,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_ld32(tO + 32u * c4, ov);
         tmem_wait_ld();
         if (row_valid) {
+          float of[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) of[e] = __uint_as_float(ov[e]) * inv_l;
+          if (a.gate != nullptr) {
+            // pooled coarse branch: O += gate * o_coarse of this row's query tile
+            const uint4* gp = reinterpret_cast<const uint4*>(a.gate + token_offset(g, slot.bh, n_tok) + 32 * c4);
+            const float4* cp = reinterpret_cast<const float4*>(
+                a.coarse + (static_cast<size_t>(slot.bh) * g.nT + slot.tile + (in_b ? 1 : 0)) * D + 32 * c4);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint4 gv = __ldg(gp + e);
+              const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+              const float4 c0 = __ldg(cp + 2 * e), c1 = __ldg(cp + 2 * e + 1);
+              const float cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const float2 gf = unpack_elem2<F16>(gw[u]);
+                of[8 * e + 2 * u] = fmaf(gf.x, cw[2 * u], of[8 * e + 2 * u]);
+                of[8 * e + 2 * u + 1] = fmaf(gf.y, cw[2 * u + 1], of[8 * e + 2 * u + 1]);
+              }
+            }
+          }
           uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = pack_elem2<F16>(__uint_as_float(ov[2 * e]) * inv_l, __uint_as_float(ov[2 * e + 1]) * inv_l);
+          for (int e = 0; e < 16; ++e) pk[e] = pack_elem2<F16>(of[2 * e], of[2 * e + 1]);
           // streaming stores: O is not read again by this kernel, so it
           // should not sit dirty in L2 for whatever kernel runs next
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c4);

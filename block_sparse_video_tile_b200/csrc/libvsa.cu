@@ -214,13 +214,35 @@ static int launch_score(const Geom& gq, const Geom& gk, int topk, int32_t* idx, 
                              : launch_score_narrow<D, kNarrowKeys, kNarrowStages>(gq, gk, topk, idx, means, attr, st);
 }
 
-template <int D, bool F16>
-static int launch_select(const Geom& gq, const Geom& gk, const void* q, const void* k, int topk, int32_t* idx, void* ws,
+// Tile-level attention of the pooled coarse branch: a warp per query tile,
+// MAXJ key tiles per lane (see coarse_kernel).
+template <int D, int MAXJ>
+static int launch_coarse_j(const Geom& gq, const Geom& gk, const float* means, float scale_log2, float* out,
+                           cudaStream_t st) {
+  coarse_kernel<D, MAXJ><<<dim3(ceil_div(gq.nT, kCoarseWarps), gq.B * gq.H), kCoarseWarps * 32, 0, st>>>(
+      gq, gk, means, scale_log2, out);
+  return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
+template <int D>
+static int launch_coarse(const Geom& gq, const Geom& gk, const float* means, float scale_log2, float* out,
                          cudaStream_t st) {
-  CUtensorMap mq, mk;
+  if (gk.nT <= 256) return launch_coarse_j<D, 8>(gq, gk, means, scale_log2, out, st);
+  if (gk.nT <= 512) return launch_coarse_j<D, 16>(gq, gk, means, scale_log2, out, st);
+  if (gk.nT <= 768) return launch_coarse_j<D, 24>(gq, gk, means, scale_log2, out, st);
+  return launch_coarse_j<D, 48>(gq, gk, means, scale_log2, out, st);
+}
+
+// Pooling (Q and K; with v != nullptr also V for the coarse branch), then
+// scores + top-k; with v, then the coarse branch's tile-level attention.
+template <int D, bool F16>
+static int launch_select(const Geom& gq, const Geom& gk, const void* q, const void* k, const void* v, int topk,
+                         int32_t* idx, void* ws, float scale_log2, float* coarse, cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
   int rc;
   if ((rc = encode_qkv_map(&mq, q, gq, gq.tt, F16)) != VSA_OK || (rc = encode_qkv_map(&mk, k, gk, gk.tt, F16)) != VSA_OK)
     return rc;
+  if (v != nullptr && (rc = encode_qkv_map(&mv, v, gk, gk.tt, F16)) != VSA_OK) return rc;
   unsigned int* err = device_error_ptr();
   if (err == nullptr) return VSA_ERR_CUDA;
   float* means = static_cast<float*>(ws);
@@ -228,10 +250,11 @@ static int launch_select(const Geom& gq, const Geom& gk, const void* q, const vo
   if (cudaFuncSetAttribute(pool_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(psmem)) != cudaSuccess)
     return VSA_ERR_CUDA;
-  pool_kernel<D, F16><<<dim3(max(gq.nT, gk.nT), gq.B * gq.H, 2), kPoolThreads, psmem, st>>>(mq, mk, gq, gk, means,
-                                                                                              err);
+  pool_kernel<D, F16><<<dim3(max(gq.nT, gk.nT), gq.B * gq.H, v != nullptr ? 3 : 2), kPoolThreads, psmem, st>>>(
+      mq, mk, v != nullptr ? mv : mk, gq, gk, means, err);
   if (cudaGetLastError() != cudaSuccess) return VSA_ERR_CUDA;
-  return launch_score<D>(gq, gk, topk, idx, means, st);
+  if ((rc = launch_score<D>(gq, gk, topk, idx, means, st)) != VSA_OK) return rc;
+  return v != nullptr ? launch_coarse<D>(gq, gk, means, scale_log2, coarse, st) : VSA_OK;
 }
 
 template <int D, int MODE, bool F16, bool SAME, bool BNHD>
@@ -295,11 +318,12 @@ static int dispatch_attn(int d, int mode, const CUtensorMap& mq, const CUtensorM
 }
 
 static int dispatch_select(const Geom& gq, const Geom& gk, const void* q, const void* k, int topk, int32_t* idx,
-                           void* ws, cudaStream_t st) {
-  if (gq.d == 128) return gq.f16 ? launch_select<128, true>(gq, gk, q, k, topk, idx, ws, st)
-                                 : launch_select<128, false>(gq, gk, q, k, topk, idx, ws, st);
-  return gq.f16 ? launch_select<64, true>(gq, gk, q, k, topk, idx, ws, st)
-                : launch_select<64, false>(gq, gk, q, k, topk, idx, ws, st);
+                           void* ws, cudaStream_t st, const void* v = nullptr, float scale_log2 = 0.f,
+                           float* coarse = nullptr) {
+  if (gq.d == 128) return gq.f16 ? launch_select<128, true>(gq, gk, q, k, v, topk, idx, ws, scale_log2, coarse, st)
+                                 : launch_select<128, false>(gq, gk, q, k, v, topk, idx, ws, scale_log2, coarse, st);
+  return gq.f16 ? launch_select<64, true>(gq, gk, q, k, v, topk, idx, ws, scale_log2, coarse, st)
+                : launch_select<64, false>(gq, gk, q, k, v, topk, idx, ws, scale_log2, coarse, st);
 }
 
 static int tile_count_of(const Geom& g, int32_t* num_tiles, int32_t* tiles_per_axis) {
@@ -384,17 +408,25 @@ int vsa_select_noalloc(const vsa_shape* shape, const void* q, const void* k, int
   return dispatch_select(gq, gk, q, k, topk, idx_out, ws, st);
 }
 
-int vsa_attn_fwd(const vsa_shape* shape, const void* q, const void* k, const void* v, const int32_t* idx,
-                 int32_t topk, float softmax_scale, void* o, float* lse, void* stream) {
+}  // extern "C"
+
+namespace vsa {
+
+// vsa_attn_fwd and its gated form (gate, coarse: both or neither).
+static int attn_fwd_impl(const vsa_shape* shape, const void* q, const void* k, const void* v, const int32_t* idx,
+                         int32_t topk, float softmax_scale, const float* coarse, const void* gate, void* o,
+                         float* lse, void* stream) {
   Geom gq, gk;
   int rc = make_geoms(shape, &gq, &gk);
   if (rc != VSA_OK) return rc;
   if (q == nullptr || k == nullptr || v == nullptr || idx == nullptr || o == nullptr || lse == nullptr)
     return VSA_ERR_INVALID_ARG;
+  if ((gate == nullptr) != (coarse == nullptr)) return VSA_ERR_INVALID_ARG;
   if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return VSA_ERR_INVALID_ARG;
   if (topk <= 0 || topk > gk.nT) return VSA_ERR_TOPK_RANGE;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
-      (reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+      (reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (gate != nullptr && (!aligned16(gate) || !aligned16(coarse))))
     return VSA_ERR_ALIGNMENT;
   const int vol = gq.vol;                    // equal on both sides
   const int mode = vol == 256 ? MODE_SHARED : (vol == 128 ? MODE_TILE : MODE_PAIR);
@@ -415,6 +447,8 @@ int vsa_attn_fwd(const vsa_shape* shape, const void* q, const void* k, const voi
   a.err = device_error_ptr();
   a.box_tq = shared ? gq.tt / 2 : gq.tt;
   a.box_tk = shared ? gk.tt / 2 : gk.tt;
+  a.gate = static_cast<const uint16_t*>(gate);
+  a.coarse = coarse;
   if (a.err == nullptr) return VSA_ERR_CUDA;
   CUtensorMap mq, mk, mv;
   const bool f16 = gq.f16 != 0;
@@ -425,6 +459,48 @@ int vsa_attn_fwd(const vsa_shape* shape, const void* q, const void* k, const voi
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return f16 ? dispatch_attn<true>(gq.d, mode, mq, mk, mv, a, st)
              : dispatch_attn<false>(gq.d, mode, mq, mk, mv, a, st);
+}
+
+}  // namespace vsa
+
+extern "C" {
+
+int vsa_attn_fwd(const vsa_shape* shape, const void* q, const void* k, const void* v, const int32_t* idx,
+                 int32_t topk, float softmax_scale, void* o, float* lse, void* stream) {
+  return attn_fwd_impl(shape, q, k, v, idx, topk, softmax_scale, nullptr, nullptr, o, lse, stream);
+}
+
+size_t vsa_select_coarse_workspace_bytes(const vsa_shape* shape) {
+  Geom gq, gk;
+  if (make_geoms(shape, &gq, &gk) != VSA_OK) return 0;
+  return coarse_workspace_bytes(gq, gk);
+}
+
+int vsa_select_coarse(const vsa_shape* shape, const void* q, const void* k, const void* v, int32_t topk,
+                      float softmax_scale, int32_t* idx_out, float* coarse_out, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  Geom gq, gk;
+  int rc = make_geoms(shape, &gq, &gk);
+  if (rc != VSA_OK) return rc;
+  if (q == nullptr || k == nullptr || v == nullptr || idx_out == nullptr || coarse_out == nullptr)
+    return VSA_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return VSA_ERR_INVALID_ARG;
+  if (topk <= 0 || topk > gk.nT || topk < gk.prefix) return VSA_ERR_TOPK_RANGE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(workspace) ||
+      (reinterpret_cast<uintptr_t>(idx_out) & 3u) || (reinterpret_cast<uintptr_t>(coarse_out) & 3u))
+    return VSA_ERR_ALIGNMENT;
+  if (workspace == nullptr || workspace_bytes < coarse_workspace_bytes(gq, gk)) return VSA_ERR_WORKSPACE;
+  if ((rc = check_arch()) != VSA_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return dispatch_select(gq, gk, q, k, topk, idx_out, workspace, st, v, softmax_scale * 1.4426950408889634f,
+                         coarse_out);
+}
+
+int vsa_attn_fwd_gated(const vsa_shape* shape, const void* q, const void* k, const void* v, const int32_t* idx,
+                       int32_t topk, float softmax_scale, const float* coarse, const void* gate, void* o,
+                       float* lse, void* stream) {
+  if (coarse == nullptr || gate == nullptr) return VSA_ERR_INVALID_ARG;
+  return attn_fwd_impl(shape, q, k, v, idx, topk, softmax_scale, coarse, gate, o, lse, stream);
 }
 
 int vsa_device_error(uint32_t* code, int32_t reset) {

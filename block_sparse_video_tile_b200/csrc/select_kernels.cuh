@@ -38,11 +38,17 @@ inline size_t select_workspace_bytes(const Geom& gq, const Geom& gk) {
   return sizeof(float) * static_cast<size_t>(gq.B) * gq.H * gq.d * (means_ld(gq.nT) + means_ld(gk.nT));
 }
 
-// Start of head bh's means of side z (0: Q, 1: K) in the workspace.
+// The coarse branch also pools V (its means follow the K means).
+inline size_t coarse_workspace_bytes(const Geom& gq, const Geom& gk) {
+  return sizeof(float) * static_cast<size_t>(gq.B) * gq.H * gq.d * (means_ld(gq.nT) + 2 * means_ld(gk.nT));
+}
+
+// Start of head bh's means of tensor z (0: Q, 1: K, 2: V) in the workspace.
 __host__ __device__ inline size_t means_offset(const Geom& gq, const Geom& gk, int z, int bh) {
   const size_t BH = static_cast<size_t>(gq.B) * gq.H;
+  const size_t kv = static_cast<size_t>(gk.d) * means_ld(gk.nT);
   return z == 0 ? static_cast<size_t>(bh) * gq.d * means_ld(gq.nT)
-                : BH * gq.d * means_ld(gq.nT) + static_cast<size_t>(bh) * gk.d * means_ld(gk.nT);
+                : BH * gq.d * means_ld(gq.nT) + (z == 2 ? BH * kv : 0) + static_cast<size_t>(bh) * kv;
 }
 
 // Larger float -> larger unsigned key (total order; -0 < +0, scores are
@@ -115,8 +121,9 @@ __device__ __forceinline__ void bsearch_topk_row(const uint32_t* kr, int nT, int
   }
 }
 
-// One CTA per (tile j, head bh, tensor z in {Q, K}), each side with its own
-// grid and tile (CTAs past a side's tile count exit).  The whole tile is one
+// One CTA per (tile j, head bh, tensor z in {Q, K} -- and V for the coarse
+// branch), each side with its own grid and tile (CTAs past a side's tile
+// count exit).  The whole tile is one
 // 5-D TMA box per 64-channel slab (the same views the attend kernel uses), so
 // a 256-token tile of d = 128 puts 64 KB in flight per CTA without using
 // registers; positions past the y and x edges arrive as zeros, and rows past
@@ -126,7 +133,8 @@ __device__ __forceinline__ void bsearch_topk_row(const uint32_t* kr, int nT, int
 // Dynamic shared memory: box (slabs x vol x 128 B, 1024-aligned) | partial sums | mbarrier.
 template <int D, bool F16>
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __grid_constant__ CUtensorMap tmQ,
-                                                            const __grid_constant__ CUtensorMap tmK, Geom gq,
+                                                            const __grid_constant__ CUtensorMap tmK,
+                                                            const __grid_constant__ CUtensorMap tmV, Geom gq,
                                                             Geom gk, float* __restrict__ means, unsigned int* err) {
   constexpr int kSlabs = D / 64;
   constexpr int TPR = D / 8;                 // threads per row (one 16-byte chunk each)
@@ -154,7 +162,9 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __grid_constan
     mbar_arrive_expect_tx(bar, static_cast<uint32_t>(kSlabs * box_bytes));
     const BoxCoord bc = box_coord(g, bh, c.bt * g.tt, c.by * g.th, c.bx * g.tw);
     for (int sl = 0; sl < kSlabs; ++sl)
-      tma_load_5d(base + sl * box_bytes, z == 0 ? static_cast<const void*>(&tmQ) : static_cast<const void*>(&tmK),
+      tma_load_5d(base + sl * box_bytes,
+                  z == 0 ? static_cast<const void*>(&tmQ)
+                         : (z == 1 ? static_cast<const void*>(&tmK) : static_cast<const void*>(&tmV)),
                   bar, sl * 64, bc.c1, bc.c2, bc.c3, bc.c4);
   }
   // let the score kernel's launch begin while this grid drains
@@ -476,6 +486,74 @@ template <int D, int KEYS, int STAGES>
 inline size_t score_narrow_smem_bytes(const Geom& gk) {
   return sizeof(float) * (static_cast<size_t>(D) * kNarrowRows + STAGES * kNarrowSlice * KEYS) +
          sizeof(uint32_t) * static_cast<size_t>(kNarrowRows) * gk.nT;
+}
+
+// ------------------------------------------------------------ coarse branch
+// Tile-level attention (pooled coarse branch): for query tile i of head bh,
+// o[i] = sum_j softmax_j(scale * qbar_i . kbar_j) vbar_j over every
+// key/value tile j, from the channel-major means in the workspace.  One warp
+// per query tile: lane l holds the scores of key tiles l, l + 32, ...  (the
+// means rows are contiguous in j, so each channel's loads coalesce), the
+// softmax is a warp reduction, and each output channel is a warp sum of
+// p_j * vbar_j[c].  float32 throughout; reads the means from L2.
+constexpr int kCoarseWarps = 8;
+
+template <int D, int MAXJ>
+__global__ void __launch_bounds__(kCoarseWarps * 32) coarse_kernel(Geom gq, Geom gk, const float* __restrict__ means,
+                                                                   float scale_log2, float* __restrict__ out) {
+  __shared__ float qs[kCoarseWarps][D];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int bh = blockIdx.y;
+  const int i = blockIdx.x * kCoarseWarps + warp;
+  if (i >= gq.nT) return;
+  const int nT = gk.nT, ldq = means_ld(gq.nT), ldk = means_ld(nT);
+  const float* mq = means + means_offset(gq, gk, 0, bh);
+  const float* mk = means + means_offset(gq, gk, 1, bh);
+  const float* mv = means + means_offset(gq, gk, 2, bh);
+  for (int c = lane; c < D; c += 32) qs[warp][c] = mq[static_cast<size_t>(c) * ldq + i];
+  __syncwarp();
+  float s[MAXJ];
+#pragma unroll
+  for (int t = 0; t < MAXJ; ++t) s[t] = 0.f;
+  for (int c = 0; c < D; ++c) {
+    const float qc = qs[warp][c];
+    const float* row = mk + static_cast<size_t>(c) * ldk;
+#pragma unroll
+    for (int t = 0; t < MAXJ; ++t) {
+      const int j = lane + 32 * t;
+      if (j < nT) s[t] = fmaf(qc, row[j], s[t]);
+    }
+  }
+  float mx = -INFINITY;
+#pragma unroll
+  for (int t = 0; t < MAXJ; ++t) {
+    s[t] = (lane + 32 * t < nT) ? s[t] * scale_log2 : -INFINITY;
+    mx = fmaxf(mx, s[t]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float l = 0.f;
+#pragma unroll
+  for (int t = 0; t < MAXJ; ++t) {
+    s[t] = ex2_approx(s[t] - mx);              // 0 past the last key tile
+    l += s[t];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+  const float inv_l = 1.f / l;
+  float* orow = out + (static_cast<size_t>(bh) * gq.nT + i) * D;
+  for (int c = 0; c < D; ++c) {
+    const float* row = mv + static_cast<size_t>(c) * ldk;
+    float acc = 0.f;
+#pragma unroll
+    for (int t = 0; t < MAXJ; ++t) {
+      const int j = lane + 32 * t;
+      if (j < nT) acc = fmaf(s[t], row[j], acc);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == (c & 31)) orow[c] = acc * inv_l;
+  }
 }
 
 }  // namespace vsa

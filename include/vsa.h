@@ -211,6 +211,45 @@ int vsa_attn_fwd(const vsa_shape* shape, const void* q, const void* k, const voi
                  const int32_t* idx, int32_t topk, float softmax_scale,
                  void* o, float* lse, void* stream);
 
+/* Pooled coarse branch (FastVideo VSA guide, "Checkpoint behavior": Wan
+ * checkpoints that carry learned to_gate_compress weights add a gated
+ * compensation to the sparse branch; without them the sparse branch runs
+ * alone).  The pages give no formula; this library's reading: attention at
+ * tile granularity,
+ *   o_coarse[i] = sum_j softmax_j(scale * qbar_i . kbar_j) vbar_j
+ * over every key/value tile j (one softmax entry per tile, whatever its
+ * token count), with qbar, kbar, vbar the tiles' means over their valid
+ * tokens, and O[n] = O_sparse[n] + gate[n] * o_coarse[tile of n], the gate
+ * being the caller's projection output (same shape and type as O).
+ *
+ * Bytes of workspace vsa_select_coarse needs: the Q, K and V tile means,
+ * float32, channel-major ([B*H, d, ldq], then [B*H, d, ldk] twice).
+ * Returns 0 for an invalid shape. */
+size_t vsa_select_coarse_workspace_bytes(const vsa_shape* shape);
+
+/* vsa_select plus the coarse branch's tile-level attention.
+ *   q, k, v       : device Q, K, V as for vsa_attn_fwd
+ *   softmax_scale : > 0 and finite (the fine branch's scale)
+ *   idx_out       : as vsa_select
+ *   coarse_out    : device float32 [B, H, nTq, d], o_coarse of every query
+ *                   tile (16-byte aligned for vsa_attn_fwd_gated)
+ *   workspace     : at least vsa_select_coarse_workspace_bytes(shape) bytes,
+ *                   16-byte aligned
+ * Three kernel launches on `stream`. */
+int vsa_select_coarse(const vsa_shape* shape, const void* q, const void* k, const void* v, int32_t topk,
+                      float softmax_scale, int32_t* idx_out, float* coarse_out, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+/* vsa_attn_fwd whose output also carries the gated coarse branch:
+ * O[n] = sparse attention (as vsa_attn_fwd) + gate[n] * coarse[tile of n],
+ * added in float32 before O is rounded to the input type; LSE is the sparse
+ * branch's.  coarse: device float32 [B, H, nTq, d] (from vsa_select_coarse),
+ * gate: device tensor of O's layout and type; both 16-byte aligned and both
+ * required (VSA_ERR_INVALID_ARG otherwise).  One kernel launch on `stream`. */
+int vsa_attn_fwd_gated(const vsa_shape* shape, const void* q, const void* k, const void* v,
+                       const int32_t* idx, int32_t topk, float softmax_scale, const float* coarse,
+                       const void* gate, void* o, float* lse, void* stream);
+
 /* Reads (and with reset != 0 clears) the kernels' device error word on the
  * current device: 0 = no error; otherwise a VSA_DEVERR_* code.  Synchronizes
  * the device.  Returns a vsa_status for the read itself. */

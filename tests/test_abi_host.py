@@ -183,3 +183,32 @@ def test_prefix_tiles_checked_before_launch():
     assert _sel(shp, topk=14) == 2
     assert _native.lib().vsa_tile_count(ctypes.byref(shp), ctypes.byref(n), None) == 0
     assert api.topk_from_sparsity((31, 22, 40), (4, 8, 8), 0.99, prefix_tiles=15) == 15
+
+
+def _selc(shp, q=256, k=512, v=768, topk=4, scale=0.1, idx=1024, coarse=2048, ws=4096, ws_bytes=1 << 30):
+    return _native.lib().vsa_select_coarse(ctypes.byref(shp), q, k, v, topk, scale, idx, coarse, ws, ws_bytes, None)
+
+
+def _attg(shp, coarse=8192, gate=16384, **kw):
+    a = dict(q=256, k=512, v=768, idx=1024, topk=4, scale=0.1, o=2048, lse=4096)
+    a.update(kw)
+    return _native.lib().vsa_attn_fwd_gated(ctypes.byref(shp), a["q"], a["k"], a["v"], a["idx"], a["topk"],
+                                            a["scale"], coarse, gate, a["o"], a["lse"], None)
+
+
+def test_coarse_entry_points_check_arguments_before_launch():
+    """The pooled coarse branch's calls validate like the others: no device is touched."""
+    shp = api.make_shape(1, 2, (31, 22, 40), 128, (4, 8, 8))
+    need = int(_native.lib().vsa_select_coarse_workspace_bytes(ctypes.byref(shp)))
+    assert need == 4 * 2 * 128 * (120 + 2 * 120)            # Q, K and V means, float32
+    assert _selc(shp, v=0) == 1
+    assert _selc(shp, coarse=0) == 1
+    assert _selc(shp, scale=0.0) == 1
+    assert _selc(shp, topk=121) == 2
+    assert _selc(shp, v=8) == 4
+    assert _selc(shp, ws_bytes=need - 1) == 5
+    assert _attg(shp, coarse=0) == 1                        # the gate needs its coarse output
+    assert _attg(shp, gate=0) == 1
+    assert _attg(shp, gate=24) == 4
+    assert _attg(shp, coarse=8200) == 4
+    assert _attg(shp, topk=0) == 2
