@@ -48,6 +48,18 @@ from block_sparse_video_tile_b200 import api  # noqa: E402
 from block_sparse_video_tile_b200.workloads import ALL  # noqa: E402
 
 METRIC = "block-sparse attn fwd ms/call & effective TFLOP/s (select+attend) at Wan shape"
+SHAPE_NAMES = {"tiny": "Tiny", "wan14b": "Wan-14B", "longcat": "LongCat-like", "longcat_kv": "LongCat-style call"}
+
+
+def metric_for(w) -> str:
+    """The headline metric's wording for the workload measured (the Wan-5B
+    shape and its top-k sweep keep the headline's own words)."""
+    base = w.name.split("_h")[0]
+    if base == "wan5b" or base.startswith("sweep_"):
+        return METRIC
+    return METRIC.replace("at Wan shape", f"at {SHAPE_NAMES.get(base, base)} shape")
+
+
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -222,19 +234,23 @@ def make_inputs(w, device, seed):
 
 
 # ---------------------------------------------------------------- oracle arm
-def oracle_sample(q_bits, k_bits, v_bits, w, n_tiles):
+def oracle_sample(q_bits, k_bits, v_bits, w, n_tiles, idx_attend=None):
     """Time the float64 oracle on one head: full selection, then attention for
-    the first n_tiles query tiles.  Returns (seconds, exact FLOPs of the sample)."""
+    the first n_tiles query tiles (over the oracle's own selection, or over
+    idx_attend when given -- the GPU's, so that a near-tie row is compared
+    on equal terms).  Returns (seconds, exact FLOPs of the sample,
+    (idx, scores, O, LSE))."""
     from oracle import vsa_oracle as vo
     t0 = time.perf_counter()
-    Q, K, V = (vo.bf16_to_f64(x) for x in (q_bits, k_bits, v_bits))
-    idx, _, _ = vo.select_head(Q, K, w.grid, w.tile, w.topk, w.kv_grid, w.kv_tile, w.prefix_tiles)
-    vo.attend_head(Q, K, V, w.grid, w.tile, idx, w.d ** -0.5, query_tiles=range(n_tiles),
-                   grid_k=w.kv_grid, tile_k=w.kv_tile)
+    Q, K, V = (vo.widen(x, w.dtype) for x in (q_bits, k_bits, v_bits))
+    idx, scores, _ = vo.select_head(Q, K, w.grid, w.tile, w.topk, w.kv_grid, w.kv_tile, w.prefix_tiles)
+    use = idx if idx_attend is None else idx_attend
+    O, L = vo.attend_head(Q, K, V, w.grid, w.tile, use, w.d ** -0.5, query_tiles=range(n_tiles),
+                          grid_k=w.kv_grid, tile_k=w.kv_tile)
     dt = time.perf_counter() - t0
     cq, ck = tile_counts(w), tile_counts(w, kv=True)
-    fl = float(4 * w.d * sum(cq[i] * ck[idx[i]].sum() for i in range(n_tiles)))
-    return dt, fl
+    fl = float(4 * w.d * sum(cq[i] * ck[use[i]].sum() for i in range(n_tiles)))
+    return dt, fl, (idx, scores, O, L)
 
 
 def head_bits(x: torch.Tensor, w, b=0, h=0) -> np.ndarray:
@@ -256,14 +272,14 @@ def run_reference(args, w, rank):
         oracle_sample(*qkv, w, 1)
     secs, flops = 0.0, 0.0
     for _ in range(args.steps):
-        dt, fl = oracle_sample(*qkv, w, n_tiles)
+        dt, fl, _ = oracle_sample(*qkv, w, n_tiles)
         secs += dt
         flops += fl
     value = flops / secs / 1e12
     sample = (f"one head of {w.name}: full tile selection + attention for {n_tiles} of "
               f"{len(tile_counts(w))} query tiles per step")
     return {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+        "metric": metric_for(w), "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "impl": "reference",
@@ -353,33 +369,63 @@ def run_ours(args, w, rank, world, device):
     sel_ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
     att_ms = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
 
-    # end to end through the public host-to-host API (api.forward_host): the
-    # timed region holds the uploads of Q, K, V from pinned host memory, the
-    # kernels and the downloads of O, LSE and idx, pipelined by chunks of heads.
-    # forward_host covers [B, H, N, d] self-attention without prefix tiles.
-    host_path = w.grid_k is None and w.tile_k is None and w.layout == "bhnd" and not w.prefix_tiles
-    e2e_ms = float("nan")
-    if host_path:
-        hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
-        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-        hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-        hx = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
-        e2e_steps = max(3, min(args.steps, 10))
+    # end to end through the C ABI's host-to-host call (vsa_forward_host, via
+    # api.forward_host): the timed region holds the uploads of Q, K, V from
+    # pinned host memory, the kernels and the downloads of O, LSE and idx,
+    # pipelined by chunks of heads, for every workload's layout and grids.
+    hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    hx = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+    e2e_steps = max(3, min(args.steps, 10))
 
-        def e2e_step():
-            api.forward_host(hq, hk, hv, grid, tile, w.topk, out=ho, lse=hl, idx=hx, chunk_heads=2)
+    def e2e_step():
+        api.forward_host(hq, hk, hv, grid, tile, w.topk, out=ho, lse=hl, idx=hx, chunk_heads=2,
+                         prefix_tiles=w.prefix_tiles, **geo)
 
+    e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(e2e_steps):
         e2e_step()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if world > 1:
-            dist.barrier()
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if not torch.equal(hx, idx.cpu()):
+        raise RuntimeError("host-to-host call selected other tiles than the device path")
+
+    # the pooled coarse branch's extra cost: select with V pooling and the
+    # tile-level attention, attend with the gate in its epilogue
+    gate = torch.randn(q.shape, generator=torch.Generator(device=device).manual_seed(7), device=device,
+                       dtype=torch.float32).to(q.dtype)
+    coarse = torch.empty((w.B, w.H, nT, w.d), dtype=torch.float32, device=device)
+    o_c, lse_c = torch.empty_like(o), torch.empty_like(lse)
+    idx_c = torch.empty_like(idx)
+    ws_c = torch.empty(api.select_coarse_workspace_bytes(w.B, w.H, grid, w.d, tile, w.grid_k, w.tile_k),
+                       dtype=torch.uint8, device=device)
+
+    def coarse_step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        api.select_coarse(q, k, v, grid, tile, w.topk, out=idx_c, coarse=coarse, workspace=ws_c,
+                          prefix_tiles=w.prefix_tiles, **geo)
+        if ev is not None:
+            ev[1].record(stream)
+        api.attn_fwd(q, k, v, idx_c, grid, tile, out=o_c, lse=lse_c, coarse=coarse, gate=gate, **geo)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(2):
+        coarse_step()
+    cevs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(5)]
+    for e in cevs:
+        coarse_step(e)
+    torch.cuda.synchronize()
+    csel_ms = statistics.median(e[0].elapsed_time(e[1]) for e in cevs)
+    catt_ms = statistics.median(e[1].elapsed_time(e[2]) for e in cevs)
 
     ms_max, e2e_max = max_over_ranks([ms, e2e_ms], world, device)
     if rank != 0:
@@ -393,7 +439,7 @@ def run_ours(args, w, rank, world, device):
     sel_gbs = select_bytes(w) / (sel_ms * 1e-3) / 1e9
     value = aggregate_tflops(flops, ms_max, args.steps, world)
     out = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "metric": metric_for(w), "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": describe(w), "parallelism": f"replicas x{world} (heads shard, no exchange)",
@@ -412,24 +458,56 @@ def run_ours(args, w, rank, world, device):
                             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": sel_gbs / peaks["hbm_gbs"],
                             "peak_source": f"{src} hbm_gbs",
                             "traffic": recorded_traffic("pool_kernel", w.name)},
-        "e2e": ({"value": aggregate_tflops(flops, e2e_max, 1, world), "unit": "TFLOP/s", "ms_per_step": e2e_max,
-                 "h2d_bytes_per_step": int((q.numel() + k.numel() + v.numel()) * 2),
-                 "d2h_bytes_per_step": int(o.numel() * 2 + lse.numel() * 4 + idx.numel() * 4),
-                 "api": "forward_host (pinned host buffers, 2-head chunks on 3 streams)"} if host_path else
-                {"value": None, "unit": "TFLOP/s",
-                 "why": "forward_host covers [B, H, N, d] self-attention without prefix tiles"}),
+        "e2e": {"value": aggregate_tflops(flops, e2e_max, 1, world), "unit": "TFLOP/s", "ms_per_step": e2e_max,
+                "h2d_bytes_per_step": int((q.numel() + k.numel() + v.numel()) * 2),
+                "d2h_bytes_per_step": int(o.numel() * 2 + lse.numel() * 4 + idx.numel() * 4),
+                "api": "vsa_forward_host (C ABI; pinned host buffers, 2-head chunks, library streams)"},
+        "coarse_branch": {"select_ms": csel_ms, "attend_gated_ms": catt_ms,
+                          "extra_ms_per_step": csel_ms + catt_ms - sel_ms - att_ms,
+                          "what": "V pooling + tile-level attention in select; gate * o_coarse in the attend epilogue"},
         "gpu_launches": 3 * args.steps,
         "clocks": clk.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:
         # whole heads (full selection + attention of every query tile) until
         # about 10 s of CPU work, at most all heads of the workload
+        # The same oracle runs double as a parity check of those heads: every
+        # selected index (near-ties counted), and O and LSE of every query tile.
+        from oracle import vsa_oracle as vo
+        gidx = idx.cpu().numpy()
+        o_bhnd = (o.permute(0, 2, 1, 3) if w.layout == "bnhd" else o).float().cpu().numpy()
+        lse_h = lse.cpu().numpy()
+        toks = vo.tile_tokens(w.grid, w.tile)
         dt = fl = 0.0
         heads = 0
+        par = {"heads": 0, "rows": 0, "exact_rows": 0, "near_tie_rows": 0, "o_max_abs": 0.0, "o_sum_abs": 0.0,
+               "o_count": 0, "lse_max_abs": 0.0}
         while heads < w.B * w.H and (heads == 0 or dt < 10.0):
             b, h = divmod(heads, w.H)
-            t, f = oracle_sample(head_bits(q, w, b, h), head_bits(k, w, b, h), head_bits(v, w, b, h), w, nT)
+            t, f, (ridx, scores, O, L) = oracle_sample(head_bits(q, w, b, h), head_bits(k, w, b, h),
+                                                       head_bits(v, w, b, h), w, nT, idx_attend=gidx[b, h])
             dt, fl, heads = dt + t, fl + f, heads + 1
+            for i in range(nT):
+                par["rows"] += 1
+                if np.array_equal(ridx[i], gidx[b, h, i]):
+                    par["exact_rows"] += 1
+                elif vo.selection_is_valid(gidx[b, h, i], scores[i], w.topk):
+                    par["near_tie_rows"] += 1
+            rows = np.concatenate(toks)
+            e = np.abs(o_bhnd[b, h][rows] - O[rows])
+            par["o_max_abs"] = max(par["o_max_abs"], float(e.max()))
+            par["o_sum_abs"] += float(e.sum())
+            par["o_count"] += e.size
+            par["lse_max_abs"] = max(par["lse_max_abs"], float(np.abs(lse_h[b, h][rows] - L[rows]).max()))
+            par["heads"] += 1
+        bad = par["rows"] - par["exact_rows"] - par["near_tie_rows"]
+        out["parity"] = {"heads": par["heads"], "rows": par["rows"], "exact_rows": par["exact_rows"],
+                         "near_tie_rows": par["near_tie_rows"], "invalid_rows": bad,
+                         "o_max_abs": par["o_max_abs"], "o_mean_abs": par["o_sum_abs"] / max(par["o_count"], 1),
+                         "lse_max_abs": par["lse_max_abs"],
+                         "tolerance": {"o_max_abs": 2e-2, "o_mean_abs": 2e-3, "lse_abs": 1e-3},
+                         "oracle": "float64 CPU oracle on the same device inputs (attention over the GPU's "
+                                   "selection)"}
         out["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
                                "kind": "oracle",
                                "sample": f"{heads} of {w.B * w.H} heads, each a full tile selection + attention "

@@ -21,7 +21,8 @@ DEVERR = {0: "none", 1: "wait timeout", 2: "tile index out of range", 3: "kept l
 
 EXPORTS = ("vsa_tile_count", "vsa_kv_tile_count", "vsa_topk_from_sparsity", "vsa_select_workspace_bytes",
            "vsa_select", "vsa_select_noalloc", "vsa_attn_fwd", "vsa_select_coarse_workspace_bytes",
-           "vsa_select_coarse", "vsa_attn_fwd_gated", "vsa_device_error", "vsa_status_string")
+           "vsa_select_coarse", "vsa_attn_fwd_gated", "vsa_forward_host_workspace_bytes", "vsa_forward_host",
+           "vsa_device_error", "vsa_status_string")
 SELECT_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
@@ -74,6 +75,10 @@ def lib() -> ctypes.CDLL:
         L.vsa_select_coarse.restype = ctypes.c_int
         L.vsa_attn_fwd_gated.argtypes = [S, P, P, P, P, I32, ctypes.c_float, P, P, P, P, P]
         L.vsa_attn_fwd_gated.restype = ctypes.c_int
+        L.vsa_forward_host_workspace_bytes.argtypes = [S, I32, I32]
+        L.vsa_forward_host_workspace_bytes.restype = SZ
+        L.vsa_forward_host.argtypes = [S, P, P, P, I32, ctypes.c_float, P, P, P, I32, P, SZ, P]
+        L.vsa_forward_host.restype = ctypes.c_int
         L.vsa_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), I32]
         L.vsa_device_error.restype = ctypes.c_int
         L.vsa_status_string.argtypes = [I32]

@@ -17,7 +17,7 @@ import torch
 from ._native import DTYPE_BF16, DTYPE_F16, LAYOUT_BHND, LAYOUT_BNHD, VsaShape, check, lib
 
 __all__ = ["make_shape", "tile_count", "kv_tile_count", "topk_from_sparsity", "select", "select_coarse", "attn_fwd",
-           "forward", "forward_host", "device_error", "select_workspace_bytes"]
+           "forward", "forward_host", "device_error", "select_workspace_bytes", "select_coarse_workspace_bytes"]
 
 
 _DTYPES = {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_F16}
@@ -65,6 +65,11 @@ def topk_from_sparsity(grid, tile, sparsity: float, grid_k=None, tile_k=None, d:
 def select_workspace_bytes(B, H, grid, d, tile, grid_k=None, tile_k=None) -> int:
     shp = make_shape(B, H, grid, d, tile, grid_k=grid_k, tile_k=tile_k)
     return int(lib().vsa_select_workspace_bytes(ctypes.byref(shp)))
+
+
+def select_coarse_workspace_bytes(B, H, grid, d, tile, grid_k=None, tile_k=None) -> int:
+    shp = make_shape(B, H, grid, d, tile, grid_k=grid_k, tile_k=tile_k)
+    return int(lib().vsa_select_coarse_workspace_bytes(ctypes.byref(shp)))
 
 
 def _dims(x, layout):
@@ -206,93 +211,55 @@ def forward(q, k, v, grid, tile, topk: int | None = None, *, sparsity: float | N
     return o, lse, idx
 
 
-class _HostPipeline:
-    """Device buffers, streams and events reused by forward_host for one shape."""
-
-    def __init__(self, chunk, N, d, nT, topk, device, ws_bytes, dtype):
-        mk = lambda *shape, dt=dtype: [torch.empty(shape, dtype=dt, device=device) for _ in range(2)]
-        self.q, self.k, self.v, self.o = (mk(1, chunk, N, d) for _ in range(4))
-        self.lse = mk(1, chunk, N, dt=torch.float32)
-        self.idx = mk(1, chunk, nT, topk, dt=torch.int32)
-        self.ws = [torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device) for _ in range(2)]
-        self.s_in = torch.cuda.Stream(device)
-        self.s_comp = torch.cuda.Stream(device)
-        self.s_out = torch.cuda.Stream(device)
-        self.key = (chunk, N, d, nT, topk, device, dtype)
+_HOST_WS = {}
 
 
-_PIPE = {}
+def forward_host(q, k, v, grid, tile, topk: int, *, scale=None, chunk_heads: int = 2, grid_k=None, tile_k=None,
+                 layout: str = "bhnd", prefix_tiles: int = 0, out=None, lse=None, idx=None, device=None,
+                 stream=None):
+    """Host-to-host forward through vsa_forward_host: select + attention for CPU tensors.
 
-
-def forward_host(q, k, v, grid, tile, topk: int, *, scale=None, chunk_heads: int = 2,
-                 out=None, lse=None, idx=None, device=None):
-    """Host-to-host forward: select + attention for pinned CPU tensors.
-
-    q, k, v: pinned CPU bfloat16 [B, H, N, d].  Returns (O, LSE, idx) in pinned
-    CPU tensors (allocated unless given).  The (batch, head) pairs are
-    processed in chunks of ``chunk_heads``: the upload of chunk c+1 and the
-    download of chunk c-1 overlap the kernels of chunk c (three streams,
-    double-buffered device memory).  Every chunk is one vsa_select and one
-    vsa_attn_fwd call with H = chunk.  The caller's current stream waits for
-    all of it, so work queued on it afterwards sees the outputs.
+    q, k, v: CPU bfloat16/float16 tensors in ``layout`` (pinned for the copies
+    to overlap the kernels).  Returns (O, LSE, idx) in CPU tensors (pinned,
+    allocated unless given), complete when the call returns.  The (batch,
+    head) pairs go through the GPU in chunks of ``chunk_heads`` heads,
+    uploads and downloads overlapping the kernels (streams of the library);
+    the device workspace is allocated here once per shape and reused.
     """
-    B, H, N, d = q.shape
-    device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
-    for name, x in (("q", q), ("k", k), ("v", v)):
+    B, H, Nq, d = _dims(q, layout)
+    Nk = _grid_tokens(grid_k if grid_k is not None else grid)
+    for name, x, n in (("q", q, Nq), ("k", k, Nk), ("v", v, Nk)):
         if x.is_cuda or x.dtype != q.dtype or q.dtype not in _DTYPES or not x.is_contiguous():
             raise ValueError(f"{name} must be a contiguous CPU bfloat16/float16 tensor like q "
                              "(pinned for overlap)")
+        if _dims(x, layout) != (B, H, n, d):
+            raise ValueError(f"{name} has (B, H, N, d) = {_dims(x, layout)}, expected {(B, H, n, d)}")
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    shp = make_shape(B, H, grid, d, tile, q.dtype, layout=layout, grid_k=grid_k, tile_k=tile_k,
+                     prefix_tiles=prefix_tiles)
     nT, _ = tile_count(grid, tile, d, B, H)
-    BH = B * H
-    chunk = max(1, min(chunk_heads, BH))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
     if out is None:
-        out = torch.empty((B, H, N, d), dtype=q.dtype).pin_memory()
+        out = torch.empty(q.shape, dtype=q.dtype).pin_memory()
     if lse is None:
-        lse = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+        lse = torch.empty((B, H, Nq), dtype=torch.float32).pin_memory()
     if idx is None:
         idx = torch.empty((B, H, nT, topk), dtype=torch.int32).pin_memory()
-    key = (chunk, N, d, nT, topk, device, q.dtype)
-    pipe = _PIPE.get(key)
-    if pipe is None:
-        pipe = _HostPipeline(chunk, N, d, nT, topk, device, select_workspace_bytes(1, chunk, grid, d, tile),
-                             q.dtype)
-        _PIPE.clear()
-        _PIPE[key] = pipe
-    caller = torch.cuda.current_stream(device)
-    for s_ in (pipe.s_in, pipe.s_comp, pipe.s_out):
-        s_.wait_stream(caller)
-    qf, kf, vf = (x.view(BH, N, d) for x in (q, k, v))
-    of, lf, xf = out.view(BH, N, d), lse.view(BH, N), idx.view(BH, nT, topk)
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_comp = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [None, None]
-    for c, h0 in enumerate(range(0, BH, chunk)):
-        nh = min(chunk, BH - h0)
-        b = c % 2
-        dq, dk, dv, do = (t[b][:, :nh] for t in (pipe.q, pipe.k, pipe.v, pipe.o))
-        dl, di = pipe.lse[b][:, :nh], pipe.idx[b][:, :nh]
-        with torch.cuda.stream(pipe.s_in):
-            if ev_out[b] is not None:          # buffer b's previous outputs are downloaded
-                pipe.s_in.wait_event(ev_out[b])
-            dq.copy_(qf[h0:h0 + nh].unsqueeze(0), non_blocking=True)
-            dk.copy_(kf[h0:h0 + nh].unsqueeze(0), non_blocking=True)
-            dv.copy_(vf[h0:h0 + nh].unsqueeze(0), non_blocking=True)
-            ev_in[b].record(pipe.s_in)
-        with torch.cuda.stream(pipe.s_comp):
-            pipe.s_comp.wait_event(ev_in[b])
-            select(dq, dk, grid, tile, topk, out=di, workspace=pipe.ws[b], stream=pipe.s_comp)
-            attn_fwd(dq, dk, dv, di, grid, tile, scale=scale, out=do, lse=dl, stream=pipe.s_comp)
-            ev_comp[b].record(pipe.s_comp)
-        with torch.cuda.stream(pipe.s_out):
-            pipe.s_out.wait_event(ev_comp[b])
-            of[h0:h0 + nh].unsqueeze(0).copy_(do, non_blocking=True)
-            lf[h0:h0 + nh].unsqueeze(0).copy_(dl, non_blocking=True)
-            xf[h0:h0 + nh].unsqueeze(0).copy_(di, non_blocking=True)
-            e = torch.cuda.Event()
-            e.record(pipe.s_out)
-            ev_out[b] = e
-    for s_ in (pipe.s_in, pipe.s_comp, pipe.s_out):
-        caller.wait_stream(s_)
+    ws_bytes = int(lib().vsa_forward_host_workspace_bytes(ctypes.byref(shp), int(topk), int(chunk_heads)))
+    if ws_bytes == 0:
+        raise ValueError("invalid shape or topk")
+    key = (device, ws_bytes)
+    ws = _HOST_WS.get(key)
+    if ws is None:
+        _HOST_WS.clear()
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
+        _HOST_WS[key] = ws
+    st = torch.cuda.current_stream(device) if stream is None else stream
+    check("vsa_forward_host", lib().vsa_forward_host(
+        ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(), int(topk), float(scale), out.data_ptr(),
+        lse.data_ptr(), idx.data_ptr(), int(chunk_heads), ws.data_ptr(), ws_bytes, st.cuda_stream))
+    st.synchronize()
     return out, lse, idx
 
 

@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "vsa.h"
@@ -214,12 +215,16 @@ static int launch_score(const Geom& gq, const Geom& gk, int topk, int32_t* idx, 
                              : launch_score_narrow<D, kNarrowKeys, kNarrowStages>(gq, gk, topk, idx, means, attr, st);
 }
 
-// Tile-level attention of the pooled coarse branch: a warp per query tile,
+// Tile-level attention of the pooled coarse branch: QT query tiles per warp,
 // MAXJ key tiles per lane (see coarse_kernel).
-template <int D, int MAXJ>
+template <int D, int MAXJ, int QT>
 static int launch_coarse_j(const Geom& gq, const Geom& gk, const float* means, float scale_log2, float* out,
                            cudaStream_t st) {
-  coarse_kernel<D, MAXJ><<<dim3(ceil_div(gq.nT, kCoarseWarps), gq.B * gq.H), kCoarseWarps * 32, 0, st>>>(
+  const size_t smem = coarse_smem_bytes<D>(gk, QT);
+  if (cudaFuncSetAttribute(coarse_kernel<D, MAXJ, QT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return VSA_ERR_CUDA;
+  coarse_kernel<D, MAXJ, QT><<<dim3(ceil_div(gq.nT, kCoarseWarps * QT), gq.B * gq.H), kCoarseWarps * 32, smem, st>>>(
       gq, gk, means, scale_log2, out);
   return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
@@ -227,10 +232,11 @@ static int launch_coarse_j(const Geom& gq, const Geom& gk, const float* means, f
 template <int D>
 static int launch_coarse(const Geom& gq, const Geom& gk, const float* means, float scale_log2, float* out,
                          cudaStream_t st) {
-  if (gk.nT <= 256) return launch_coarse_j<D, 8>(gq, gk, means, scale_log2, out, st);
-  if (gk.nT <= 512) return launch_coarse_j<D, 16>(gq, gk, means, scale_log2, out, st);
-  if (gk.nT <= 768) return launch_coarse_j<D, 24>(gq, gk, means, scale_log2, out, st);
-  return launch_coarse_j<D, 48>(gq, gk, means, scale_log2, out, st);
+  if (gk.nT <= 256) return launch_coarse_j<D, 8, 4>(gq, gk, means, scale_log2, out, st);
+  if (gk.nT <= 512) return launch_coarse_j<D, 16, 4>(gq, gk, means, scale_log2, out, st);
+  if (gk.nT <= 768) return launch_coarse_j<D, 24, 4>(gq, gk, means, scale_log2, out, st);
+  if (gk.nT <= 1024) return launch_coarse_j<D, 32, 2>(gq, gk, means, scale_log2, out, st);
+  return launch_coarse_j<D, 48, 2>(gq, gk, means, scale_log2, out, st);
 }
 
 // Pooling (Q and K; with v != nullptr also V for the coarse branch), then
@@ -461,6 +467,74 @@ static int attn_fwd_impl(const vsa_shape* shape, const void* q, const void* k, c
              : dispatch_attn<false>(gq.d, mode, mq, mk, mv, a, st);
 }
 
+// ----------------------------------------------------- host-to-host forward
+// Chunks of `c` heads: [B, H, N, d] holds a head's tokens contiguously and
+// consecutive heads back to back, so a chunk is one contiguous range of
+// (b, h) pairs; in [B, N, H, d] a chunk is c heads of one batch, a strided
+// block copied with a 2-D copy into a dense [N, c, d] buffer.  Two buffer
+// sets in the caller's workspace; uploads, kernels and downloads run on
+// three streams of the library so chunk i+1's upload and chunk i-1's
+// download overlap chunk i's kernels.
+static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct HostPlan {
+  int c;                     // heads per chunk
+  size_t q, k, o, lse, idx, sel, set;   // bytes of each buffer of one set (256-aligned), and of the set
+};
+
+static HostPlan host_plan(const vsa_shape* s, const Geom& gq, const Geom& gk, int topk, int chunk_heads) {
+  HostPlan p;
+  const int maxc = s->layout == VSA_LAYOUT_BNHD ? s->H : s->B * s->H;
+  p.c = chunk_heads < 1 ? 1 : (chunk_heads > maxc ? maxc : chunk_heads);
+  const size_t Nq = static_cast<size_t>(gq.T) * gq.Hh * gq.W, Nk = static_cast<size_t>(gk.T) * gk.Hh * gk.W;
+  const size_t c = static_cast<size_t>(p.c), d = static_cast<size_t>(s->d);
+  Geom cq = gq, ck = gk;
+  cq.B = ck.B = 1;
+  cq.H = ck.H = p.c;
+  p.q = align256(c * Nq * d * 2);
+  p.k = align256(c * Nk * d * 2);
+  p.o = p.q;
+  p.lse = align256(c * Nq * 4);
+  p.idx = align256(c * static_cast<size_t>(gq.nT) * topk * 4);
+  p.sel = align256(select_workspace_bytes(cq, ck));
+  p.set = p.q + 2 * p.k + p.o + p.lse + p.idx + p.sel;
+  return p;
+}
+
+struct HostStreams {
+  cudaStream_t in, comp, out;
+  cudaEvent_t start, ev_in[2], ev_comp[2], ev_out[2], done_in, done_comp, done_out;
+  std::atomic<bool> ready{false};
+};
+
+// The three streams and their events, created once per device (the first
+// host-to-host call on a device creates them: driver objects, no device
+// memory of the caller's).
+static int host_streams(HostStreams** out, std::mutex** mu) {
+  static HostStreams hs[kMaxDevices];
+  static std::mutex mus[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VSA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return VSA_ERR_ARCH;
+  *mu = &mus[dev];
+  HostStreams& h = hs[dev];
+  if (!h.ready) {
+    std::lock_guard<std::mutex> lock(mus[dev]);
+    if (!h.ready) {
+      bool ok = cudaStreamCreateWithFlags(&h.in, cudaStreamNonBlocking) == cudaSuccess &&
+                cudaStreamCreateWithFlags(&h.comp, cudaStreamNonBlocking) == cudaSuccess &&
+                cudaStreamCreateWithFlags(&h.out, cudaStreamNonBlocking) == cudaSuccess;
+      cudaEvent_t* evs[] = {&h.start, &h.ev_in[0], &h.ev_in[1], &h.ev_comp[0], &h.ev_comp[1], &h.ev_out[0],
+                            &h.ev_out[1], &h.done_in, &h.done_comp, &h.done_out};
+      for (cudaEvent_t* e : evs) ok = ok && cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
+      if (!ok) return VSA_ERR_CUDA;
+      h.ready = true;
+    }
+  }
+  *out = &h;
+  return VSA_OK;
+}
+
 }  // namespace vsa
 
 extern "C" {
@@ -501,6 +575,130 @@ int vsa_attn_fwd_gated(const vsa_shape* shape, const void* q, const void* k, con
                        float* lse, void* stream) {
   if (coarse == nullptr || gate == nullptr) return VSA_ERR_INVALID_ARG;
   return attn_fwd_impl(shape, q, k, v, idx, topk, softmax_scale, coarse, gate, o, lse, stream);
+}
+
+size_t vsa_forward_host_workspace_bytes(const vsa_shape* shape, int32_t topk, int32_t chunk_heads) {
+  Geom gq, gk;
+  if (make_geoms(shape, &gq, &gk) != VSA_OK || topk <= 0 || topk > gk.nT) return 0;
+  return 2 * host_plan(shape, gq, gk, topk, chunk_heads).set;
+}
+
+int vsa_forward_host(const vsa_shape* shape, const void* q, const void* k, const void* v, int32_t topk,
+                     float softmax_scale, void* o, float* lse, int32_t* idx, int32_t chunk_heads, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  Geom gq, gk;
+  int rc = make_geoms(shape, &gq, &gk);
+  if (rc != VSA_OK) return rc;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr || idx == nullptr)
+    return VSA_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return VSA_ERR_INVALID_ARG;
+  if (topk <= 0 || topk > gk.nT || topk < gk.prefix) return VSA_ERR_TOPK_RANGE;
+  if (!aligned16(workspace)) return VSA_ERR_ALIGNMENT;
+  const HostPlan pl = host_plan(shape, gq, gk, topk, chunk_heads);
+  if (workspace == nullptr || workspace_bytes < 2 * pl.set) return VSA_ERR_WORKSPACE;
+  if ((rc = check_arch()) != VSA_OK) return rc;
+  HostStreams* hs = nullptr;
+  std::mutex* mu = nullptr;
+  if ((rc = host_streams(&hs, &mu)) != VSA_OK) return rc;
+  std::lock_guard<std::mutex> lock(*mu);
+  cudaStream_t caller = static_cast<cudaStream_t>(stream);
+  const bool bnhd = shape->layout == VSA_LAYOUT_BNHD;
+  const size_t Nq = static_cast<size_t>(gq.T) * gq.Hh * gq.W, Nk = static_cast<size_t>(gk.T) * gk.Hh * gk.W;
+  const size_t d = static_cast<size_t>(shape->d), es = 2;
+  const int B = shape->B, H = shape->H;
+  // chunk list: (first (b, h) pair as b * H + h, heads); in [B, N, H, d] chunks stay within a batch
+  const int per_b = bnhd ? (H + pl.c - 1) / pl.c : 0;
+  const int nchunk = bnhd ? B * per_b : (B * H + pl.c - 1) / pl.c;
+  auto ck = [&](int i, int* bh0, int* nh) {
+    if (bnhd) {
+      const int b = i / per_b, h0 = (i % per_b) * pl.c;
+      *bh0 = b * H + h0;
+      *nh = (H - h0 < pl.c) ? H - h0 : pl.c;
+    } else {
+      *bh0 = i * pl.c;
+      *nh = (B * H - *bh0 < pl.c) ? B * H - *bh0 : pl.c;
+    }
+  };
+  auto fail = [&]() { return VSA_ERR_CUDA; };
+  if (cudaEventRecord(hs->start, caller) != cudaSuccess || cudaStreamWaitEvent(hs->in, hs->start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(hs->comp, hs->start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(hs->out, hs->start, 0) != cudaSuccess)
+    return fail();
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  const unsigned char* hq = static_cast<const unsigned char*>(q);
+  const unsigned char* hk = static_cast<const unsigned char*>(k);
+  const unsigned char* hv = static_cast<const unsigned char*>(v);
+  unsigned char* ho = static_cast<unsigned char*>(o);
+  for (int i = 0; i < nchunk; ++i) {
+    const int bs = i & 1;
+    int bh0, nh;
+    ck(i, &bh0, &nh);
+    unsigned char* set = ws + bs * pl.set;
+    unsigned char *dq = set, *dk = dq + pl.q, *dv = dk + pl.k, *dob = dv + pl.k;
+    float* dl = reinterpret_cast<float*>(dob + pl.o);
+    int32_t* di = reinterpret_cast<int32_t*>(dob + pl.o + pl.lse);
+    void* dsel = dob + pl.o + pl.lse + pl.idx;
+    const size_t nhs = static_cast<size_t>(nh);
+    // uploads (after this buffer set's previous downloads)
+    if (i >= 2 && cudaStreamWaitEvent(hs->in, hs->ev_out[bs], 0) != cudaSuccess) return fail();
+    if (!bnhd) {
+      const size_t oq = static_cast<size_t>(bh0) * Nq * d * es, okv = static_cast<size_t>(bh0) * Nk * d * es;
+      if (cudaMemcpyAsync(dq, hq + oq, nhs * Nq * d * es, cudaMemcpyHostToDevice, hs->in) != cudaSuccess ||
+          cudaMemcpyAsync(dk, hk + okv, nhs * Nk * d * es, cudaMemcpyHostToDevice, hs->in) != cudaSuccess ||
+          cudaMemcpyAsync(dv, hv + okv, nhs * Nk * d * es, cudaMemcpyHostToDevice, hs->in) != cudaSuccess)
+        return fail();
+    } else {
+      const int b = bh0 / H, h0 = bh0 % H;
+      const size_t row = static_cast<size_t>(H) * d * es, w = nhs * d * es;
+      const size_t oq = (static_cast<size_t>(b) * Nq * H + h0) * d * es;
+      const size_t okv = (static_cast<size_t>(b) * Nk * H + h0) * d * es;
+      if (cudaMemcpy2DAsync(dq, w, hq + oq, row, w, Nq, cudaMemcpyHostToDevice, hs->in) != cudaSuccess ||
+          cudaMemcpy2DAsync(dk, w, hk + okv, row, w, Nk, cudaMemcpyHostToDevice, hs->in) != cudaSuccess ||
+          cudaMemcpy2DAsync(dv, w, hv + okv, row, w, Nk, cudaMemcpyHostToDevice, hs->in) != cudaSuccess)
+        return fail();
+    }
+    if (cudaEventRecord(hs->ev_in[bs], hs->in) != cudaSuccess) return fail();
+    // kernels on the chunk: the same shape with B = 1 and H = nh
+    vsa_shape cs = *shape;
+    cs.B = 1;
+    cs.H = nh;
+    Geom cq, ckv;
+    if ((rc = make_geoms(&cs, &cq, &ckv)) != VSA_OK) return rc;
+    if (cudaStreamWaitEvent(hs->comp, hs->ev_in[bs], 0) != cudaSuccess) return fail();
+    if ((rc = dispatch_select(cq, ckv, dq, dk, topk, di, dsel, hs->comp)) != VSA_OK) return rc;
+    if ((rc = attn_fwd_impl(&cs, dq, dk, dv, di, topk, softmax_scale, nullptr, nullptr, dob, dl, hs->comp)) !=
+        VSA_OK)
+      return rc;
+    if (cudaEventRecord(hs->ev_comp[bs], hs->comp) != cudaSuccess) return fail();
+    // downloads
+    if (cudaStreamWaitEvent(hs->out, hs->ev_comp[bs], 0) != cudaSuccess) return fail();
+    const size_t ol = static_cast<size_t>(bh0) * Nq * 4;
+    const size_t oi = static_cast<size_t>(bh0) * gq.nT * topk * 4;
+    if (!bnhd) {
+      if (cudaMemcpyAsync(ho + static_cast<size_t>(bh0) * Nq * d * es, dob, nhs * Nq * d * es, cudaMemcpyDeviceToHost,
+                          hs->out) != cudaSuccess)
+        return fail();
+    } else {
+      const int b = bh0 / H, h0 = bh0 % H;
+      const size_t row = static_cast<size_t>(H) * d * es, w = nhs * d * es;
+      if (cudaMemcpy2DAsync(ho + (static_cast<size_t>(b) * Nq * H + h0) * d * es, row, dob, w, w, Nq,
+                            cudaMemcpyDeviceToHost, hs->out) != cudaSuccess)
+        return fail();
+    }
+    if (cudaMemcpyAsync(reinterpret_cast<unsigned char*>(lse) + ol, dl, nhs * Nq * 4, cudaMemcpyDeviceToHost,
+                        hs->out) != cudaSuccess ||
+        cudaMemcpyAsync(reinterpret_cast<unsigned char*>(idx) + oi, di, nhs * gq.nT * topk * 4,
+                        cudaMemcpyDeviceToHost, hs->out) != cudaSuccess ||
+        cudaEventRecord(hs->ev_out[bs], hs->out) != cudaSuccess)
+      return fail();
+  }
+  // the caller's stream waits for all of it
+  if (cudaEventRecord(hs->done_in, hs->in) != cudaSuccess || cudaEventRecord(hs->done_comp, hs->comp) != cudaSuccess ||
+      cudaEventRecord(hs->done_out, hs->out) != cudaSuccess || cudaStreamWaitEvent(caller, hs->done_in, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(caller, hs->done_comp, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(caller, hs->done_out, 0) != cudaSuccess)
+    return fail();
+  return VSA_OK;
 }
 
 int vsa_device_error(uint32_t* code, int32_t reset) {

@@ -491,69 +491,137 @@ inline size_t score_narrow_smem_bytes(const Geom& gk) {
 // ------------------------------------------------------------ coarse branch
 // Tile-level attention (pooled coarse branch): for query tile i of head bh,
 // o[i] = sum_j softmax_j(scale * qbar_i . kbar_j) vbar_j over every
-// key/value tile j, from the channel-major means in the workspace.  One warp
-// per query tile: lane l holds the scores of key tiles l, l + 32, ...  (the
-// means rows are contiguous in j, so each channel's loads coalesce), the
-// softmax is a warp reduction, and each output channel is a warp sum of
-// p_j * vbar_j[c].  float32 throughout; reads the means from L2.
+// key/value tile j, from the channel-major means in the workspace.  One CTA
+// per (8 * QT query tiles, head); each warp takes QT query tiles and lane l
+// holds their scores for key tiles l, l + 32, ... (QT tiles per warp, so
+// each mean read from shared memory feeds QT FMAs: with one, the kernel ran
+// at the shared-memory bandwidth).  The key means, then the value means,
+// stream through shared memory in slices of kCoarseSlice channels on a
+// cp.async ring (kCoarseStages deep, one barrier per slice), each slice read
+// from L2 once per CTA.  The softmax is a warp reduction between the two
+// passes, and each output channel a warp sum of p_j * vbar_j[c].  float32
+// throughout.
 constexpr int kCoarseWarps = 8;
+constexpr int kCoarseSlice = 8;
+constexpr int kCoarseStages = 3;
 
-template <int D, int MAXJ>
+template <int D, int MAXJ, int QT>
 __global__ void __launch_bounds__(kCoarseWarps * 32) coarse_kernel(Geom gq, Geom gk, const float* __restrict__ means,
                                                                    float scale_log2, float* __restrict__ out) {
-  __shared__ float qs[kCoarseWarps][D];
+  constexpr int SPP = D / kCoarseSlice;            // slices per pass
+  extern __shared__ __align__(16) float csm[];
+  float* qs = csm;                                  // [kCoarseWarps * QT][D]
+  float* ring = csm + kCoarseWarps * QT * D;        // [kCoarseStages][kCoarseSlice][ldk]
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int bh = blockIdx.y;
-  const int i = blockIdx.x * kCoarseWarps + warp;
-  if (i >= gq.nT) return;
+  const int i0 = (blockIdx.x * kCoarseWarps + warp) * QT;       // the warp's first query tile
   const int nT = gk.nT, ldq = means_ld(gq.nT), ldk = means_ld(nT);
   const float* mq = means + means_offset(gq, gk, 0, bh);
   const float* mk = means + means_offset(gq, gk, 1, bh);
   const float* mv = means + means_offset(gq, gk, 2, bh);
-  for (int c = lane; c < D; c += 32) qs[warp][c] = mq[static_cast<size_t>(c) * ldq + i];
-  __syncwarp();
-  float s[MAXJ];
+  const int slice_f = kCoarseSlice * ldk;           // floats per slice
+  // slice st: K channels for st < SPP, then V channels; one cp.async group per call
+  auto issue = [&](int st) {
+    if (st < 2 * SPP) {
+      const float* m = st < SPP ? mk : mv;
+      const int c0 = (st % SPP) * kCoarseSlice;
+      float* dst = ring + (st % kCoarseStages) * slice_f;
+      for (int f = threadIdx.x; f < slice_f / 4; f += kCoarseWarps * 32) {
+        const int c = (4 * f) / ldk, j = (4 * f) % ldk;
+        cp_async16(smem_u32(dst + 4 * f), m + static_cast<size_t>(c0 + c) * ldk + j, 16u);
+      }
+    }
+    cp_async_commit();
+  };
 #pragma unroll
-  for (int t = 0; t < MAXJ; ++t) s[t] = 0.f;
-  for (int c = 0; c < D; ++c) {
-    const float qc = qs[warp][c];
-    const float* row = mk + static_cast<size_t>(c) * ldk;
+  for (int st = 0; st < kCoarseStages - 1; ++st) issue(st);
+  float* qw = qs + warp * QT * D;
 #pragma unroll
-    for (int t = 0; t < MAXJ; ++t) {
-      const int j = lane + 32 * t;
-      if (j < nT) s[t] = fmaf(qc, row[j], s[t]);
+  for (int u = 0; u < QT; ++u)
+    for (int c = lane; c < D; c += 32) qw[u * D + c] = i0 + u < gq.nT ? mq[static_cast<size_t>(c) * ldq + i0 + u] : 0.f;
+  float s[QT][MAXJ];
+#pragma unroll
+  for (int u = 0; u < QT; ++u)
+#pragma unroll
+    for (int t = 0; t < MAXJ; ++t) s[u][t] = 0.f;
+  float inv_l[QT];
+  for (int st = 0; st < 2 * SPP; ++st) {
+    cp_async_wait<kCoarseStages - 2>();
+    __syncthreads();                                // slice st visible; the slot of slice st-1 is free
+    issue(st + kCoarseStages - 1);
+    const float* sl = ring + (st % kCoarseStages) * slice_f;
+    const int c0 = (st % SPP) * kCoarseSlice;
+    if (st < SPP) {
+#pragma unroll
+      for (int c = 0; c < kCoarseSlice; ++c) {
+        float qc[QT];
+#pragma unroll
+        for (int u = 0; u < QT; ++u) qc[u] = qw[u * D + c0 + c];
+#pragma unroll
+        for (int t = 0; t < MAXJ; ++t) {
+          const int j = lane + 32 * t;
+          if (j < nT) {
+            const float kv = sl[c * ldk + j];
+#pragma unroll
+            for (int u = 0; u < QT; ++u) s[u][t] = fmaf(qc[u], kv, s[u][t]);
+          }
+        }
+      }
+      if (st == SPP - 1) {                          // scores complete: softmax weights
+#pragma unroll
+        for (int u = 0; u < QT; ++u) {
+          float mx = -INFINITY;
+#pragma unroll
+          for (int t = 0; t < MAXJ; ++t) {
+            s[u][t] = (lane + 32 * t < nT) ? s[u][t] * scale_log2 : -INFINITY;
+            mx = fmaxf(mx, s[u][t]);
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          float l = 0.f;
+#pragma unroll
+          for (int t = 0; t < MAXJ; ++t) {
+            s[u][t] = ex2_approx(s[u][t] - mx);     // 0 past the last key tile
+            l += s[u][t];
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+          inv_l[u] = 1.f / l;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < kCoarseSlice; ++c) {
+        float acc[QT];
+#pragma unroll
+        for (int u = 0; u < QT; ++u) acc[u] = 0.f;
+#pragma unroll
+        for (int t = 0; t < MAXJ; ++t) {
+          const int j = lane + 32 * t;
+          if (j < nT) {
+            const float vv = sl[c * ldk + j];
+#pragma unroll
+            for (int u = 0; u < QT; ++u) acc[u] = fmaf(s[u][t], vv, acc[u]);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < QT; ++u) {
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], o);
+          if (i0 + u < gq.nT && lane == ((c0 + c) & 31))
+            out[(static_cast<size_t>(bh) * gq.nT + i0 + u) * D + c0 + c] = acc[u] * inv_l[u];
+        }
+      }
     }
   }
-  float mx = -INFINITY;
-#pragma unroll
-  for (int t = 0; t < MAXJ; ++t) {
-    s[t] = (lane + 32 * t < nT) ? s[t] * scale_log2 : -INFINITY;
-    mx = fmaxf(mx, s[t]);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  float l = 0.f;
-#pragma unroll
-  for (int t = 0; t < MAXJ; ++t) {
-    s[t] = ex2_approx(s[t] - mx);              // 0 past the last key tile
-    l += s[t];
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-  const float inv_l = 1.f / l;
-  float* orow = out + (static_cast<size_t>(bh) * gq.nT + i) * D;
-  for (int c = 0; c < D; ++c) {
-    const float* row = mv + static_cast<size_t>(c) * ldk;
-    float acc = 0.f;
-#pragma unroll
-    for (int t = 0; t < MAXJ; ++t) {
-      const int j = lane + 32 * t;
-      if (j < nT) acc = fmaf(s[t], row[j], acc);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == (c & 31)) orow[c] = acc * inv_l;
-  }
+  cp_async_wait<0>();
+}
+
+// Key tiles per lane (MAXJ) and query tiles per warp (QT) by key tile count.
+template <int D>
+inline size_t coarse_smem_bytes(const Geom& gk, int qt) {
+  return sizeof(float) * (static_cast<size_t>(kCoarseWarps) * qt * D +
+                          static_cast<size_t>(kCoarseStages) * kCoarseSlice * means_ld(gk.nT));
 }
 
 }  // namespace vsa

@@ -250,6 +250,30 @@ int vsa_attn_fwd_gated(const vsa_shape* shape, const void* q, const void* k, con
                        const int32_t* idx, int32_t topk, float softmax_scale, const float* coarse,
                        const void* gate, void* o, float* lse, void* stream);
 
+/* Host-to-host forward (the per-call, end-to-end figure of the fastbsa page,
+ * "The number"): vsa_select + vsa_attn_fwd on Q, K, V in HOST memory, with
+ * O, LSE and idx written back to host memory.  The (batch, head) pairs go
+ * through the GPU in chunks of chunk_heads heads: while chunk i runs its
+ * kernels, chunk i+1 is uploaded and chunk i-1 downloaded (three streams
+ * of the library, created on the first call on a device; the caller's
+ * stream waits for all of it, so the host outputs are complete once the
+ * caller synchronizes that stream).  Every vsa_shape field applies; in the
+ * [B, N, H, d] layout a chunk is heads of one batch, copied as strided 2-D
+ * blocks.
+ *   q, k, v      : host Q, K, V in shape->layout and shape->dtype (pinned
+ *                  memory for the copies to overlap the kernels)
+ *   o, lse, idx  : host outputs, layouts as for vsa_attn_fwd / vsa_select
+ *   chunk_heads  : heads per chunk (clamped to [1, H] in [B, N, H, d], to
+ *                  [1, B*H] otherwise)
+ *   workspace    : device buffer of at least
+ *                  vsa_forward_host_workspace_bytes(shape, topk, chunk_heads)
+ *                  bytes, 16-byte aligned: two sets of chunk buffers
+ * A failure part-way returns VSA_ERR_CUDA with some chunks enqueued. */
+size_t vsa_forward_host_workspace_bytes(const vsa_shape* shape, int32_t topk, int32_t chunk_heads);
+int vsa_forward_host(const vsa_shape* shape, const void* q, const void* k, const void* v, int32_t topk,
+                     float softmax_scale, void* o, float* lse, int32_t* idx, int32_t chunk_heads,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
 /* Reads (and with reset != 0 clears) the kernels' device error word on the
  * current device: 0 = no error; otherwise a VSA_DEVERR_* code.  Synchronizes
  * the device.  Returns a vsa_status for the read itself. */

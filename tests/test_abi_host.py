@@ -212,3 +212,22 @@ def test_coarse_entry_points_check_arguments_before_launch():
     assert _attg(shp, gate=24) == 4
     assert _attg(shp, coarse=8200) == 4
     assert _attg(shp, topk=0) == 2
+
+
+def test_forward_host_checks_arguments_before_launch():
+    shp = api.make_shape(1, 2, (31, 22, 40), 128, (4, 8, 8))
+    L = _native.lib()
+    need = int(L.vsa_forward_host_workspace_bytes(ctypes.byref(shp), 64, 2))
+    assert need > 0 and need % 256 == 0
+    assert int(L.vsa_forward_host_workspace_bytes(ctypes.byref(shp), 121, 2)) == 0
+    args = [ctypes.byref(shp), 256, 512, 768, 64, 0.1, 1024, 2048, 4096, 2, 8192, need, None]
+    def call(**kw):
+        a = list(args)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return L.vsa_forward_host(*a)
+    assert call(a1=0) == 1                     # q
+    assert call(a5=0.0) == 1                   # scale
+    assert call(a4=0) == 2                     # topk
+    assert call(a10=8200) == 4                 # workspace alignment
+    assert call(a11=need - 1) == 5             # workspace size

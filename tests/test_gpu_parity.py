@@ -297,16 +297,30 @@ def test_full_size_sweep_all_tiles_is_dense():
         assert np.abs(lg[0, bh][rows] - Ld).max() <= gu.LSE_ABS
 
 
-@pytest.mark.parametrize("chunk", [1, 2, 5])
-def test_forward_host_matches_device_path(chunk):
-    """The pipelined host-to-host call gives the device path's bits."""
-    w = Workload("host_pipe", 2, 3, (9, 20, 20), 128, (4, 8, 8), 5)
+HOST_CASES = [
+    (Workload("host_pipe", 2, 3, (9, 20, 20), 128, (4, 8, 8), 5), 1),
+    (Workload("host_pipe", 2, 3, (9, 20, 20), 128, (4, 8, 8), 5), 2),
+    (Workload("host_pipe", 2, 3, (9, 20, 20), 128, (4, 8, 8), 5), 5),
+    # [B, N, H, d]: chunks are strided blocks of one batch's heads (3 heads in chunks of 2: a short last one)
+    (Workload("host_bnhd", 2, 3, (6, 10, 14), 128, (4, 4, 4), 5, "field", layout="bnhd"), 2),
+    # own key/value grid and tile, always-kept prefix tiles, fp16, [B, N, H, d]
+    (Workload("host_kv_prefix", 2, 2, (8, 12, 16), 64, (4, 4, 4), 12, "field", grid_k=(12, 12, 16),
+              prefix_tiles=12, layout="bnhd", dtype="f16"), 1),
+]
+
+
+@pytest.mark.parametrize("w,chunk", HOST_CASES, ids=[f"{w.name}-c{c}" for w, c in HOST_CASES])
+def test_forward_host_matches_device_path(w, chunk):
+    """vsa_forward_host (host buffers in and out) gives the device path's bits,
+    and those match the oracle."""
     (q, k, v), (qd, kd, vd) = gu.inputs(w, seed=6)
-    o_ref, l_ref, i_ref = api.forward(qd, kd, vd, w.grid, w.tile, w.topk)
+    kw = dict(grid_k=w.grid_k, tile_k=w.tile_k, layout=w.layout, prefix_tiles=w.prefix_tiles)
+    o_ref, l_ref, i_ref = api.forward(qd, kd, vd, w.grid, w.tile, w.topk, **kw)
     hq, hk, hv = (qd.cpu().pin_memory(), kd.cpu().pin_memory(), vd.cpu().pin_memory())
-    o, l, i = api.forward_host(hq, hk, hv, w.grid, w.tile, w.topk, chunk_heads=chunk)
-    torch.cuda.synchronize()
+    o, l, i = api.forward_host(hq, hk, hv, w.grid, w.tile, w.topk, chunk_heads=chunk, **kw)
     gu.assert_no_device_error()
     assert torch.equal(i, i_ref.cpu())
     assert torch.equal(o.view(torch.int16), o_ref.cpu().view(torch.int16))
     assert torch.equal(l, l_ref.cpu())
+    gu.check_selection(i.numpy(), gu.oracle_scores(q, k, w), w.topk)
+    gu.check_attention(o, l, q, k, v, w, i.numpy(), w.d ** -0.5)

@@ -1,6 +1,7 @@
 """seqpar.forward_ulysses on one GPU: a one-rank NCCL group, so both
 all-to-alls go through NCCL (as identity exchanges) around the CUDA forward;
-the result must be bit-identical to calling the forward directly."""
+the result must be bit-identical to calling the forward directly, and match
+the float64 oracle (selection and attention of every head)."""
 import os
 import socket
 
@@ -24,7 +25,7 @@ def _free_port():
 def test_one_rank_nccl_equals_direct():
     w = Workload("seqpar1", 1, 4, (8, 12, 16), 128, (4, 4, 4), 6, "field", layout="bnhd", grid_k=(12, 12, 16),
                  prefix_tiles=12)
-    (_, _, _), (qd, kd, vd) = gu.inputs(w, seed=5)
+    (q, k, v), (qd, kd, vd) = gu.inputs(w, seed=5)
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
     dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
     try:
@@ -39,3 +40,7 @@ def test_one_rank_nccl_equals_direct():
     gu.assert_no_device_error()
     assert torch.equal(idx, idx2) and torch.equal(o, o2) and torch.equal(lse, lse2)
     assert (idx[..., :w.prefix_tiles].cpu() == torch.arange(w.prefix_tiles)).all()
+    wt = w.with_(topk=topk)
+    gi = idx.cpu().numpy()
+    gu.check_selection(gi, gu.oracle_scores(q, k, wt), topk)
+    gu.check_attention(o, lse, q, k, v, wt, gi, w.d ** -0.5)
