@@ -389,7 +389,8 @@ __device__ __forceinline__ int build_union(const AttnArgs& a, const int32_t* row
 template <int D, int MODE, bool F16, bool SAME, bool BNHD>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                    const AttnArgs a) {
   constexpr bool SHARED = MODE == MODE_SHARED;
   constexpr bool PAIR = MODE == MODE_PAIR;
   constexpr int P = PAIR ? 2 : 1;                            // pieces per K/V sub-block
@@ -471,6 +472,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     *abort_flag = 0;
     fence_mbar_init();
+    // Q needs nothing of the set-up below: its load overlaps it
+    const int nbox = (PAIR && slot.has_b) ? 2 : 1;
+    mbar_arrive_expect_tx(bar(BAR_Q_FULL), static_cast<uint32_t>(nbox * L::kSlabs) * box_bytes);
+    const BoxCoord ca = box_coord_l<BNHD>(g, slot.bh, slot.t0, slot.y0, slot.x0);
+    const BoxCoord cb = box_coord_l<BNHD>(g, slot.bh, slot.tb0, slot.yb0, slot.xb0);
+    for (int sl = 0; sl < L::kSlabs; ++sl) {
+      tma_load_5d(sQ + sl * L::kSlabBytes, &tmQ, bar(BAR_Q_FULL), sl * 64, ca.c1, ca.c2, ca.c3, ca.c4);
+      if (nbox == 2)
+        tma_load_5d(sQ + sl * L::kSlabBytes + box_bytes, &tmQ, bar(BAR_Q_FULL), sl * 64, cb.c1, cb.c2, cb.c3, cb.c4);
+    }
   }
   if (!PAIR) {
     const int32_t* r0 = a.idx + (static_cast<size_t>(slot.bh) * g.nT + slot.tile) * a.topk;
@@ -497,7 +508,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tmem_relinquish();
   }
   if (warp == kWarpK && lane == 0) {
-    tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
@@ -505,30 +515,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The softmax warps alone read the sub-block table: the producers and
+  // issuers start at once, and the softmax warps meet warp 0 at named
+  // barrier 2 once it has written the table.
   if (warp == 0) build_sub_desc<MODE, SAME>(a, tile_tab, unions, PAIR ? *union_len : a.topk, sub_desc);
-  __syncthreads();
 
   if (warp >= 8) setmaxnreg_dec<RegSplit<MODE>::kProducer>();
   if (warp == kWarpK || warp == kWarpV) {
     // ====================================================== TMA producers
-    // Warp 8: Q, then K(j) into stage j & 1 once S(j-2) has released it;
+    // Warp 8: K(j) into stage j & 1 once S(j-2) has released it;
     // warp 9: V(j) once PV(j-2) has.  Separate streams, so a K load never
     // waits behind a V release.
     if (lane == 0) {
       const bool is_k = warp == kWarpK;
       bool ok = true;
-      if (is_k) {
-        const int nbox = (PAIR && slot.has_b) ? 2 : 1;
-        mbar_arrive_expect_tx(bar(BAR_Q_FULL), static_cast<uint32_t>(nbox * L::kSlabs) * box_bytes);
-        const BoxCoord ca = box_coord_l<BNHD>(g, slot.bh, slot.t0, slot.y0, slot.x0);
-        const BoxCoord cb = box_coord_l<BNHD>(g, slot.bh, slot.tb0, slot.yb0, slot.xb0);
-        for (int sl = 0; sl < L::kSlabs; ++sl) {
-          tma_load_5d(sQ + sl * L::kSlabBytes, &tmQ, bar(BAR_Q_FULL), sl * 64, ca.c1, ca.c2, ca.c3, ca.c4);
-          if (nbox == 2)
-            tma_load_5d(sQ + sl * L::kSlabBytes + box_bytes, &tmQ, bar(BAR_Q_FULL), sl * 64, cb.c1, cb.c2, cb.c3,
-                        cb.c4);
-        }
-      }
       const CUtensorMap* tm = is_k ? &tmK : &tmV;
       const uint32_t buf0 = is_k ? sK : sV;
       const int full = is_k ? BAR_K_FULL : BAR_V_FULL;
@@ -627,6 +627,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_wait(bar(BAR_DRAIN), 0, nullptr, a.err);
   } else if (warp < 8) {
     // ====================================================== softmax
+    named_bar_sync(2, 256);                           // the sub-block table is written
     setmaxnreg_inc<RegSplit<MODE>::kSoftmax>();
     const int wg = warp / 4;                          // takes the sub-blocks it with it % 2 == wg
     const int r = threadIdx.x % 128;                  // query row = TMEM lane
@@ -854,12 +855,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const float mf_use = (m_fin == -INFINITY) ? 0.f : m_fin;
     const float l_tot = (m_own == -INFINITY ? 0.f : l_own * ex2_approx((m_own) - mf_use)) +
                         (m_o == -INFINITY ? 0.f : l_o * ex2_approx(m_o - mf_use));
+    // O leaves through the Q buffer (every MMA that read Q has completed by
+    // O_FULL), in the layout the Q boxes were loaded with (128-byte swizzle:
+    // 16-byte chunk c of row r sits at chunk c ^ (r % 8)), then one TMA store
+    // per box and slab writes whole lines and drops the rows outside the grid.
+    bool staged = false;
     if (ok && __all_sync(0xffffffffu, mbar_wait(bar(BAR_O_FULL), 0, abort_flag, a.err))) {
       tc_fence_after();
       const float inv_l = 1.f / l_tot;
       const size_t N = static_cast<size_t>(g.T) * g.Hh * g.W;
       const size_t n_tok = (static_cast<size_t>(tok_t) * g.Hh + tok_y) * g.W + tok_x;
-      uint16_t* orow = a.o + token_offset(g, slot.bh, n_tok);
+      const uint32_t orow_s = sQ + static_cast<uint32_t>(r) * 128u;
 #pragma unroll
       for (int c4 = wg * (D / 64); c4 < (wg + 1) * (D / 64); ++c4) {
         uint32_t ov[32];
@@ -891,15 +897,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) pk[e] = pack_elem2<F16>(of[2 * e], of[2 * e + 1]);
-          // streaming stores: O is not read again by this kernel, so it
-          // should not sit dirty in L2 for whatever kernel runs next
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c4);
+          const uint32_t slab_row = orow_s + static_cast<uint32_t>(c4 >> 1) * L::kSlabBytes;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) __stcs(dst + e, make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]));
+          for (int e = 0; e < 4; ++e)
+            st_shared_v4(slab_row + static_cast<uint32_t>(((c4 & 1) * 4 + e) ^ (r & 7)) * 16u, pk[4 * e],
+                         pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
         }
       }
+      fence_proxy_async_smem();
+      staged = true;
       if (row_valid && wg == 0)
         __stcs(a.lse + static_cast<size_t>(slot.bh) * N + n_tok, (m_fin + log2f(l_tot)) * 0.69314718055994530942f);
+    }
+    named_bar_sync(1, 256);                           // O staged by both warpgroups
+    if (threadIdx.x == 0 && staged) {
+      const int b = slot.bh / g.H, h = slot.bh - b * g.H;
+      for (int sl = 0; sl < L::kSlabs; ++sl) {
+        // [B, N, H, d]: channel coordinate h * d + slab, batch last (the O
+        // map's dimensions); [B, H, N, d]: as the Q map
+        const int c0 = BNHD ? h * D + sl * 64 : sl * 64, c4 = BNHD ? b : slot.bh;
+        const uint32_t src = sQ + static_cast<uint32_t>(sl * L::kSlabBytes);
+        tma_store_5d(&tmO, src, c0, slot.x0, slot.y0, slot.t0, c4);
+        if (PAIR && slot.has_b) tma_store_5d(&tmO, src + box_bytes, c0, slot.xb0, slot.yb0, slot.tb0, c4);
+      }
+      bulk_commit_group();
+      bulk_wait_group_read0();
     }
   }
 

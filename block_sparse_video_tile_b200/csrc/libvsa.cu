@@ -264,8 +264,8 @@ static int launch_select(const Geom& gq, const Geom& gk, const void* q, const vo
 }
 
 template <int D, int MODE, bool F16, bool SAME, bool BNHD>
-static int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const AttnArgs& a,
-                       cudaStream_t st) {
+static int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+                       const AttnArgs& a, cudaStream_t st) {
   const int smem = AttnSmem<D>::alloc(a.gk.nT, a.topk, MODE == MODE_PAIR);
   if (cudaFuncSetAttribute(attn_fwd_kernel<D, MODE, F16, SAME, BNHD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            smem) !=
@@ -276,7 +276,7 @@ static int launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   if (MODE == MODE_SHARED) grid = BH * a.gq.nT * 2;                        // a t-half of a tile
   else if (MODE == MODE_TILE) grid = BH * a.gq.nT;                         // a tile
   else grid = BH * ((a.gq.nT + 1) / 2);                                    // a pair of tiles
-  attn_fwd_kernel<D, MODE, F16, SAME, BNHD><<<static_cast<unsigned>(grid), kAttnThreads, smem, st>>>(mq, mk, mv, a);
+  attn_fwd_kernel<D, MODE, F16, SAME, BNHD><<<static_cast<unsigned>(grid), kAttnThreads, smem, st>>>(mq, mk, mv, mo, a);
   return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 
@@ -298,29 +298,29 @@ static int select_scratch_ptr(float** out) {
 // reads one geometry; see kv_geom).
 template <bool F16, bool SAME, bool BNHD>
 static int dispatch_attn_d(int d, int mode, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                           const AttnArgs& a, cudaStream_t st) {
+                           const CUtensorMap& mo, const AttnArgs& a, cudaStream_t st) {
   if (d == 128) {
-    if (mode == MODE_SHARED) return launch_attn<128, MODE_SHARED, F16, SAME, BNHD>(mq, mk, mv, a, st);
-    if (mode == MODE_TILE) return launch_attn<128, MODE_TILE, F16, SAME, BNHD>(mq, mk, mv, a, st);
-    return launch_attn<128, MODE_PAIR, F16, SAME, BNHD>(mq, mk, mv, a, st);
+    if (mode == MODE_SHARED) return launch_attn<128, MODE_SHARED, F16, SAME, BNHD>(mq, mk, mv, mo, a, st);
+    if (mode == MODE_TILE) return launch_attn<128, MODE_TILE, F16, SAME, BNHD>(mq, mk, mv, mo, a, st);
+    return launch_attn<128, MODE_PAIR, F16, SAME, BNHD>(mq, mk, mv, mo, a, st);
   }
-  if (mode == MODE_SHARED) return launch_attn<64, MODE_SHARED, F16, SAME, BNHD>(mq, mk, mv, a, st);
-  if (mode == MODE_TILE) return launch_attn<64, MODE_TILE, F16, SAME, BNHD>(mq, mk, mv, a, st);
-  return launch_attn<64, MODE_PAIR, F16, SAME, BNHD>(mq, mk, mv, a, st);
+  if (mode == MODE_SHARED) return launch_attn<64, MODE_SHARED, F16, SAME, BNHD>(mq, mk, mv, mo, a, st);
+  if (mode == MODE_TILE) return launch_attn<64, MODE_TILE, F16, SAME, BNHD>(mq, mk, mv, mo, a, st);
+  return launch_attn<64, MODE_PAIR, F16, SAME, BNHD>(mq, mk, mv, mo, a, st);
 }
 
 template <bool F16>
 static int dispatch_attn(int d, int mode, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                         const AttnArgs& a, cudaStream_t st) {
+                         const CUtensorMap& mo, const AttnArgs& a, cudaStream_t st) {
   const bool same = a.gq.T == a.gk.T && a.gq.Hh == a.gk.Hh && a.gq.W == a.gk.W && a.gq.tt == a.gk.tt &&
                     a.gq.th == a.gk.th && a.gq.tw == a.gk.tw;
   // the layout is a template parameter too: the producer's box coordinates
   // of the default layout then need no division (measured ~8% at 64-token tiles)
   if (a.gq.layout == VSA_LAYOUT_BNHD)
-    return same ? dispatch_attn_d<F16, true, true>(d, mode, mq, mk, mv, a, st)
-                : dispatch_attn_d<F16, false, true>(d, mode, mq, mk, mv, a, st);
-  return same ? dispatch_attn_d<F16, true, false>(d, mode, mq, mk, mv, a, st)
-              : dispatch_attn_d<F16, false, false>(d, mode, mq, mk, mv, a, st);
+    return same ? dispatch_attn_d<F16, true, true>(d, mode, mq, mk, mv, mo, a, st)
+                : dispatch_attn_d<F16, false, true>(d, mode, mq, mk, mv, mo, a, st);
+  return same ? dispatch_attn_d<F16, true, false>(d, mode, mq, mk, mv, mo, a, st)
+              : dispatch_attn_d<F16, false, false>(d, mode, mq, mk, mv, mo, a, st);
 }
 
 static int dispatch_select(const Geom& gq, const Geom& gk, const void* q, const void* k, int topk, int32_t* idx,
@@ -456,15 +456,16 @@ static int attn_fwd_impl(const vsa_shape* shape, const void* q, const void* k, c
   a.gate = static_cast<const uint16_t*>(gate);
   a.coarse = coarse;
   if (a.err == nullptr) return VSA_ERR_CUDA;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   const bool f16 = gq.f16 != 0;
   if ((rc = encode_qkv_map(&mq, q, gq, a.box_tq, f16)) != VSA_OK ||
       (rc = encode_qkv_map(&mk, k, gk, a.box_tk, f16)) != VSA_OK ||
-      (rc = encode_qkv_map(&mv, v, gk, a.box_tk, f16)) != VSA_OK)
+      (rc = encode_qkv_map(&mv, v, gk, a.box_tk, f16)) != VSA_OK ||
+      (rc = encode_o_map(&mo, o, gq, a.box_tq, f16)) != VSA_OK)
     return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return f16 ? dispatch_attn<true>(gq.d, mode, mq, mk, mv, a, st)
-             : dispatch_attn<false>(gq.d, mode, mq, mk, mv, a, st);
+  return f16 ? dispatch_attn<true>(gq.d, mode, mq, mk, mv, mo, a, st)
+             : dispatch_attn<false>(gq.d, mode, mq, mk, mv, mo, a, st);
 }
 
 // ----------------------------------------------------- host-to-host forward

@@ -70,4 +70,29 @@ inline int encode_qkv_map(CUtensorMap* m, const void* ptr, const Geom& g, int bo
   return r == CUDA_SUCCESS ? VSA_OK : VSA_ERR_CUDA;
 }
 
+// The output map: the query side's boxes, with dimensions that keep every
+// box inside its own batch, so that a store clips the rows outside the grid.
+// [B, H, N, d] as the Q map (T is a dimension of its own); [B, N, H, d]:
+// (H * d channels, W, Hh, T, B) -- a head's d channels are contiguous and the
+// heads of a token follow each other, so the box's channel coordinate is
+// h * d + c.
+inline int encode_o_map(CUtensorMap* m, void* ptr, const Geom& g, int box_t, bool f16 = false) {
+  if (g.layout != 1) return encode_qkv_map(m, ptr, g, box_t, f16);
+  EncodeTiledFn fn = get_encode_fn();
+  if (fn == nullptr) return VSA_ERR_CUDA;
+  const cuuint64_t e = 2;
+  const cuuint64_t d = static_cast<cuuint64_t>(g.d), W = static_cast<cuuint64_t>(g.W),
+                   Hh = static_cast<cuuint64_t>(g.Hh), T = static_cast<cuuint64_t>(g.T),
+                   B = static_cast<cuuint64_t>(g.B), H = static_cast<cuuint64_t>(g.H);
+  cuuint64_t dims[5] = {H * d, W, Hh, T, B};
+  cuuint64_t strides[4] = {e * d * H, e * d * H * W, e * d * H * W * Hh, e * d * H * W * Hh * T};
+  cuuint32_t box[5] = {64u, static_cast<cuuint32_t>(g.tw), static_cast<cuuint32_t>(g.th),
+                       static_cast<cuuint32_t>(box_t), 1u};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, ptr, dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? VSA_OK : VSA_ERR_CUDA;
+}
+
 }  // namespace vsa
