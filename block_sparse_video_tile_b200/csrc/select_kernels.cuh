@@ -63,15 +63,26 @@ constexpr uint32_t kKeepKey = 0xffffffffu;
 
 // Exact top-k of one row of order keys by one warp, keys held in registers
 // (lane l holds tiles l, l + 32, ...).  The topk-th largest key T is found
-// bit by bit from the top: T keeps a bit when at least topk keys are >= T
-// with that bit set (a warp-wide count per bit, no shared-memory atomics).
-// Bits on which all keys agree are decided without counting, and the search
-// stops once exactly topk keys are >= T.  Every key above T is taken, then
-// the keys equal to T in ascending tile order until topk are taken (ties go
-// to the lower tile index); indices are written in ascending order.  Order
+// from the top bit down.  Bits on which all keys agree are decided without
+// counting.  With a scratch histogram (256 words of shared memory for the
+// warp), 8 bits at a time are decided by a pass over the candidates (the
+// keys sharing T's decided bits, at first all): each adds one to the bin of
+// its next 8-bit digit (shared-memory atomics), a warp scan of the bins from
+// the top finds the digit d of the topk-th key and adds the candidates of
+// higher bins to `above`; d's bin holds the next candidates.  Passes repeat
+// (at most three) while more than 128 candidates remain; when d's bin holds
+// exactly the keys still missing, T is decided, else the candidates (at most
+// 128, else all keys) are gathered into four registers per lane and the
+// remaining bits are decided one by one on them: T keeps a bit when at least
+// topk keys are >= T with that bit set (above + a warp-wide count over the
+// gathered keys).  The
+// search stops once exactly topk keys are >= T.  Every key above T is taken,
+// then the keys equal to T in ascending tile order until topk are taken (ties
+// go to the lower tile index); indices are written in ascending order.  Order
 // keys of finite scores are never 0, so 0 marks padding slots.
 template <int MAXE>
-__device__ __forceinline__ void bsearch_topk_row(const uint32_t* kr, int nT, int topk, int32_t* out) {
+__device__ __forceinline__ void bsearch_topk_row(const uint32_t* kr, int nT, int topk, int32_t* out,
+                                                 uint32_t* hist = nullptr) {
   const int lane = threadIdx.x % 32;
   const uint32_t lt_mask = (1u << lane) - 1u;
   uint32_t key[MAXE];
@@ -89,16 +100,97 @@ __device__ __forceinline__ void bsearch_topk_row(const uint32_t* kr, int nT, int
   kor = __reduce_or_sync(0xffffffffu, kor);
   const int common = __clz(kand ^ kor);          // leading bits shared by all keys (32: all equal)
   uint32_t T = common == 0 ? 0u : (kand & (0xffffffffu << (32 - common)));
-  for (int b = 31 - common; b >= 0; --b) {
-    const uint32_t cand = T | (1u << b);
-    uint32_t p[4] = {0u, 0u, 0u, 0u};            // four independent chains of adds
+  int b_next = 31 - common;                      // highest undecided bit
+  bool gathered = false, done = false;
+  uint32_t above = 0u;                           // keys above the candidates (the bins passed over)
+  uint32_t g[4] = {0u, 0u, 0u, 0u};             // the gathered candidates, lane l: l, l + 32, ...
+  if (hist != nullptr) {
+    uint32_t ncand = static_cast<uint32_t>(nT); // keys sharing T's decided bits
+    for (int pass = 0; pass < 3 && !done && b_next >= 7 && ncand > 128u; ++pass) {
+      const int sh = b_next - 7;                 // digit = bits b_next .. sh
+      const uint32_t hi = b_next == 31 ? 0u : (0xffffffffu << (b_next + 1));   // decided bits
+      for (int i = lane; i < 256; i += 32) hist[i] = 0u;
+      __syncwarp();
 #pragma unroll
-    for (int e = 0; e < MAXE; ++e) p[e & 3] += (key[e] >= cand) ? 1u : 0u;
-    const uint32_t c = __reduce_add_sync(0xffffffffu, (p[0] + p[1]) + (p[2] + p[3]));
-    if (c >= static_cast<uint32_t>(topk)) {
-      T = cand;
-      // exactly topk keys are >= T: they are the answer whatever the lower bits
-      if (c == static_cast<uint32_t>(topk)) break;
+      for (int e = 0; e < MAXE; ++e)
+        if (lane + 32 * e < nT && (key[e] & hi) == (T & hi)) atomicAdd(hist + ((key[e] >> sh) & 255u), 1u);
+      __syncwarp();
+      // lane l holds bins 255 - 8l .. 248 - 8l; candidates in higher bins by a scan
+      const uint4 ha = *reinterpret_cast<const uint4*>(hist + 248 - 8 * lane);
+      const uint4 hb = *reinterpret_cast<const uint4*>(hist + 252 - 8 * lane);
+      const uint32_t h[8] = {hb.w, hb.z, hb.y, hb.x, ha.w, ha.z, ha.y, ha.x};   // bins 255-8l downwards
+      uint32_t own = 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) own += h[i];
+      uint32_t incl = own;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const uint32_t need = static_cast<uint32_t>(topk) - above;
+      uint32_t run = incl - own;                 // candidates in bins above this lane's
+      int dig = -1;
+      uint32_t abv = 0u, cnt_d = 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (dig < 0 && run + h[i] >= need) {
+          dig = 255 - 8 * lane - i;
+          abv = run;
+          cnt_d = h[i];
+        }
+        run += h[i];
+      }
+      const uint32_t who = __ballot_sync(0xffffffffu, dig >= 0);
+      const int src = __ffs(who) - 1;            // the lowest lane holds the highest qualifying bin
+      dig = __shfl_sync(0xffffffffu, dig, src);
+      above += __shfl_sync(0xffffffffu, abv, src);
+      ncand = __shfl_sync(0xffffffffu, cnt_d, src);
+      T |= static_cast<uint32_t>(dig) << sh;
+      b_next = sh - 1;
+      // every candidate of bin d is in: T (low bits 0) decides
+      if (above + ncand == static_cast<uint32_t>(topk)) done = true;
+      __syncwarp();                              // every lane has read the bins
+    }
+    if (!done && ncand <= 128u) {
+      // gather the candidates (keys sharing T's decided bits) into registers
+      const uint32_t hi = b_next >= 31 ? 0u : (0xffffffffu << (b_next + 1));
+      const uint32_t lt_m = (1u << lane) - 1u;
+      uint32_t base = 0u;
+#pragma unroll
+      for (int e = 0; e < MAXE; ++e) {
+        const bool in = lane + 32 * e < nT && (key[e] & hi) == (T & hi);
+        const uint32_t m = __ballot_sync(0xffffffffu, in);
+        if (in) hist[base + __popc(m & lt_m)] = key[e];
+        base += __popc(m);
+      }
+      __syncwarp();
+#pragma unroll
+      for (int m = 0; m < 4; ++m) g[m] = lane + 32 * m < static_cast<int>(ncand) ? hist[lane + 32 * m] : 0u;
+      gathered = true;
+    } else {
+      above = 0u;                                // count over all keys below
+    }
+    __syncwarp();                                // the scratch is reused by the warp's next row
+  }
+  if (!done) {
+    for (int b = b_next; b >= 0; --b) {
+      const uint32_t cand = T | (1u << b);
+      uint32_t c;
+      if (gathered) {
+        c = above + __reduce_add_sync(0xffffffffu, ((g[0] >= cand ? 1u : 0u) + (g[1] >= cand ? 1u : 0u)) +
+                                                       ((g[2] >= cand ? 1u : 0u) + (g[3] >= cand ? 1u : 0u)));
+      } else {
+        uint32_t p[4] = {0u, 0u, 0u, 0u};        // four independent chains of adds
+#pragma unroll
+        for (int e = 0; e < MAXE; ++e) p[e & 3] += (key[e] >= cand) ? 1u : 0u;
+        c = __reduce_add_sync(0xffffffffu, (p[0] + p[1]) + (p[2] + p[3]));
+      }
+      if (c >= static_cast<uint32_t>(topk)) {
+        T = cand;
+        // exactly topk keys are >= T: they are the answer whatever the lower bits
+        if (c == static_cast<uint32_t>(topk)) break;
+      }
     }
   }
   uint32_t gt = 0;
@@ -220,23 +312,25 @@ inline size_t pool_smem_bytes(const Geom& g) {
 // 8 x 8 block of the wide kernel balances the two (4 x 4 would run at half
 // the FMA rate).
 
-// One warp per row picks each row's top-k from the order keys in shared memory.
+// One warp per row picks each row's top-k from the order keys in shared memory;
+// `scratch` (16-byte aligned, 256 words per warp) holds each warp's histogram.
 __device__ __forceinline__ void topk_rows(const uint32_t* keys, int kst, int nT, int nrows, int topk,
-                                          int32_t* out_rows, int warps) {
+                                          int32_t* out_rows, int warps, uint32_t* scratch) {
   const int warp = threadIdx.x / 32;
+  uint32_t* hist = scratch + 256 * warp;
   for (int r = warp; r < nrows; r += warps) {
     const uint32_t* kr = keys + r * kst;
     int32_t* out = out_rows + static_cast<size_t>(r) * topk;
     if (nT <= 32 * 8)
-      bsearch_topk_row<8>(kr, nT, topk, out);
+      bsearch_topk_row<8>(kr, nT, topk, out, hist);
     else if (nT <= 32 * 12)
-      bsearch_topk_row<12>(kr, nT, topk, out);
+      bsearch_topk_row<12>(kr, nT, topk, out, hist);
     else if (nT <= 32 * 16)
-      bsearch_topk_row<16>(kr, nT, topk, out);
+      bsearch_topk_row<16>(kr, nT, topk, out, hist);
     else if (nT <= 32 * 24)
-      bsearch_topk_row<24>(kr, nT, topk, out);
+      bsearch_topk_row<24>(kr, nT, topk, out, hist);
     else
-      bsearch_topk_row<48>(kr, nT, topk, out);
+      bsearch_topk_row<48>(kr, nT, topk, out, hist);
   }
 }
 
@@ -362,7 +456,9 @@ __global__ void __launch_bounds__(kWideThreads, 1) score_topk_kernel(Geom gq, Ge
   }
   cp_async_wait<0>();
   __syncthreads();
-  topk_rows(keys, nT, nT, nrows, topk, idx + (static_cast<size_t>(bh) * gq.nT + row0) * topk, kWideThreads / 32);
+  // (the ring is free now: it holds the warps' histograms)
+  topk_rows(keys, nT, nT, nrows, topk, idx + (static_cast<size_t>(bh) * gq.nT + row0) * topk, kWideThreads / 32,
+            reinterpret_cast<uint32_t*>(ring));
 }
 
 template <int D, int STAGES, int KEYS>
@@ -479,7 +575,8 @@ __global__ void __launch_bounds__(kNarrowThreads) score_topk_narrow_kernel(Geom 
   }
   cp_async_wait<0>();
   __syncthreads();
-  topk_rows(keys, nT, nT, nrows, topk, idx + (static_cast<size_t>(bh) * gq.nT + row0) * topk, kNarrowThreads / 32);
+  topk_rows(keys, nT, nT, nrows, topk, idx + (static_cast<size_t>(bh) * gq.nT + row0) * topk, kNarrowThreads / 32,
+            reinterpret_cast<uint32_t*>(ring));
 }
 
 template <int D, int KEYS, int STAGES>
