@@ -367,7 +367,8 @@ def run_ours(args, w, rank, world, device):
     # also holds the host's launch latency while the device waits for it; the
     # whole-step figure above counts everything)
     sel_ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
-    att_ms = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
+    att_steps = [e[1].elapsed_time(e[2]) for e in evs]
+    att_ms = statistics.median(att_steps)
 
     # end to end through the C ABI's host-to-host call (vsa_forward_host, via
     # api.forward_host): the timed region holds the uploads of Q, K, V from
@@ -447,6 +448,9 @@ def run_ours(args, w, rank, world, device):
                    "inputs": ("structured field + noise (torch, on device)" if w.kind == "field"
                               else "N(0,1) (torch, on device)") + f", rounded to {w.dtype}"},
         "select_ms": sel_ms, "attend_ms": att_ms,
+        # per-step spread: on this part a sustained load settles ~50-100 ms in,
+        # ~12 % slower than the first steps (not a clock the sampler reports)
+        "attend_ms_steps": {"min": min(att_steps), "median": att_ms, "max": max(att_steps)},
         "attend_tflops_exact": att_tflops,
         "attend_tflops_nominal": nominal_flops(w) / (att_ms * 1e-3) / 1e12,
         "exact_flops_per_step": flops, "nominal_flops_per_step": nominal_flops(w),
