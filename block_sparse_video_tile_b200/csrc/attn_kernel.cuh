@@ -24,10 +24,11 @@
 // on the slot's 128 rows (thread = query row = TMEM lane), warpgroup w taking
 // the sub-blocks it with it % 2 == w, so two warps per SM sub-partition hide
 // each other's latencies and each has two sub-block periods for its work;
-// warp 8 loads Q and the K stream by TMA, warp 9 the V stream (and in
-// MODE_PAIR first builds the union list), warp 10 issues the PV MMAs and
-// warp 11 the score MMAs (tcgen05.mma kind::f16, float32 accumulation); the
-// third warpgroup gives registers to the softmax (setmaxnreg).
+// thread 0 issues Q's TMA load as soon as the barriers exist (it overlaps the
+// rest of the set-up), warp 8 loads the K stream by TMA, warp 9 the V stream
+// (and in MODE_PAIR first builds the union list), warp 10 issues the PV MMAs
+// and warp 11 the score MMAs (tcgen05.mma kind::f16, float32 accumulation);
+// the third warpgroup gives registers to the softmax (setmaxnreg).
 // TMEM (512 columns): three score buffers of 128 columns and O at 384.  The
 // scores of sub-block it go to buffer it % 3 and the softmax writes P (16-bit
 // pairs, 64 columns) over them; PV(it) reads P from there, and S(it+3) goes
@@ -47,6 +48,10 @@
 // sub-block before from shared memory (M_READY), settles its own and passes
 // it on; when the other warpgroup moved the reference meanwhile (rare), it
 // rescales the P it already stored.
+// Epilogue: O / l (plus the gated coarse term) in the input type is staged in
+// the Q buffer, swizzled as the Q boxes arrived, and written by one TMA store
+// per box and slab; the output map keeps every box inside its batch, so the
+// stores drop the rows past the grid edge.  LSE goes out by plain stores.
 #pragma once
 
 #include <cuda.h>
