@@ -412,11 +412,14 @@ __global__ void __launch_bounds__(kWideThreads, 1) score_topk_kernel(Geom gq, Ge
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int qg = lane / 8, kg = lane % 8;
-  float acc[8][8];
+  // acc2[i][p] holds the scores of query tile i with key tiles 2p, 2p + 1 of
+  // the block: packed fma.rn.f32x2, each lane the same fused multiply-add in
+  // the same channel order as a scalar one
+  uint64_t acc2[8][4];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    for (int p = 0; p < 4; ++p) acc2[i][p] = 0ull;
 
   for (int st = 0; st < nstage; ++st) {
     cp_async_wait<STAGES - 2>();
@@ -434,11 +437,13 @@ __global__ void __launch_bounds__(kWideThreads, 1) score_topk_kernel(Geom gq, Ge
         const float4 k0 = *reinterpret_cast<const float4*>(kb + c * KEYS);
         const float4 k1 = *reinterpret_cast<const float4*>(kb + c * KEYS + 32);
         const float qa[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-        const float ka[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+        const uint64_t kp[4] = {f2_pack(k0.x, k0.y), f2_pack(k0.z, k0.w), f2_pack(k1.x, k1.y), f2_pack(k1.z, k1.w)};
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 8; ++i) {
+          const uint64_t qq = f2_pack(qa[i], qa[i]);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(qa[i], ka[j], acc[i][j]);
+          for (int p = 0; p < 4; ++p) acc2[i][p] = f2_fma(qq, kp[p], acc2[i][p]);
+        }
       }
     }
     if (sl == SPP - 1 && warp < MW) {   // end of a pass: scores -> order keys
@@ -446,10 +451,16 @@ __global__ void __launch_bounds__(kWideThreads, 1) score_topk_kernel(Geom gq, Ge
       for (int i = 0; i < 8; ++i) {
         const int row = (i < 4 ? 0 : 16) + 4 * qg + (i & 3);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int key = kw0 + (j < 4 ? 0 : 32) + 4 * kg + (j & 3);
-          if (row < nrows && key < nT) keys[row * nT + key] = key < gk.prefix ? kKeepKey : order_key(acc[i][j] + 0.f);
-          acc[i][j] = 0.f;
+        for (int p = 0; p < 4; ++p) {
+          float sc[2];
+          f2_unpack(acc2[i][p], sc[0], sc[1]);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int j = 2 * p + h;
+            const int key = kw0 + (j < 4 ? 0 : 32) + 4 * kg + (j & 3);
+            if (row < nrows && key < nT) keys[row * nT + key] = key < gk.prefix ? kKeepKey : order_key(sc[h] + 0.f);
+          }
+          acc2[i][p] = 0ull;
         }
       }
     }
